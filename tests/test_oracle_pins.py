@@ -1,0 +1,348 @@
+"""Pins for the CPU oracle (no GPU): the oracle is checked against closed forms,
+special cases that reduce to independent library routines, brute force on tiny
+inputs, invariants of the method and hand-derived worked examples, so that a
+dropped term, a wrong sign or index or a transposed operand fails a test.
+
+Method source: "Joint Subspace Sparse Attention for Efficient Long-Context
+Decoding" (arXiv 2610.19026v1) — Figure 1, §2.1 (FASA = restricted orthonormal
+projection), §3.1-§3.4, §4.5 (full-KV baseline), §A.3, §E.3.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests._util import u16, f32
+from token_level_sparse_jssa_b200 import synth
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16_bits_of(x: np.ndarray) -> np.ndarray:
+    return u16(torch.from_numpy(np.asarray(x, np.float32)).to(torch.bfloat16))
+
+
+def _rand_bf16(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return u16((torch.randn(*shape, generator=g) * scale).to(torch.bfloat16))
+
+
+# ----------------------------------------------------------------------------- bf16
+def test_bf16_round_matches_torch_cast_on_fp32_values():
+    g = torch.Generator().manual_seed(1)
+    x = torch.randn(200000, generator=g) * torch.exp2(torch.randint(-140, 120, (200000,), generator=g).float())
+    x = x.to(torch.float32)
+    ours = oracle.bf16_round(x.double().numpy())
+    ref = u16(x.to(torch.bfloat16))
+    np.testing.assert_array_equal(ours, ref)
+
+
+def test_bf16_round_hand_cases():
+    d = json.load(open(os.path.join(GOLD, "projection_small.json")))["rounding_cases"]
+    got = [oracle.bf16_round_scalar(x) for x in d["x"]]
+    assert got == d["bits"]
+
+
+def test_bf16_decode_is_exact_inverse():
+    bits = np.arange(0, 65536, dtype=np.uint32).astype(np.uint16)
+    vals = oracle.bf16_to_f64(bits)
+    finite = np.isfinite(vals)
+    back = oracle.bf16_round(vals[finite])
+    # every finite pattern round-trips, except that -0 keeps its sign bit
+    np.testing.assert_array_equal(back, bits[finite])
+
+
+# ----------------------------------------------------------------------------- projection
+def test_projection_identity_basis_is_exact():
+    K = _rand_bf16((300, 64), 2, scale=3.0)
+    P = np.eye(64, dtype=np.float32)
+    Kp, ex = oracle.project_rows(K, P)
+    np.testing.assert_array_equal(Kp, K)
+
+
+def test_projection_column_selector_is_channel_subset():
+    # §2.1: keeping r original channels is a restricted orthonormal projection (FASA).
+    K = _rand_bf16((257, 128), 3)
+    cols = [5, 0, 77, 127, 64, 33, 2, 100]
+    P = np.zeros((128, len(cols)), np.float32)
+    for j, c in enumerate(cols):
+        P[c, j] = 1.0
+    Kp, _ = oracle.project_rows(K, P)
+    np.testing.assert_array_equal(Kp, K[:, cols])
+
+
+def test_projection_matches_numpy_matmul_and_rounds_once():
+    K = _rand_bf16((500, 128), 4)
+    P = synth.orthonormal_basis(128, 32, seed=9).numpy()
+    Kp, ex = oracle.project_rows(K, P)
+    ref = oracle.bf16_to_f64(K) @ P.astype(np.float64)
+    np.testing.assert_allclose(ex, ref, rtol=0, atol=1e-12)
+    # rounding the exact product once gives the stored cache
+    np.testing.assert_array_equal(Kp, oracle.bf16_round(ref))
+
+
+def test_projection_golden():
+    d = json.load(open(os.path.join(GOLD, "projection_small.json")))
+    K = _bf16_bits_of(np.array(d["K"]))
+    P = np.array(d["P"], np.float32)
+    Kp, ex = oracle.project_rows(K, P)
+    np.testing.assert_array_equal(ex, np.array(d["Kp_exact"]))
+    np.testing.assert_array_equal(Kp, np.array(d["Kp_bf16_bits"], np.uint16).reshape(Kp.shape))
+    Q = _bf16_bits_of(np.array(d["Q"]))
+    qs = oracle.query_proj(Q, P)
+    np.testing.assert_array_equal(qs, np.array(d["qs"]))
+    np.testing.assert_array_equal(oracle.scores(qs, Kp), np.array(d["scores"]))
+
+
+# ----------------------------------------------------------------------------- query projection / scores
+def test_query_projection_is_a_sum_over_the_group():
+    # G copies of one head give G times the single-head projection (sum, not mean).
+    q = _rand_bf16((1, 128), 5)
+    P = synth.orthonormal_basis(128, 16, seed=3).numpy()
+    one = oracle.query_proj(q, P)
+    four = oracle.query_proj(np.repeat(q, 4, axis=0), P)
+    np.testing.assert_allclose(four, 4 * one, rtol=1e-15, atol=0)
+    ref = P.astype(np.float64).T @ oracle.bf16_to_f64(q[0])
+    np.testing.assert_allclose(one, ref, rtol=0, atol=1e-14)
+
+
+def test_query_projection_transposition_is_pinned():
+    # A non-square, non-symmetric P: using P instead of P^T would not even type-check,
+    # and swapping the roles of rows/columns changes every value.
+    q = _rand_bf16((3, 6), 6)
+    P = np.arange(12, dtype=np.float32).reshape(6, 2) / 7.0
+    qs = oracle.query_proj(q, P)
+    ref = (oracle.bf16_to_f64(q).sum(0)) @ P.astype(np.float64)
+    np.testing.assert_allclose(qs, ref, rtol=1e-14)
+
+
+def test_scores_identity_basis_equal_full_dot_products():
+    G, d, T = 4, 64, 200
+    Q = _rand_bf16((G, d), 7)
+    K = _rand_bf16((T, d), 8)
+    P = np.eye(d, dtype=np.float32)
+    Kp, _ = oracle.project_rows(K, P)
+    s = oracle.scores(oracle.query_proj(Q, P), Kp)
+    ref = oracle.bf16_to_f64(K) @ oracle.bf16_to_f64(Q).sum(0)
+    np.testing.assert_allclose(s, ref, rtol=1e-13, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------- top-k
+def test_topk_golden_cases():
+    d = json.load(open(os.path.join(GOLD, "topk_ties.json")))
+    for c in d["cases"]:
+        idx, k_eff = oracle.topk(np.array(c["scores"], np.float64), c["k"])
+        assert k_eff == c["k_eff"], c
+        assert idx.tolist() == c["idx"], c
+
+
+def _pairwise_valid(s, sel_set):
+    # every selected token beats every unselected one: larger score, or equal score and lower index
+    for i in sel_set:
+        for j in range(len(s)):
+            if j in sel_set:
+                continue
+            if not (s[i] > s[j] or (s[i] == s[j] and i < j)):
+                return False
+    return True
+
+
+@pytest.mark.parametrize("seed", range(25))
+def test_topk_pairwise_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    n = int(rng.integers(1, 65))
+    k = int(rng.integers(1, n + 3))
+    # few distinct values to force many ties
+    s = rng.integers(-4, 5, size=n).astype(np.float64) * 0.5
+    idx, k_eff = oracle.topk(s, k)
+    assert k_eff == min(k, n)
+    sel = [int(i) for i in idx[:k_eff]]
+    assert sel == sorted(sel) and len(set(sel)) == k_eff
+    assert all(i == -1 for i in idx[k_eff:])
+    assert _pairwise_valid(s, set(sel))
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_topk_exhaustive_subset_maximisation(seed):
+    rng = np.random.default_rng(100 + seed)
+    n = int(rng.integers(2, 13))
+    k = int(rng.integers(1, n + 1))
+    s = rng.integers(-3, 4, size=n).astype(np.float64)
+    best = None
+    for comb in itertools.combinations(range(n), k):
+        key = (sum(s[list(comb)]), tuple(-c for c in comb))  # max sum, then lexicographically lowest
+        if best is None or key > best[0]:
+            best = (key, comb)
+    idx, _ = oracle.topk(s, k)
+    assert tuple(idx.tolist()) == best[1]
+
+
+def test_topk_matches_numpy_lexsort():
+    rng = np.random.default_rng(7)
+    s = np.round(rng.standard_normal(5000), 2)    # many exact ties
+    order = np.lexsort((np.arange(s.size), -s))   # primary: score desc, secondary: index asc
+    idx, _ = oracle.topk(s, 300)
+    np.testing.assert_array_equal(idx, np.sort(order[:300]))
+
+
+def test_topk_permutation_invariance():
+    rng = np.random.default_rng(3)
+    s = rng.standard_normal(1000)                  # distinct values
+    perm = rng.permutation(1000)
+    idx, _ = oracle.topk(s, 50)
+    idx_p, _ = oracle.topk(s[perm], 50)
+    assert set(perm[idx_p].tolist()) == set(idx.tolist())
+
+
+# ----------------------------------------------------------------------------- attention
+def _torch_attention(Q, K, V, tokens, scale):
+    q = torch.from_numpy(oracle.bf16_to_f64(Q))
+    k = torch.from_numpy(oracle.bf16_to_f64(K))[tokens]
+    v = torch.from_numpy(oracle.bf16_to_f64(V))[tokens]
+    logits = scale * q @ k.T
+    return (torch.softmax(logits, dim=-1) @ v).numpy(), torch.logsumexp(logits, dim=-1).numpy()
+
+
+def test_attention_golden_two_tokens():
+    d = json.load(open(os.path.join(GOLD, "attention_two_tokens.json")))
+    Q, K, V = (_bf16_bits_of(np.array(d[x])) for x in ("Q", "K", "V"))
+    O, lse = oracle.attention(Q, K, V, d["tokens"], d["scale"])
+    np.testing.assert_allclose(O, np.array(d["O"]), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse, np.array(d["lse"]), rtol=0, atol=1e-15)
+
+
+def test_attention_matches_torch_softmax_on_all_tokens():
+    G, dk, dv, T = 4, 128, 96, 300
+    Q, K, V = _rand_bf16((G, dk), 11, 0.2), _rand_bf16((T, dk), 12), _rand_bf16((T, dv), 13)
+    tokens = np.arange(T)
+    O, lse = oracle.attention(Q, K, V, tokens, 1 / math.sqrt(dk))
+    Or, lr = _torch_attention(Q, K, V, tokens, 1 / math.sqrt(dk))
+    np.testing.assert_allclose(O, Or, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, lr, rtol=0, atol=1e-12)
+
+
+def test_attention_single_token_returns_its_value_row():
+    Q, K, V = _rand_bf16((3, 64), 14), _rand_bf16((50, 64), 15), _rand_bf16((50, 64), 16)
+    O, _ = oracle.attention(Q, K, V, [37], 0.125)
+    np.testing.assert_array_equal(O, np.repeat(oracle.bf16_to_f64(V[37:38]), 3, axis=0))
+
+
+def test_attention_zero_query_is_value_mean():
+    K, V = _rand_bf16((40, 32), 17), _rand_bf16((40, 32), 18)
+    Q = np.zeros((2, 32), np.uint16)
+    tokens = [1, 5, 9, 30]
+    O, lse = oracle.attention(Q, K, V, tokens, 1.0)
+    np.testing.assert_allclose(O[0], oracle.bf16_to_f64(V[tokens]).mean(0), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse, math.log(4.0), atol=1e-15)
+
+
+def test_attention_is_order_free_and_empty_is_zero():
+    Q, K, V = _rand_bf16((2, 32), 19), _rand_bf16((60, 32), 20), _rand_bf16((60, 16), 21)
+    a, la = oracle.attention(Q, K, V, [3, 50, 7, 22], 0.3)
+    b, lb = oracle.attention(Q, K, V, [22, 3, 7, 50], 0.3)
+    np.testing.assert_allclose(a, b, atol=1e-15)
+    np.testing.assert_allclose(la, lb, atol=1e-15)
+    O, lse = oracle.attention(Q, K, V, [], 0.3)
+    assert np.all(O == 0) and np.all(np.isneginf(lse))
+
+
+# ----------------------------------------------------------------------------- whole step
+def _small_problem(seed, G=4, d=64, r=16, T=400):
+    Q = _rand_bf16((G, d), seed, 0.3)
+    K = _rand_bf16((T, d), seed + 1)
+    V = _rand_bf16((T, d), seed + 2)
+    P = synth.orthonormal_basis(d, r, seed=seed + 3).numpy()
+    Kp, _ = oracle.project_rows(K, P)
+    return Q, K, V, P, Kp
+
+
+def test_step_identity_basis_selects_full_score_topk():
+    # r = d and P = I: the selection is the exact top-k of the full group scores.
+    G, d, T, k = 4, 64, 500, 40
+    Q, K, V, _, _ = _small_problem(30, G, d, d, T)
+    P = np.eye(d, dtype=np.float32)
+    Kp, _ = oracle.project_rows(K, P)
+    res = oracle.decode_head(Q, K, V, Kp, P, T, k, 0, 0.125)
+    full = oracle.bf16_to_f64(K) @ oracle.bf16_to_f64(Q).sum(0)
+    order = np.lexsort((np.arange(T), -full))
+    np.testing.assert_array_equal(res["idx"], np.sort(order[:k]))
+
+
+def test_step_with_k_equal_T_is_dense_attention():
+    # §4.5's full-KV baseline: with k = T the sparse step attends to every token.
+    Q, K, V, P, Kp = _small_problem(40)
+    T = K.shape[0]
+    res = oracle.decode_head(Q, K, V, Kp, P, T, T, 0, 0.125)
+    O, lse = _torch_attention(Q, K, V, np.arange(T), 0.125)
+    np.testing.assert_allclose(res["O"], O, atol=1e-13)
+    np.testing.assert_allclose(res["lse"], lse, atol=1e-12)
+    assert res["k_eff"] == T
+
+
+def test_step_window_covering_everything_is_dense():
+    Q, K, V, P, Kp = _small_problem(50)
+    T = K.shape[0]
+    res = oracle.decode_head(Q, K, V, Kp, P, T, 16, T + 5, 0.125)
+    O, _ = _torch_attention(Q, K, V, np.arange(T), 0.125)
+    np.testing.assert_allclose(res["O"], O, atol=1e-13)
+    assert res["k_eff"] == 0 and np.all(res["idx"] == -1)
+
+
+def test_step_window_attends_selection_plus_recent_tokens():
+    Q, K, V, P, Kp = _small_problem(60)
+    T, k, W = K.shape[0], 20, 50
+    res = oracle.decode_head(Q, K, V, Kp, P, T, k, W, 0.125)
+    s = oracle.scores(oracle.query_proj(Q, P), Kp[: T - W])
+    idx, _ = oracle.topk(s, k)
+    assert np.all(idx < T - W)
+    np.testing.assert_array_equal(res["idx"], idx)
+    toks = np.concatenate([idx, np.arange(T - W, T)])
+    O, _ = _torch_attention(Q, K, V, toks, 0.125)
+    np.testing.assert_allclose(res["O"], O, atol=1e-13)
+
+
+def test_step_permuting_cache_rows_keeps_selected_rows_and_output():
+    Q, K, V, P, Kp = _small_problem(70, T=300)
+    T, k = 300, 25
+    res = oracle.decode_head(Q, K, V, Kp, P, T, k, 0, 0.125)
+    s = res["scores"]
+    kth = np.sort(s)[::-1][k - 1]
+    assert np.sum(s == kth) == 1                  # no tie at the boundary for this seed
+    perm = np.random.default_rng(1).permutation(T)
+    res_p = oracle.decode_head(Q, K[perm], V[perm], Kp[perm], P, T, k, 0, 0.125)
+    assert set(perm[res_p["idx"]].tolist()) == set(res["idx"].tolist())
+    np.testing.assert_allclose(res_p["O"], res["O"], atol=1e-13)
+
+
+def test_step_mla_shape_reduces_to_gqa_formula():
+    # MLA (§3.3, §A.3): one latent row per token serves as the key (576 dims) and, on its
+    # first 512 dims, as the value; all 128 query heads share one index set.
+    G, dk, dv, r, T, k = 128, 576, 512, 64, 160, 12
+    Q = _rand_bf16((G, dk), 80, 0.05)
+    L = _rand_bf16((T, dk), 81)
+    P = synth.orthonormal_basis(dk, r, seed=82).numpy()
+    Kp, _ = oracle.project_rows(L, P)
+    res = oracle.decode_head(Q, L, L[:, :dv], Kp, P, T, k, 0, 1 / math.sqrt(dk))
+    full_q = P.astype(np.float64).T @ oracle.bf16_to_f64(Q).sum(0)
+    s = oracle.bf16_to_f64(Kp) @ full_q
+    order = np.lexsort((np.arange(T), -s))
+    np.testing.assert_array_equal(res["idx"], np.sort(order[:k]))
+    O, _ = _torch_attention(Q, L, np.ascontiguousarray(L[:, :dv]), res["idx"], 1 / math.sqrt(dk))
+    np.testing.assert_allclose(res["O"], O, atol=1e-13)
+
+
+def test_whole_batch_decode_step_on_tiny_workload():
+    w = synth.WORKLOADS["tiny"].with_(T=512, k=32)
+    x = synth.make_inputs(w, seq_lens=[500])
+    Q, K, V, P = u16(x["Q"]), u16(x["K"]), u16(x["V"]), f32(x["P"])
+    Kp = oracle.project_cache(K, P)
+    out = oracle.decode_step(Q, K, V, Kp, P, x["seq_lens"].numpy(), w.k, 0, w.sm_scale)
+    assert out["idx"].shape == (1, 2, 32) and np.all(out["n_sel"] == 32)
+    assert np.all(out["idx"] < 500) and np.all(np.diff(out["idx"], axis=-1) > 0)
+    # heavy (x4) rows dominate the selection of this generator
+    assert np.isfinite(out["O"]).all()
