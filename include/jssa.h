@@ -1,0 +1,209 @@
+/*
+ * jssa.h — C ABI of libjssa.so: the decode-step hot path of Joint Subspace Sparse
+ * Attention on NVIDIA B200 (sm_100a).
+ *
+ * Method: "Joint Subspace Sparse Attention for Efficient Long-Context Decoding"
+ * (Song, Kim, Kim; arXiv 2610.19026v1, paperlayer.ai summary).  At each decoding
+ * step, per KV head, the projected group query scores a projected-key cache
+ * Kp = K P, the top-B positions are selected per sequence and KV head, and the
+ * group's query heads attend over the original full-dimensional K/V rows at those
+ * positions, read in place (Figure 1; §3.1 Overview; §3.3 Gather-free indexed
+ * attention; §3.4 Projected scoring cache; §E.1 the new key is projected on write).
+ * "B" (the token budget) is called k here.
+ *
+ * Conventions fixed by this library (the summary leaves them open):
+ *   - group query = SUM of the G query heads of a KV head (the page's "mean" times
+ *     G; the ranking is identical);
+ *   - score of token t for KV head h = fp32 dot product of (sum_g P_h^T q_g) with
+ *     Kp[t] — the projected query is formed in fp32 from bf16 Q and fp32 P;
+ *   - ties in the top-k break toward the lower token index; selected indices are
+ *     written in ascending order; unused slots are -1;
+ *   - Kp is stored in bf16, rounded to nearest-even once from an fp64 accumulation
+ *     of K P (bit-identical to rounding the exact product, except in cases where
+ *     the exact value lies within ~1e-16 relative of a rounding midpoint);
+ *   - attention uses an explicit softmax scale sm_scale (logit = sm_scale * q . k);
+ *     split partials are combined by a log-sum-exp merge;
+ *   - with a sliding window W > 0 (hybrid local/global models, §A.1/§A.3), the
+ *     candidates are [0, T - W) and the attended set is the selection plus the
+ *     window [T - W, T);
+ *   - MLA (§3.3, §A.3): one latent row per token per layer (Hkv = 1) serves as the
+ *     key (d_k dims) and, on its first d_v dims, as the value; all query heads
+ *     share one index set.
+ *
+ * Memory model.  Every pointer argument named "device" points to GPU memory owned
+ * by the caller; the library never allocates, frees or synchronises on the compute
+ * calls.  All compute calls are asynchronous on `stream` (a cudaStream_t passed as
+ * void*; NULL = the legacy default stream) and contain no host synchronisation, so
+ * they can be captured into a CUDA graph.  Scratch memory is a caller-provided
+ * workspace of at least jssa_workspace_size() bytes, 256-byte aligned; its
+ * contents need not be initialised.
+ *
+ * Errors.  Arguments are validated on the host before any launch; an invalid call
+ * returns an error status and launches nothing.  A launch failure returns
+ * JSSA_ERR_CUDA.  Values only visible on the device (seq_lens, n_sel, indices) are
+ * clamped or skipped by the kernels, which record what they saw in a status word
+ * inside the workspace; jssa_read_device_status() returns and clears it.
+ * No C++ exception crosses this interface.
+ */
+#ifndef JSSA_H_
+#define JSSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define JSSA_API __attribute__((visibility("default")))
+#else
+#define JSSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  JSSA_OK = 0,
+  JSSA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, stride or alignment      */
+  JSSA_ERR_UNSUPPORTED = 2,  /* a valid but unimplemented shape (d, r, G, mode)  */
+  JSSA_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small       */
+  JSSA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed             */
+  JSSA_ERR_DEVICE_CHECK = 5, /* the kernels flagged out-of-range device data     */
+  JSSA_ERR_TIMEOUT = 6       /* a bounded wait inside a kernel gave up           */
+} jssa_status;
+
+enum { JSSA_MODE_GQA = 0, JSSA_MODE_MLA = 1 };
+enum { JSSA_OUT_F32 = 0, JSSA_OUT_BF16 = 1 };
+
+/* Device status bits reported by jssa_read_device_status(). */
+enum {
+  JSSA_DEV_BAD_SEQ_LEN = 1, /* a seq_lens[b] outside [0, T_cap] (clamped)        */
+  JSSA_DEV_BAD_INDEX = 2,   /* an index outside its candidate range (skipped)    */
+  JSSA_DEV_BAD_NSEL = 4,    /* an n_sel outside [0, k] (clamped)                 */
+  JSSA_DEV_TIMEOUT = 8      /* a bounded wait gave up                            */
+};
+
+/*
+ * Shapes and cache layout.  Element strides, last dimension contiguous.
+ *   Q    [B, Hq, d_k]      bf16, contiguous
+ *   K    element (b, h, t, i) at K[b*k_stride[0] + h*k_stride[1] + t*k_stride[2] + i], i < d_k
+ *   V    element (b, h, t, i) at V[b*v_stride[0] + h*v_stride[1] + t*v_stride[2] + i], i < d_v
+ *   Kp   element (b, h, t, j) at Kp[b*kp_stride[0] + h*kp_stride[1] + t*kp_stride[2] + j], j < r
+ *   P    [Hkv, d_k, r]     fp32, contiguous (column j of P_h is the j-th basis vector)
+ *   O    [B, Hq, d_v]      fp32 or bf16 (out_dtype), contiguous
+ *   lse  [B, Hq]           fp32 natural-log log-sum-exp of the scaled logits (optional)
+ * GQA: Hq = G * Hkv; query head hq belongs to KV head hq / G.  Supported: d_k = d_v in
+ * {64, 128, 256}, G in {1, 2, 4, 8, 16}, r in {8, 16, 32, 64} (r <= d_k).
+ * MLA: Hkv = 1, d_k = 576, d_v = 512, Hq = 128, r in {16, 32, 64}; V may alias K.
+ * K/V/Kp base pointers and strides (except the unit inner stride) must be
+ * multiples of 16 bytes.
+ */
+typedef struct {
+  int32_t mode;      /* JSSA_MODE_GQA or JSSA_MODE_MLA                    */
+  int32_t B, Hq, Hkv;
+  int32_t d_k, d_v, r;
+  int32_t out_dtype; /* JSSA_OUT_F32 or JSSA_OUT_BF16                      */
+  int64_t T_cap;     /* rows allocated per (b, h) in K, V and Kp            */
+  int64_t k_stride[3];
+  int64_t v_stride[3];
+  int64_t kp_stride[3];
+} jssa_layout;
+
+/* Human-readable name of a status code (static string). */
+JSSA_API const char* jssa_status_string(jssa_status s);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+JSSA_API int32_t jssa_version(void);
+
+/*
+ * Bytes of workspace needed by every compute call below for this layout, a budget
+ * of at most k tokens and a window of at most `window` tokens, on the current
+ * device.  Host-only.
+ */
+JSSA_API jssa_status jssa_workspace_size(const jssa_layout* L, int32_t k, int32_t window, size_t* bytes);
+
+/*
+ * Projected scoring cache on write (§3.1, §3.4, §E.1):
+ *   Kp[b, h, t, :] = bf16(K[b, h, t, :] . P_h)   for t in [t_begin[b], t_begin[b] + n_tokens)
+ * t_begin: device int32 [B] (rows past T_cap are skipped), or NULL to mean
+ * t_begin[b] = seq_lens[b] - n_tokens (the last n_tokens rows; then seq_lens is
+ * required).  n_tokens = 0 is a no-op.
+ */
+JSSA_API jssa_status jssa_project_keys(const jssa_layout* L, const void* K, const float* P, void* Kp,
+                              const int32_t* t_begin, const int32_t* seq_lens, int64_t n_tokens,
+                              void* stream);
+
+/*
+ * Subspace score scan (Figure 1; §2 "score every candidate position"):
+ *   scores[b, h, t] = fp32( (sum_g P_h^T q_{hG+g}) . Kp[b, h, t] )   for t in [0, T_b - W)
+ * with T_b = seq_lens[b] (device int32 [B]) and W = window clamped to [0, T_b].
+ * scores: device fp32 [B, Hkv, T_cap]; entries at t >= T_b - W are not written.
+ */
+JSSA_API jssa_status jssa_score(const jssa_layout* L, const void* Q, const float* P, const void* Kp,
+                       const int32_t* seq_lens, int32_t window, float* scores,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Per-(sequence, KV head) top-k (Figure 1 "top-B positions"; §E.3 per-KV-head
+ * selection) over scores[b, h, 0 : T_b - W):
+ *   idx[b, h, :]  the k_eff = min(k, T_b - W) positions of largest score, ties to the
+ *                 lower index, ascending; slots >= k_eff are -1      (device int32 [B, Hkv, k])
+ *   n_sel[b, h]   k_eff                                               (device int32 [B, Hkv])
+ * Scores must be finite.
+ */
+JSSA_API jssa_status jssa_topk(const jssa_layout* L, const float* scores, const int32_t* seq_lens,
+                      int32_t k, int32_t window, int32_t* idx, int32_t* n_sel,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Gather-free indexed attention (§3.3) with split-T partials and a log-sum-exp merge.
+ * For query head hq of KV head h: attended set = {idx[b, h, j] : j < n_sel[b, h]} plus
+ * the window [T_b - W, T_b); logits = sm_scale * q . K_t; O = softmax . V.  K/V rows
+ * are read in place.  idx entries must be distinct and in [0, T_b - W); out-of-range
+ * entries are skipped and flagged.  lse may be NULL.
+ */
+JSSA_API jssa_status jssa_indexed_attn(const jssa_layout* L, const void* Q, const void* K, const void* V,
+                              const int32_t* idx, int32_t k, const int32_t* n_sel,
+                              const int32_t* seq_lens, int32_t window, float sm_scale,
+                              void* O, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * One fused decode step (Figure 1): project the last n_new rows of each sequence
+ * into Kp (n_new may be 0 when Kp is already current), score, select the top-k per
+ * (sequence, KV head), attend over the selection (plus the window) and merge.
+ * idx_out / n_sel_out (nullable) receive the selection; otherwise it stays in the
+ * workspace.  lse may be NULL.
+ */
+JSSA_API jssa_status jssa_decode_step(const jssa_layout* L, const void* Q, const void* K, const void* V,
+                             void* Kp, const float* P, const int32_t* seq_lens, int32_t n_new,
+                             int32_t k, int32_t window, float sm_scale, void* O, float* lse,
+                             int32_t* idx_out, int32_t* n_sel_out, void* workspace,
+                             size_t ws_bytes, void* stream);
+
+/*
+ * Dense full-KV flash-decode (the full-KV baseline of §4.5), same kernel family as
+ * jssa_indexed_attn with the index list replaced by the contiguous range
+ * [T_b - W, T_b) (W = window clamped to T_b; window = 0 means all of [0, T_b)).
+ */
+JSSA_API jssa_status jssa_dense_decode(const jssa_layout* L, const void* Q, const void* K, const void* V,
+                              const int32_t* seq_lens, int32_t window, float sm_scale, void* O,
+                              float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Zero the device status word at the start of a freshly allocated workspace (the
+ * compute calls only ever set bits in it).  Needed once per workspace, before the
+ * first jssa_read_device_status(); the compute results do not depend on it.
+ */
+JSSA_API jssa_status jssa_workspace_init(void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Read and clear the device status word kept in the workspace (JSSA_DEV_* bits).
+ * Synchronises `stream`.  Returns JSSA_ERR_DEVICE_CHECK if any bit other than
+ * JSSA_DEV_TIMEOUT was set, JSSA_ERR_TIMEOUT if that bit was set, else JSSA_OK.
+ */
+JSSA_API jssa_status jssa_read_device_status(void* workspace, size_t ws_bytes, int32_t* flags, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JSSA_H_ */

@@ -1,0 +1,158 @@
+"""C ABI of libjssa.so on the CPU: the library builds, loads and exports every entry
+point that include/jssa.h declares; host-side validation rejects bad arguments
+before any CUDA call (so these run without a GPU)."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "jssa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from token_level_sparse_jssa_b200 import build
+    build.build()
+    from token_level_sparse_jssa_b200 import _binding
+    return _binding.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"JSSA_API\s+[\w\s\*]+?\b(jssa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("jssa_project_keys", "jssa_score", "jssa_topk", "jssa_indexed_attn", "jssa_decode_step",
+                     "jssa_dense_decode", "jssa_workspace_size"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from token_level_sparse_jssa_b200 import _binding
+    out = subprocess.run(["nm", "-D", "--defined-only", _binding.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\sT\s(jssa_\w+)$", out, flags=re.M))
+    assert set(declared_functions()) <= exported
+    for name in declared_functions():
+        assert hasattr(lib, name)
+    assert set(_binding.EXPORTS) == set(declared_functions())
+
+
+def test_header_compiles_as_plain_c(tmp_path):
+    src = tmp_path / "t.c"
+    src.write_text('#include "jssa.h"\nint main(void){ jssa_layout L; (void)L; return (int)JSSA_OK; }\n')
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), "-c", str(src),
+                    "-o", str(tmp_path / "t.o")], check=True)
+
+
+def test_layout_struct_matches_header_size(tmp_path):
+    from token_level_sparse_jssa_b200 import Layout
+    src = tmp_path / "s.c"
+    src.write_text('#include <stdio.h>\n#include "jssa.h"\nint main(void){ printf("%zu", sizeof(jssa_layout)); return 0; }\n')
+    exe = tmp_path / "s"
+    subprocess.run(["gcc", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)], check=True)
+    assert int(subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout) == C.sizeof(Layout)
+
+
+def test_status_strings_and_version(lib):
+    from token_level_sparse_jssa_b200 import status_string, version
+    assert status_string(0) == "ok"
+    assert "workspace" in status_string(3)
+    assert status_string(99) == "unknown status"
+    assert version() >= 10000
+
+
+def _layout(**kw):
+    from token_level_sparse_jssa_b200 import Layout
+    L = Layout()
+    B, Hq, Hkv, d, r, T = kw.get("B", 2), kw.get("Hq", 8), kw.get("Hkv", 2), kw.get("d", 128), kw.get("r", 32), \
+        kw.get("T", 1024)
+    L.mode, L.B, L.Hq, L.Hkv, L.d_k, L.d_v, L.r, L.out_dtype = kw.get("mode", 0), B, Hq, Hkv, d, kw.get("dv", d), r, \
+        kw.get("out", 0)
+    L.T_cap = T
+    for i, v in enumerate((Hkv * T * d, T * d, d)):
+        L.k_stride[i] = v
+        L.v_stride[i] = v
+    for i, v in enumerate((Hkv * T * r, T * r, r)):
+        L.kp_stride[i] = v
+    for key in ("k_stride", "v_stride", "kp_stride"):
+        if key in kw:
+            for i, v in enumerate(kw[key]):
+                getattr(L, key)[i] = v
+    return L
+
+
+FAKE = 0x10000  # a 16-byte aligned non-null value; validation rejects the call before it is used
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=7), 1),                 # Hq not a multiple of Hkv
+    (dict(r=0), 1),
+    (dict(r=256), 1),                # r > d
+    (dict(r=24), 2),                 # r not a supported power of two
+    (dict(d=96), 2),                 # unsupported head dim
+    (dict(Hq=64, Hkv=2), 2),         # G = 32
+    (dict(dv=64), 1),                # d_v != d_k in GQA -> invalid? d_v < d_k is unsupported
+    (dict(mode=1), 2),               # MLA needs Hkv=1, 576/512, 128 heads
+    (dict(mode=5), 1),
+    (dict(out=3), 1),
+    (dict(T=0), 1),
+    (dict(k_stride=(8, 8, 100)), 1),  # stride not a multiple of 16 bytes
+    (dict(kp_stride=(0, 0, 64)), 2),  # Kp rows must be contiguous
+])
+def test_bad_layouts_are_rejected_on_the_host(lib, kw, code):
+    L = _layout(**kw)
+    got = lib.jssa_project_keys(C.byref(L), FAKE, FAKE, FAKE, FAKE, None, 1, None)
+    if kw == dict(dv=64):
+        assert got in (1, 2)
+    else:
+        assert got == code
+
+
+def test_bad_arguments_are_rejected_before_launch(lib):
+    L = _layout()
+    ws = C.c_void_p(FAKE)
+    # null pointers
+    assert lib.jssa_project_keys(C.byref(L), None, FAKE, FAKE, FAKE, None, 4, None) == 1
+    assert lib.jssa_project_keys(C.byref(L), FAKE, FAKE, FAKE, None, None, 4, None) == 1
+    # misaligned cache pointer
+    assert lib.jssa_project_keys(C.byref(L), FAKE + 2, FAKE, FAKE, FAKE, None, 4, None) == 1
+    # n_tokens out of range
+    assert lib.jssa_project_keys(C.byref(L), FAKE, FAKE, FAKE, FAKE, None, -1, None) == 1
+    assert lib.jssa_project_keys(C.byref(L), FAKE, FAKE, FAKE, FAKE, None, 5000, None) == 1
+    # n_tokens = 0 is a no-op that touches nothing
+    assert lib.jssa_project_keys(C.byref(L), None, None, None, None, None, 0, None) == 0
+    # k < 1, negative window
+    assert lib.jssa_topk(C.byref(L), FAKE, FAKE, 0, 0, FAKE, FAKE, None, 0, None) == 1
+    assert lib.jssa_topk(C.byref(L), FAKE, FAKE, 4, -1, FAKE, FAKE, None, 0, None) == 1
+    assert lib.jssa_indexed_attn(C.byref(L), FAKE, FAKE, FAKE, None, 4, FAKE, FAKE, 0, 1.0, FAKE, None, ws, 1 << 30,
+                                 None) == 1
+    assert lib.jssa_decode_step(C.byref(L), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, -1, 4, 0, 1.0, FAKE, None, None,
+                                None, ws, 1 << 30, None) == 1
+    assert lib.jssa_dense_decode(C.byref(L), FAKE, FAKE, FAKE, FAKE, -3, 1.0, FAKE, None, ws, 1 << 30, None) == 1
+    assert lib.jssa_dense_decode(None, FAKE, FAKE, FAKE, FAKE, 0, 1.0, FAKE, None, ws, 1 << 30, None) == 1
+    # workspace status helpers check their arguments
+    assert lib.jssa_workspace_init(None, 0, None) == 3
+    assert lib.jssa_workspace_init(C.c_void_p(FAKE + 16), 1024, None) == 3  # not 256-byte aligned
+    flags = C.c_int32(0)
+    assert lib.jssa_read_device_status(None, 0, C.byref(flags), None) == 3
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_workspace_size_without_a_device_reports_a_cuda_error(lib):
+    n = C.c_size_t(0)
+    assert lib.jssa_workspace_size(C.byref(_layout()), 16, 0, C.byref(n)) == 4
+
+
+def test_package_import_does_not_load_the_library_and_fails_loudly_when_missing(tmp_path):
+    code = ("import token_level_sparse_jssa_b200 as j, token_level_sparse_jssa_b200._binding as b;"
+            "assert b._lib is None\n"
+            "try:\n    b.load(r'%s')\nexcept RuntimeError as e:\n    print('LOUD', e)\n" % (tmp_path / "missing.so"))
+    out = subprocess.run(["python", "-c", code], capture_output=True, text=True, cwd=ROOT, check=True).stdout
+    assert "LOUD" in out and "no fallback" in out

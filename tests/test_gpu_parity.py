@@ -1,0 +1,380 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, stage by stage and
+end to end, on seeded synthetic inputs shaped like the pages' workloads.
+
+Stages get independent inputs from the generator (the oracle never consumes an
+output of the CUDA path): projection from K and P; scoring from Q, P and the
+projected cache; top-k from generated score rows; attention from generated index
+sets.  The fused step is compared on its selection (bit-exact up to swaps inside the
+tie window) and on its output (fp64 oracle on the same index set).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests._problem import Problem, check_attention, check_selection, score_error_bound
+from tests._util import u16, f32, rel_l2
+import token_level_sparse_jssa_b200 as jssa
+from token_level_sparse_jssa_b200 import synth
+
+pytestmark = pytest.mark.gpu
+W = synth.WORKLOADS
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    jssa.load()
+    yield
+    torch.cuda.synchronize()
+
+
+def _assert_status_clean(ws):
+    code, flags = jssa.read_device_status(ws)
+    assert code == 0 and flags == 0, (code, flags)
+
+
+# ----------------------------------------------------------------------------- a1 projection
+@pytest.mark.parametrize("name,kw", [
+    ("tiny", dict(T=700)),
+    ("tiny", dict(T=300, r=8, dk=64, dv=64)),
+    ("h128k", dict(B=2, T=1100)),
+    ("hybrid", dict(B=1, T=515)),
+    ("mla", dict(B=2, T=333)),
+])
+def test_project_keys_is_bit_exact(name, kw):
+    w = W[name].with_(**kw)
+    p = Problem(w)
+    p.fill_kp()
+    torch.cuda.synchronize()
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            ref, _ = oracle.project_rows(u16(p.K[b, h]), f32(p.P[h]))
+            np.testing.assert_array_equal(u16(p.Kp[b, h]), ref)
+
+
+def test_project_keys_last_rows_only():
+    w = W["tiny"].with_(B=3, T=500)
+    p = Problem(w, T_cap=512, seq_lens=[500, 37, 512])
+    jssa.project_keys(p.L, p.K, p.P, p.Kp, 3, seq_lens=p.seq_lens)   # rows [T_b-3, T_b)
+    torch.cuda.synchronize()
+    kp = u16(p.Kp)
+    for b, T in enumerate([500, 37, 512]):
+        for h in range(w.Hkv):
+            ref, _ = oracle.project_rows(u16(p.K[b, h, T - 3:T]), f32(p.P[h]))
+            np.testing.assert_array_equal(kp[b, h, T - 3:T], ref)
+            assert np.all(kp[b, h, :T - 3] == 0) and np.all(kp[b, h, T:] == 0)
+
+
+# ----------------------------------------------------------------------------- a2-a3 scoring
+@pytest.mark.parametrize("name,kw,seq,window", [
+    ("tiny", {}, None, 0),
+    ("h128k", dict(B=3, T=5000), [5000, 17, 4097], 0),
+    ("hybrid", dict(B=2, T=3000), [3000, 2100], 1024),
+    ("tiny", dict(T=900, r=8, dk=64, dv=64, Hq=16, Hkv=1), None, 5),
+    ("mla", dict(B=2, T=1200), [1200, 999], 0),
+])
+def test_score_within_fp32_error_bound(name, kw, seq, window):
+    w = W[name].with_(**kw)
+    p = Problem(w, seq_lens=seq)
+    p.fill_kp()
+    ws = p.workspace(1, window)
+    scores = torch.full((w.B, w.Hkv, p.T_cap), float("nan"), device="cuda")
+    jssa.score(p.L, p.Q, p.P, p.Kp, p.seq_lens, window, scores, ws)
+    torch.cuda.synchronize()
+    sc = scores.cpu().numpy().astype(np.float64)
+    for b in range(w.B):
+        T = int(p.seq_lens[b])
+        n = T - min(window, T)
+        for h in range(w.Hkv):
+            hst = p.host(b, h)
+            Kp_or, _ = oracle.project_rows(hst["K"][:n], hst["P"])
+            np.testing.assert_array_equal(hst["Kp"][:n], Kp_or)
+            s_or = oracle.scores(oracle.query_proj(hst["Q"], hst["P"]), Kp_or)
+            bound = score_error_bound(hst["Q"], hst["P"], Kp_or)
+            err = np.abs(sc[b, h, :n] - s_or)
+            assert np.all(err <= bound * 1.0001 + 1e-30), float(np.max(err / np.maximum(bound, 1e-30)))
+            assert np.all(np.isnan(sc[b, h, n:])), "entries past the candidates must not be written"
+    _assert_status_clean(ws)
+
+
+# ----------------------------------------------------------------------------- a4 top-k
+@pytest.mark.parametrize("rows_T,k,seq,window,ties", [
+    ((1, 64), 5, [64], 0, 3),
+    ((1, 2048), 128, [2048], 0, 20),
+    ((3, 20000), 2048, [20000, 1999, 15001], 0, 50),     # ragged, one row below k
+    ((4, 131072), 2048, None, 0, 200),                    # 8-CTA clusters
+    ((2, 65536), 1024, [65536, 40000], 1024, 100),        # window shrinks the candidates
+    ((2, 4096), 4096, [4096, 100], 0, 10),                # k >= n: select everything
+    ((1, 400000), 777, [400000], 0, 100),                 # slice larger than shared memory
+    ((2, 5000), 1, [5000, 1], 0, 2),
+])
+def test_topk_is_bit_exact(rows_T, k, seq, window, ties):
+    B, T = rows_T
+    Hkv = 1
+    scores = synth.random_scores(B * Hkv, T, seed=T + k, ties=ties, zeros=8).cuda()
+    seq = seq or [T] * B
+    L = jssa.Layout()
+    L.mode, L.B, L.Hq, L.Hkv, L.d_k, L.d_v, L.r, L.out_dtype, L.T_cap = 0, B, 4, Hkv, 128, 128, 16, 0, T
+    for i, v in enumerate((Hkv * T * 128, T * 128, 128)):
+        L.k_stride[i] = v
+        L.v_stride[i] = v
+    for i, v in enumerate((Hkv * T * 16, T * 16, 16)):
+        L.kp_stride[i] = v
+    sl = torch.tensor(seq, dtype=torch.int32, device="cuda")
+    idx = torch.full((B, Hkv, k), -7, dtype=torch.int32, device="cuda")
+    nsel = torch.full((B, Hkv), -7, dtype=torch.int32, device="cuda")
+    jssa.topk(L, scores, sl, k, window, idx, nsel)
+    torch.cuda.synchronize()
+    s_host = scores.cpu().numpy().astype(np.float64)
+    for b in range(B):
+        n = seq[b] - min(window, seq[b])
+        ref, k_eff = oracle.topk(s_host[b, :n], k)
+        assert int(nsel[b, 0]) == k_eff
+        np.testing.assert_array_equal(idx[b, 0].cpu().numpy(), ref)
+
+
+# ----------------------------------------------------------------------------- a5-a6 attention
+@pytest.mark.parametrize("name,kw,seq,k,window,out", [
+    ("tiny", {}, None, 128, 0, 0),
+    ("tiny", dict(T=1000, dk=64, dv=64, r=8), None, 100, 0, 0),
+    ("h128k", dict(B=2, T=9000), [9000, 4000], 2048, 0, 0),
+    ("h128k", dict(B=2, T=3000, Hq=16, Hkv=16), [3000, 2500], 300, 0, 0),     # G = 1
+    ("h128k", dict(B=1, T=3000, Hq=32, Hkv=4), [3000], 500, 0, 0),           # G = 8
+    ("h128k", dict(B=1, T=3000, Hq=32, Hkv=2), [3000], 257, 0, 0),           # G = 16
+    ("hybrid", dict(B=2, T=6000), [6000, 1500], 1024, 1024, 0),              # d = 256 + window
+    ("hybrid", dict(B=1, T=2000), [2000], 7, 3, 1),                          # bf16 output
+])
+def test_indexed_attention_matches_oracle(name, kw, seq, k, window, out):
+    w = W[name].with_(**kw)
+    p = Problem(w, seq_lens=seq, out_dtype=out)
+    seq = seq or [w.T] * w.B
+    ncand = [T - min(window, T) for T in seq]
+    idx = synth.random_index_sets(w.B * w.Hkv, [n for n in ncand for _ in range(w.Hkv)], k, seed=k)
+    nsel = (idx >= 0).sum(-1).to(torch.int32)
+    idx = idx.view(w.B, w.Hkv, k).cuda()
+    nsel = nsel.view(w.B, w.Hkv).cuda()
+    ws = p.workspace(k, window)
+    O = torch.full((w.B, w.Hq, w.dv), float("nan"), device="cuda",
+                   dtype=torch.bfloat16 if out else torch.float32)
+    lse = torch.full((w.B, w.Hq), float("nan"), device="cuda")
+    jssa.indexed_attn(p.L, p.Q, p.K, p.V, idx, k, nsel, p.seq_lens, window, w.sm_scale, O, lse, ws)
+    torch.cuda.synchronize()
+    G = w.G
+    for b in range(w.B):
+        T = seq[b]
+        for h in range(w.Hkv):
+            hst = p.host(b, h)
+            n = int(nsel[b, h])
+            toks = np.concatenate([idx[b, h, :n].cpu().numpy(), np.arange(T - min(window, T), T)])
+            O_ref, lse_ref = oracle.attention(hst["Q"], hst["K"], hst["V"], toks, w.sm_scale)
+            O_gpu = O[b, h * G:(h + 1) * G].float().cpu().numpy().astype(np.float64)
+            if out:
+                # bf16 output: the fp32 result rounded once
+                np.testing.assert_allclose(O_gpu, O_ref, atol=8e-3, rtol=8e-3)
+            else:
+                check_attention(O_gpu, O_ref, f"b={b} h={h}")
+            np.testing.assert_allclose(lse[b, h * G:(h + 1) * G].cpu().numpy(), lse_ref, atol=1e-4, rtol=1e-5)
+    _assert_status_clean(ws)
+
+
+@pytest.mark.parametrize("name,kw,seq,window", [
+    ("tiny", {}, None, 0),
+    ("h128k", dict(B=2, T=7000), [7000, 333], 0),
+    ("hybrid", dict(B=2, T=5000), [5000, 800], 1024),    # local layer: dense over the window
+])
+def test_dense_decode_matches_oracle(name, kw, seq, window):
+    w = W[name].with_(**kw)
+    p = Problem(w, seq_lens=seq)
+    seq = seq or [w.T] * w.B
+    ws = p.workspace(1, window)
+    O = torch.full((w.B, w.Hq, w.dv), float("nan"), device="cuda")
+    lse = torch.empty((w.B, w.Hq), device="cuda")
+    jssa.dense_decode(p.L, p.Q, p.K, p.V, p.seq_lens, window, w.sm_scale, O, lse, ws)
+    torch.cuda.synchronize()
+    G = w.G
+    for b in range(w.B):
+        T = seq[b]
+        lo = max(0, T - window) if window > 0 else 0
+        for h in range(w.Hkv):
+            hst = p.host(b, h)
+            O_ref, lse_ref = oracle.attention(hst["Q"], hst["K"], hst["V"], np.arange(lo, T), w.sm_scale)
+            check_attention(O[b, h * G:(h + 1) * G].cpu().numpy().astype(np.float64), O_ref, f"dense b={b} h={h}")
+            np.testing.assert_allclose(lse[b, h * G:(h + 1) * G].cpu().numpy(), lse_ref, atol=1e-4, rtol=1e-5)
+
+
+def test_sparse_with_k_equal_T_equals_dense():
+    w = W["tiny"].with_(T=1500, k=1500)
+    p = Problem(w)
+    p.fill_kp()
+    ws = p.workspace(w.k)
+    O_s = torch.empty((w.B, w.Hq, w.dv), device="cuda")
+    O_d = torch.empty_like(O_s)
+    jssa.decode_step(p.L, p.Q, p.K, p.V, p.Kp, p.P, p.seq_lens, 0, w.k, 0, w.sm_scale, O_s, ws=ws)
+    jssa.dense_decode(p.L, p.Q, p.K, p.V, p.seq_lens, 0, w.sm_scale, O_d, ws=ws)
+    torch.cuda.synchronize()
+    assert float((O_s - O_d).abs().max()) < 1e-5
+
+
+def test_single_token_selection_returns_the_value_row():
+    w = W["tiny"].with_(T=600)
+    p = Problem(w)
+    idx = torch.full((1, w.Hkv, 4), -1, dtype=torch.int32, device="cuda")
+    idx[0, :, 0] = torch.tensor([17, 599], dtype=torch.int32)
+    nsel = torch.ones((1, w.Hkv), dtype=torch.int32, device="cuda")
+    ws = p.workspace(4)
+    O = torch.empty((1, w.Hq, w.dv), device="cuda")
+    jssa.indexed_attn(p.L, p.Q, p.K, p.V, idx, 4, nsel, p.seq_lens, 0, w.sm_scale, O, None, ws)
+    torch.cuda.synchronize()
+    for h, t in enumerate([17, 599]):
+        ref = p.V[0, h, t].float().expand(w.G, -1)
+        assert torch.equal(O[0, h * w.G:(h + 1) * w.G], ref)
+
+
+# ----------------------------------------------------------------------------- fused step
+def _check_step(p, k, window, O, idx, nsel, rows, what):
+    w = p.w
+    G = w.G
+    n_same = 0
+    for (b, h) in rows:
+        T = int(p.seq_lens[b])
+        hst = p.host(b, h)
+        Kp_or, _ = oracle.project_rows(hst["K"][:T], hst["P"])
+        res = oracle.decode_head(hst["Q"], hst["K"][:T], hst["V"][:T], Kp_or, hst["P"], T, k, window, w.sm_scale)
+        g_idx = idx[b, h].cpu().numpy()
+        _, same = check_selection(g_idx, int(nsel[b, h]), res["scores"], k)
+        O_gpu = O[b, h * G:(h + 1) * G].float().cpu().numpy().astype(np.float64)
+        if same:
+            O_ref = res["O"]
+            n_same += 1
+        else:  # an allowed swap inside the tie window: the oracle runs on the GPU's own set
+            n = int(nsel[b, h])
+            toks = np.concatenate([g_idx[:n], np.arange(T - min(window, T), T)])
+            O_ref, _ = oracle.attention(hst["Q"], hst["K"], hst["V"], toks, w.sm_scale)
+        check_attention(O_gpu, O_ref, f"{what} b={b} h={h}")
+    return n_same
+
+
+@pytest.mark.parametrize("name,kw,seq,window", [
+    ("tiny", {}, None, 0),
+    ("llama8b", dict(B=2, T=6000, k=512), [6000, 4321], 0),
+    ("h128k", dict(B=2, T=20000, k=1024), [20000, 11111], 0),
+    ("hybrid", dict(B=2, T=9000, k=512), [9000, 3000], 1024),
+])
+def test_decode_step_end_to_end(name, kw, seq, window):
+    w = W[name].with_(**kw)
+    p = Problem(w, seq_lens=seq)
+    p.fill_kp()
+    ws = p.workspace(w.k, window)
+    O = torch.full((w.B, w.Hq, w.dv), float("nan"), device="cuda")
+    idx = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device="cuda")
+    nsel = torch.empty((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+    jssa.decode_step(p.L, p.Q, p.K, p.V, p.Kp, p.P, p.seq_lens, 1, w.k, window, w.sm_scale, O, None, idx, nsel, ws)
+    torch.cuda.synchronize()
+    rows = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    _check_step(p, w.k, window, O, idx, nsel, rows, name)
+    _assert_status_clean(ws)
+
+
+def test_decode_step_append_loop_updates_the_scoring_cache():
+    # workload 2 in miniature: each step appends one token (its K/V row is already in the
+    # cache at position T_b) and projects it on write before scoring.
+    w = W["llama8b"].with_(B=2, T=3000, k=256)
+    p = Problem(w, T_cap=3010, seq_lens=[3000, 2500])
+    tb = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+    jssa.project_keys(p.L, p.K, p.P, p.Kp, 3000, t_begin=tb)   # prefill rows [0, 3000)
+    torch.cuda.synchronize()
+    p.Kp[1, :, 2500:] = 0                                        # sequence 1 is shorter
+    ws = p.workspace(w.k)
+    O = torch.empty((w.B, w.Hq, w.dv), device="cuda")
+    idx = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device="cuda")
+    nsel = torch.empty((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+    for step in range(3):
+        p.seq_lens += 1
+        jssa.decode_step(p.L, p.Q, p.K, p.V, p.Kp, p.P, p.seq_lens, 1, w.k, 0, w.sm_scale, O, None, idx, nsel, ws)
+        torch.cuda.synchronize()
+        for b in range(w.B):
+            T = int(p.seq_lens[b])
+            for h in range(w.Hkv):
+                ref, _ = oracle.project_rows(u16(p.K[b, h, T - 1:T]), f32(p.P[h]))
+                np.testing.assert_array_equal(u16(p.Kp[b, h, T - 1:T]), ref)
+        _check_step(p, w.k, 0, O, idx, nsel, [(0, 0), (1, 7), (1, 3)], f"append step {step}")
+
+
+def test_decode_step_in_a_cuda_graph_matches_eager():
+    w = W["h128k"].with_(B=2, T=8192, k=512)
+    p = Problem(w)
+    p.fill_kp()
+    ws = p.workspace(w.k)
+    O1 = torch.empty((w.B, w.Hq, w.dv), device="cuda")
+    O2 = torch.empty_like(O1)
+    jssa.decode_step(p.L, p.Q, p.K, p.V, p.Kp, p.P, p.seq_lens, 0, w.k, 0, w.sm_scale, O1, ws=ws)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            jssa.decode_step(p.L, p.Q, p.K, p.V, p.Kp, p.P, p.seq_lens, 0, w.k, 0, w.sm_scale, O2, ws=ws)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(O1, O2)
+
+
+# ----------------------------------------------------------------------------- guards
+def test_device_checks_flag_bad_indices_and_seq_lens():
+    w = W["tiny"].with_(T=400)
+    p = Problem(w, T_cap=400)
+    ws = p.workspace(8)
+    idx = torch.tensor([[[3, 5, 9999, -4, 7, -1, -1, -1], [1, 2, 3, 4, 5, 6, 7, 8]]], dtype=torch.int32,
+                       device="cuda")
+    nsel = torch.tensor([[5, 8]], dtype=torch.int32, device="cuda")
+    O = torch.empty((1, w.Hq, w.dv), device="cuda")
+    jssa.indexed_attn(p.L, p.Q, p.K, p.V, idx, 8, nsel, p.seq_lens, 0, w.sm_scale, O, None, ws)
+    code, flags = jssa.read_device_status(ws)
+    assert code == 5 and flags & jssa._binding.DEV_BAD_INDEX
+    assert torch.isfinite(O).all()
+    # the out-of-range entries were skipped: same as attending to {3, 5, 7}
+    hst = p.host(0, 0)
+    O_ref, _ = oracle.attention(hst["Q"], hst["K"], hst["V"], [3, 5, 7], w.sm_scale)
+    check_attention(O[0, :w.G].cpu().numpy().astype(np.float64), O_ref, "skip")
+    bad = torch.tensor([401], dtype=torch.int32, device="cuda")
+    jssa.dense_decode(p.L, p.Q, p.K, p.V, bad, 0, w.sm_scale, O, None, ws)
+    code, flags = jssa.read_device_status(ws)
+    assert code == 5 and flags & jssa._binding.DEV_BAD_SEQ_LEN
+    code, flags = jssa.read_device_status(ws)
+    assert code == 0 and flags == 0
+
+
+def test_invalid_calls_launch_nothing():
+    w = W["tiny"].with_(T=256)
+    p = Problem(w)
+    ws = p.workspace(16)
+    O = torch.full((w.B, w.Hq, w.dv), float("nan"), device="cuda")
+    with pytest.raises(jssa.JssaError):
+        jssa.decode_step(p.L, p.Q, p.K, p.V, p.Kp, p.P, p.seq_lens, 0, 0, 0, w.sm_scale, O, ws=ws)   # k = 0
+    with pytest.raises(jssa.JssaError):
+        jssa.decode_step(p.L, p.Q, p.K, p.V, p.Kp, p.P, p.seq_lens, 0, 16, 0, w.sm_scale, O,
+                         ws=ws[:1024])                                                                 # too small
+    with pytest.raises(jssa.JssaError):
+        jssa.decode_step(p.L, p.Q, p.K, p.V, p.Kp, p.P, p.seq_lens, 0, 16, 0, w.sm_scale, O,
+                         ws=ws[8:])                                                                    # misaligned
+    torch.cuda.synchronize()
+    assert torch.isnan(O).all()
+
+
+def test_empty_sequences_and_short_rows():
+    w = W["tiny"].with_(B=3, T=64, k=32)
+    p = Problem(w, T_cap=64, seq_lens=[0, 5, 64])
+    p.fill_kp()
+    ws = p.workspace(w.k)
+    O = torch.full((w.B, w.Hq, w.dv), float("nan"), device="cuda")
+    idx = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device="cuda")
+    nsel = torch.empty((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+    lse = torch.empty((w.B, w.Hq), device="cuda")
+    jssa.decode_step(p.L, p.Q, p.K, p.V, p.Kp, p.P, p.seq_lens, 0, w.k, 0, w.sm_scale, O, lse, idx, nsel, ws)
+    torch.cuda.synchronize()
+    assert torch.all(O[0] == 0) and torch.all(torch.isneginf(lse[0]))
+    assert torch.all(nsel[0] == 0) and torch.all(idx[0] == -1)
+    assert torch.all(nsel[1] == 5) and torch.equal(idx[1, :, :5].cpu(), torch.arange(5).expand(w.Hkv, 5).int())
+    _check_step(p, w.k, 0, O, idx, nsel, [(1, 0), (1, 1), (2, 0), (2, 1)], "short")

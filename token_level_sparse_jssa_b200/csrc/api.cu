@@ -1,0 +1,386 @@
+// C ABI of libjssa.so (declared in include/jssa.h): host-side validation, workspace
+// carving, split policy and the launch sequence of each entry point.  No entry point
+// allocates, frees or synchronises, except jssa_read_device_status.
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/jssa.h"
+#include "common.cuh"
+#include "launch.h"
+
+namespace jssa {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxK = 1 << 24;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int num_sms_current() {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return -1;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool is_pow2_in(int x, int lo, int hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
+
+jssa_status check_layout(const jssa_layout* L) {
+  if (!L) return JSSA_ERR_INVALID_ARG;
+  if (L->mode != JSSA_MODE_GQA && L->mode != JSSA_MODE_MLA) return JSSA_ERR_INVALID_ARG;
+  if (L->B < 1 || L->Hq < 1 || L->Hkv < 1 || L->d_k < 1 || L->d_v < 1 || L->r < 1 || L->T_cap < 1)
+    return JSSA_ERR_INVALID_ARG;
+  if (L->T_cap > (int64_t(1) << 31) - 1) return JSSA_ERR_INVALID_ARG;
+  if (L->Hq % L->Hkv != 0) return JSSA_ERR_INVALID_ARG;
+  if (L->r > L->d_k || L->d_v > L->d_k) return JSSA_ERR_INVALID_ARG;
+  if (L->out_dtype != JSSA_OUT_F32 && L->out_dtype != JSSA_OUT_BF16) return JSSA_ERR_INVALID_ARG;
+  if (L->B > 1024) return JSSA_ERR_UNSUPPORTED;
+  for (int i = 0; i < 3; ++i) {
+    if (L->k_stride[i] < 0 || L->v_stride[i] < 0 || L->kp_stride[i] < 0) return JSSA_ERR_INVALID_ARG;
+    if (L->k_stride[i] % 8 || L->v_stride[i] % 8 || L->kp_stride[i] % 8) return JSSA_ERR_INVALID_ARG;
+  }
+  if (L->k_stride[2] < L->d_k || L->v_stride[2] < L->d_v) return JSSA_ERR_INVALID_ARG;
+  if (L->kp_stride[2] != L->r) return JSSA_ERR_UNSUPPORTED;  // Kp rows are streamed as one block
+  if (!is_pow2_in(L->r, 8, 64)) return JSSA_ERR_UNSUPPORTED;
+  const int G = L->Hq / L->Hkv;
+  if (L->mode == JSSA_MODE_GQA) {
+    if (L->d_k != L->d_v) return JSSA_ERR_UNSUPPORTED;
+    if (L->d_k != 64 && L->d_k != 128 && L->d_k != 256) return JSSA_ERR_UNSUPPORTED;
+    if (!is_pow2_in(G, 1, 16)) return JSSA_ERR_UNSUPPORTED;
+  } else {
+    if (L->Hkv != 1 || L->d_k != 576 || L->d_v != 512 || L->Hq != 128) return JSSA_ERR_UNSUPPORTED;
+  }
+  return JSSA_OK;
+}
+
+struct Workspace {
+  int* status;
+  float* qs;
+  float* scores;
+  int32_t* idx;
+  int32_t* n_sel;
+  float* part_lse;
+  float* part_o;
+  int S_cap;
+  size_t bytes;
+};
+
+// Carve the workspace for (layout, k, window).  With base == nullptr only sizes.
+jssa_status carve(const jssa_layout* L, int64_t k, int64_t window, void* base, Workspace* w) {
+  const int num_sms = num_sms_current();
+  if (num_sms <= 0) return JSSA_ERR_CUDA;
+  const int rows = L->B * L->Hkv;
+  // partials for every split count a call with this (k, window) can use
+  int S_cap = 1, S = 1, len = 0;
+  attn_split_policy(L->mode, true, rows, min64(k + window, L->T_cap), num_sms, &S, &len);
+  S_cap = S > S_cap ? S : S_cap;
+  attn_split_policy(L->mode, false, rows, L->T_cap, num_sms, &S, &len);
+  S_cap = S > S_cap ? S : S_cap;
+  if (window > 0) {
+    attn_split_policy(L->mode, false, rows, min64(window, L->T_cap), num_sms, &S, &len);
+    S_cap = S > S_cap ? S : S_cap;
+  }
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    const size_t o = off;
+    off += align_up(n);
+    return o;
+  };
+  const size_t o_status = take(sizeof(int));
+  const size_t o_qs = take(sizeof(float) * rows * L->r);
+  const size_t o_scores = take(sizeof(float) * static_cast<size_t>(rows) * L->T_cap);
+  const size_t o_idx = take(sizeof(int32_t) * static_cast<size_t>(rows) * k);
+  const size_t o_nsel = take(sizeof(int32_t) * rows);
+  const size_t o_lse = take(sizeof(float) * static_cast<size_t>(L->B) * L->Hq * S_cap);
+  const size_t o_po = take(sizeof(float) * static_cast<size_t>(L->B) * L->Hq * S_cap * L->d_v);
+  w->bytes = off;
+  w->S_cap = S_cap;
+  char* p = static_cast<char*>(base);
+  w->status = p ? reinterpret_cast<int*>(p + o_status) : nullptr;
+  w->qs = p ? reinterpret_cast<float*>(p + o_qs) : nullptr;
+  w->scores = p ? reinterpret_cast<float*>(p + o_scores) : nullptr;
+  w->idx = p ? reinterpret_cast<int32_t*>(p + o_idx) : nullptr;
+  w->n_sel = p ? reinterpret_cast<int32_t*>(p + o_nsel) : nullptr;
+  w->part_lse = p ? reinterpret_cast<float*>(p + o_lse) : nullptr;
+  w->part_o = p ? reinterpret_cast<float*>(p + o_po) : nullptr;
+  return JSSA_OK;
+}
+
+jssa_status get_ws(const jssa_layout* L, int64_t k, int64_t window, void* ws, size_t ws_bytes, Workspace* w) {
+  if (!ws || !aligned(ws, kAlign)) return JSSA_ERR_WORKSPACE;
+  jssa_status st = carve(L, k, window, ws, w);
+  if (st != JSSA_OK) return st;
+  if (ws_bytes < w->bytes) return JSSA_ERR_WORKSPACE;
+  return JSSA_OK;
+}
+
+jssa_status cu(cudaError_t e) {
+  if (e == cudaSuccess) return JSSA_OK;
+  if (e == cudaErrorNotSupported) return JSSA_ERR_UNSUPPORTED;
+  return JSSA_ERR_CUDA;
+}
+
+ProjectArgs project_args(const jssa_layout* L, const void* K, const float* P, void* Kp, const int32_t* t_begin,
+                         const int32_t* seq_lens, int64_t n, int* status) {
+  ProjectArgs a{};
+  a.K = K;
+  memcpy(a.ks, L->k_stride, sizeof a.ks);
+  a.P = P;
+  a.Kp = Kp;
+  memcpy(a.ps, L->kp_stride, sizeof a.ps);
+  a.t_begin = t_begin;
+  a.seq_lens = seq_lens;
+  a.n_tokens = n;
+  a.B = L->B;
+  a.Hkv = L->Hkv;
+  a.d = L->d_k;
+  a.r = L->r;
+  a.T_cap = L->T_cap;
+  a.status = status;
+  return a;
+}
+
+jssa_status run_score(const jssa_layout* L, const void* Q, const float* P, const void* Kp, const int32_t* seq_lens,
+                      int window, float* scores, int64_t sc_ld, const Workspace& w, cudaStream_t s) {
+  QprojArgs q{};
+  q.Q = Q;
+  q.P = P;
+  q.qs = w.qs;
+  q.B = L->B;
+  q.Hq = L->Hq;
+  q.Hkv = L->Hkv;
+  q.d = L->d_k;
+  q.r = L->r;
+  jssa_status st = cu(launch_qproj(q, s));
+  if (st != JSSA_OK) return st;
+  ScoreArgs a{};
+  a.Kp = Kp;
+  memcpy(a.ps, L->kp_stride, sizeof a.ps);
+  a.qs = w.qs;
+  a.scores = scores;
+  a.sc_ld = sc_ld;
+  a.seq_lens = seq_lens;
+  a.B = L->B;
+  a.Hkv = L->Hkv;
+  a.r = L->r;
+  a.T_cap = L->T_cap;
+  a.window = window;
+  a.status = w.status;
+  return cu(launch_score(a, num_sms_current(), s));
+}
+
+jssa_status run_topk(const jssa_layout* L, const float* scores, int64_t sc_ld, const int32_t* seq_lens, int k,
+                     int window, int32_t* idx, int32_t* n_sel, int* status, cudaStream_t s) {
+  TopkArgs a{};
+  a.scores = scores;
+  a.sc_ld = sc_ld;
+  a.seq_lens = seq_lens;
+  a.B = L->B;
+  a.Hkv = L->Hkv;
+  a.T_cap = L->T_cap;
+  a.k = k;
+  a.window = window;
+  a.idx = idx;
+  a.n_sel = n_sel;
+  a.status = status;
+  return cu(launch_topk(a, s));
+}
+
+jssa_status run_attention(const jssa_layout* L, const void* Q, const void* K, const void* V, const int32_t* idx,
+                          int idx_ld, const int32_t* n_sel, const int32_t* seq_lens, int window, float sm_scale,
+                          void* O, float* lse, const Workspace& w, cudaStream_t s) {
+  AttnArgs a{};
+  a.Q = Q;
+  a.K = K;
+  memcpy(a.ks, L->k_stride, sizeof a.ks);
+  a.V = V;
+  memcpy(a.vs, L->v_stride, sizeof a.vs);
+  a.idx = idx;
+  a.idx_ld = idx_ld;
+  a.n_sel = n_sel;
+  a.seq_lens = seq_lens;
+  a.B = L->B;
+  a.Hq = L->Hq;
+  a.Hkv = L->Hkv;
+  a.dk = L->d_k;
+  a.dv = L->d_v;
+  a.T_cap = L->T_cap;
+  a.window = window;
+  a.sm_scale = sm_scale;
+  const bool indexed = idx != nullptr;
+  a.list_max = indexed ? static_cast<int64_t>(idx_ld) + window : (window > 0 ? window : L->T_cap);
+  if (a.list_max > L->T_cap) a.list_max = L->T_cap;
+  attn_split_policy(L->mode, indexed, L->B * L->Hkv, a.list_max, num_sms_current(), &a.S, &a.split_len);
+  if (a.S > w.S_cap) return JSSA_ERR_WORKSPACE;
+  a.part_o = w.part_o;
+  a.part_lse = w.part_lse;
+  a.O = O;
+  a.lse = lse;
+  a.out_bf16 = (L->out_dtype == JSSA_OUT_BF16);
+  a.status = w.status;
+  jssa_status st = cu(L->mode == JSSA_MODE_MLA ? launch_mla_attention(a, s) : launch_attention(a, s));
+  if (st != JSSA_OK) return st;
+  return cu(launch_merge(a, s));
+}
+
+}  // namespace
+}  // namespace jssa
+
+using namespace jssa;
+
+extern "C" {
+
+const char* jssa_status_string(jssa_status s) {
+  switch (s) {
+    case JSSA_OK: return "ok";
+    case JSSA_ERR_INVALID_ARG: return "invalid argument";
+    case JSSA_ERR_UNSUPPORTED: return "unsupported shape or mode";
+    case JSSA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case JSSA_ERR_CUDA: return "CUDA error";
+    case JSSA_ERR_DEVICE_CHECK: return "device-side check failed";
+    case JSSA_ERR_TIMEOUT: return "bounded wait timed out";
+  }
+  return "unknown status";
+}
+
+int32_t jssa_version(void) { return 10000; }
+
+jssa_status jssa_workspace_size(const jssa_layout* L, int32_t k, int32_t window, size_t* bytes) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  if (!bytes || k < 1 || k > kMaxK || window < 0) return JSSA_ERR_INVALID_ARG;
+  Workspace w{};
+  st = carve(L, k, window, nullptr, &w);
+  if (st != JSSA_OK) return st;
+  *bytes = w.bytes;
+  return JSSA_OK;
+}
+
+jssa_status jssa_project_keys(const jssa_layout* L, const void* K, const float* P, void* Kp, const int32_t* t_begin,
+                              const int32_t* seq_lens, int64_t n_tokens, void* stream) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  if (n_tokens < 0 || n_tokens > L->T_cap) return JSSA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return JSSA_OK;
+  if (!K || !P || !Kp || (!t_begin && !seq_lens)) return JSSA_ERR_INVALID_ARG;
+  if (!aligned(K, 16) || !aligned(Kp, 16) || !aligned(P, 4)) return JSSA_ERR_INVALID_ARG;
+  ProjectArgs a = project_args(L, K, P, Kp, t_begin, seq_lens, n_tokens, nullptr);
+  return cu(launch_project_keys(a, static_cast<cudaStream_t>(stream)));
+}
+
+jssa_status jssa_score(const jssa_layout* L, const void* Q, const float* P, const void* Kp, const int32_t* seq_lens,
+                       int32_t window, float* scores, void* workspace, size_t ws_bytes, void* stream) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  if (!Q || !P || !Kp || !seq_lens || !scores || window < 0) return JSSA_ERR_INVALID_ARG;
+  if (!aligned(Q, 4) || !aligned(P, 4) || !aligned(Kp, 16) || !aligned(scores, 4)) return JSSA_ERR_INVALID_ARG;
+  Workspace w{};
+  st = get_ws(L, 1, window, workspace, ws_bytes, &w);
+  if (st != JSSA_OK) return st;
+  return run_score(L, Q, P, Kp, seq_lens, window, scores, L->T_cap, w, static_cast<cudaStream_t>(stream));
+}
+
+jssa_status jssa_topk(const jssa_layout* L, const float* scores, const int32_t* seq_lens, int32_t k, int32_t window,
+                      int32_t* idx, int32_t* n_sel, void* workspace, size_t ws_bytes, void* stream) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  if (!scores || !seq_lens || !idx || !n_sel || k < 1 || k > kMaxK || window < 0) return JSSA_ERR_INVALID_ARG;
+  if (!aligned(scores, 4) || !aligned(idx, 4) || !aligned(n_sel, 4)) return JSSA_ERR_INVALID_ARG;
+  int* status = nullptr;
+  if (workspace) {
+    Workspace w{};
+    st = get_ws(L, k, window, workspace, ws_bytes, &w);
+    if (st != JSSA_OK) return st;
+    status = w.status;
+  }
+  return run_topk(L, scores, L->T_cap, seq_lens, k, window, idx, n_sel, status, static_cast<cudaStream_t>(stream));
+}
+
+jssa_status jssa_indexed_attn(const jssa_layout* L, const void* Q, const void* K, const void* V, const int32_t* idx,
+                              int32_t k, const int32_t* n_sel, const int32_t* seq_lens, int32_t window, float sm_scale,
+                              void* O, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  if (!Q || !K || !V || !idx || !n_sel || !seq_lens || !O || k < 1 || k > kMaxK || window < 0)
+    return JSSA_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(idx, 4) || !aligned(O, 4))
+    return JSSA_ERR_INVALID_ARG;
+  Workspace w{};
+  st = get_ws(L, k, window, workspace, ws_bytes, &w);
+  if (st != JSSA_OK) return st;
+  return run_attention(L, Q, K, V, idx, k, n_sel, seq_lens, window, sm_scale, O, lse, w,
+                       static_cast<cudaStream_t>(stream));
+}
+
+jssa_status jssa_decode_step(const jssa_layout* L, const void* Q, const void* K, const void* V, void* Kp,
+                             const float* P, const int32_t* seq_lens, int32_t n_new, int32_t k, int32_t window,
+                             float sm_scale, void* O, float* lse, int32_t* idx_out, int32_t* n_sel_out, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  if (!Q || !K || !V || !Kp || !P || !seq_lens || !O || k < 1 || k > kMaxK || window < 0 || n_new < 0 ||
+      n_new > L->T_cap)
+    return JSSA_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(Kp, 16) || !aligned(P, 4) || !aligned(O, 4))
+    return JSSA_ERR_INVALID_ARG;
+  if ((idx_out && !aligned(idx_out, 4)) || (n_sel_out && !aligned(n_sel_out, 4))) return JSSA_ERR_INVALID_ARG;
+  Workspace w{};
+  st = get_ws(L, k, window, workspace, ws_bytes, &w);
+  if (st != JSSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n_new > 0) {
+    ProjectArgs pa = project_args(L, K, P, Kp, nullptr, seq_lens, n_new, w.status);
+    st = cu(launch_project_keys(pa, s));
+    if (st != JSSA_OK) return st;
+  }
+  st = run_score(L, Q, P, Kp, seq_lens, window, w.scores, L->T_cap, w, s);
+  if (st != JSSA_OK) return st;
+  int32_t* idx = idx_out ? idx_out : w.idx;
+  int32_t* nsel = n_sel_out ? n_sel_out : w.n_sel;
+  st = run_topk(L, w.scores, L->T_cap, seq_lens, k, window, idx, nsel, w.status, s);
+  if (st != JSSA_OK) return st;
+  return run_attention(L, Q, K, V, idx, k, nsel, seq_lens, window, sm_scale, O, lse, w, s);
+}
+
+jssa_status jssa_dense_decode(const jssa_layout* L, const void* Q, const void* K, const void* V,
+                              const int32_t* seq_lens, int32_t window, float sm_scale, void* O, float* lse,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  if (!Q || !K || !V || !seq_lens || !O || window < 0) return JSSA_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 4)) return JSSA_ERR_INVALID_ARG;
+  Workspace w{};
+  st = get_ws(L, 1, window, workspace, ws_bytes, &w);
+  if (st != JSSA_OK) return st;
+  return run_attention(L, Q, K, V, nullptr, 0, nullptr, seq_lens, window, sm_scale, O, lse, w,
+                       static_cast<cudaStream_t>(stream));
+}
+
+jssa_status jssa_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
+  if (!workspace || !aligned(workspace, kAlign) || ws_bytes < sizeof(int)) return JSSA_ERR_WORKSPACE;
+  return cu(cudaMemsetAsync(workspace, 0, sizeof(int), static_cast<cudaStream_t>(stream)));
+}
+
+jssa_status jssa_read_device_status(void* workspace, size_t ws_bytes, int32_t* flags, void* stream) {
+  if (!workspace || !aligned(workspace, kAlign) || ws_bytes < sizeof(int)) return JSSA_ERR_WORKSPACE;
+  if (!flags) return JSSA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof v, cudaMemcpyDeviceToHost, s) != cudaSuccess) return JSSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return JSSA_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof v, s) != cudaSuccess) return JSSA_ERR_CUDA;
+  *flags = v;
+  if (v & ~DEVFLAG_TIMEOUT) return JSSA_ERR_DEVICE_CHECK;
+  if (v & DEVFLAG_TIMEOUT) return JSSA_ERR_TIMEOUT;
+  return JSSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,418 @@
+// Gather-free indexed flash-decode (GQA) with split-T partials, and their LSE merge.
+//
+// "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", §3.3: one
+// launch per layer handles distinct per-KV-head index sets and reads the selected
+// K/V entries in place from the standard GQA cache layout, with no gather buffer and
+// no per-head launches; §2.2 / §4.7: gathering first would cost about as much as the
+// reduced attention itself.  The same kernel with a contiguous range instead of an
+// index list is the dense full-KV decode used as the baseline (§4.5).
+//
+// Grid: (split, sequence * KV head).  Each CTA owns one contiguous slice of the
+// attended list (selected positions followed by the sliding window).  Its 4 warps
+// take 16-token subtiles in turn; each warp streams the subtile's K and V rows with
+// 16-byte cp.async copies (one 2*d-byte coalesced row per token, XOR-swizzled in
+// shared memory) through a private multi-stage ring, so no block barrier sits in the
+// main loop.  All G query heads of the group stay in registers as MMA operands:
+//   S^T[16 tok x 8 heads] = K_sub[16 x d] . Q^T         (mma.sync m16n8k16, bf16 -> fp32)
+//   online softmax per head in fp32 (exp2 domain)
+//   O^T[d x 8 heads]     += V_sub^T . P^T               (P split into bf16 hi + lo parts,
+//                                                        so the weights keep ~16 bits)
+// The 4 warps' states are merged in shared memory and the CTA writes one normalised
+// partial (o, lse) per query head; the merge kernel combines the splits.
+#include <cmath>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace jssa {
+
+constexpr int kAttnWarps = 4;
+constexpr int kAttnThreads = kAttnWarps * 32;
+constexpr int kSub = 16;                 // tokens per warp subtile
+constexpr int kMaxTokList = 4096;        // indexed mode: split length bound (token list in smem)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D>
+struct AttnCfg {
+  static constexpr int STAGES = (D <= 64) ? 4 : (D <= 128 ? 3 : 2);
+  static constexpr int CPR = D / 8;                    // 16-byte chunks per row
+  static constexpr int SUB_BYTES = kSub * D * 2;       // one K or V subtile
+  static constexpr int STAGE_BYTES = 2 * SUB_BYTES;
+  static constexpr int RING_BYTES = kAttnWarps * STAGES * STAGE_BYTES;
+  static constexpr int COMBINE_BYTES = kAttnWarps * 16 * D * 4 + 2 * kAttnWarps * 16 * 4;
+  static constexpr int MAIN_BYTES = RING_BYTES > COMBINE_BYTES ? RING_BYTES : COMBINE_BYTES;
+};
+
+template <int D, bool DENSE>
+static size_t attn_smem_bytes() {
+  return AttnCfg<D>::MAIN_BYTES + (DENSE ? 0 : kMaxTokList * sizeof(int32_t));
+}
+
+template <int D, int NTILE, bool DENSE>
+__global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
+  using Cfg = AttnCfg<D>;
+  constexpr int STAGES = Cfg::STAGES, CPR = Cfg::CPR;
+  constexpr int KSTEPS = D / 16;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  unsigned char* ring = smem_raw + warp * STAGES * Cfg::STAGE_BYTES;
+  int32_t* tok_s = reinterpret_cast<int32_t*>(smem_raw + Cfg::MAIN_BYTES);
+
+  const int split = blockIdx.x, row = blockIdx.y;
+  const int b = row / a.Hkv, h = row % a.Hkv;
+  const int G = a.Hq / a.Hkv;
+  int64_t T = a.seq_lens[b];
+  if (T < 0 || T > a.T_cap) {
+    if (split == 0 && threadIdx.x == 0) flag_error(a.status, DEVFLAG_BAD_SEQ_LEN);
+    T = T < 0 ? 0 : a.T_cap;
+  }
+  int64_t list_len, win_start;
+  int64_t nsel = 0;
+  if (DENSE) {
+    win_start = (a.window > 0) ? max64(0, T - a.window) : 0;
+    list_len = T - win_start;
+  } else {
+    const int64_t Wc = min64(max64(a.window, 0), T);
+    win_start = T - Wc;
+    nsel = a.n_sel[row];
+    const int64_t nsel_max = min64(a.idx_ld, win_start);
+    if (nsel < 0 || nsel > nsel_max) {
+      if (split == 0 && threadIdx.x == 0) flag_error(a.status, DEVFLAG_BAD_NSEL);
+      nsel = nsel < 0 ? 0 : nsel_max;
+    }
+    list_len = nsel + Wc;
+  }
+  const int64_t my_lo = static_cast<int64_t>(split) * a.split_len;
+  const int my_len = static_cast<int>(max64(0, min64(list_len, my_lo + a.split_len) - my_lo));
+  const int64_t hq0 = static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * G;
+
+  if (my_len == 0) {  // empty split: weight zero in the merge
+    for (int i = threadIdx.x; i < G * D; i += kAttnThreads) {
+      const int head = i / D, dim = i % D;
+      a.part_o[((hq0 + head) * a.S + split) * D + dim] = 0.f;
+      if (dim == 0) a.part_lse[(hq0 + head) * a.S + split] = -INFINITY;
+    }
+    return;
+  }
+  if (!DENSE) {
+    const int32_t* irow = a.idx + static_cast<int64_t>(row) * a.idx_ld;
+    for (int j = threadIdx.x; j < my_len; j += kAttnThreads) {
+      const int64_t pos = my_lo + j;
+      int64_t t;
+      if (pos < nsel) {
+        t = irow[pos];
+        if (t < 0 || t >= win_start) {
+          flag_error(a.status, DEVFLAG_BAD_INDEX);
+          t = -1;
+        }
+      } else {
+        t = win_start + (pos - nsel);
+      }
+      tok_s[j] = static_cast<int32_t>(t);
+    }
+    __syncthreads();
+  }
+
+  // Q^T as MMA B fragments: head nt*8 + g, dims kk*16 + 2c (+8)
+  uint32_t qf[NTILE][KSTEPS][2];
+  const __nv_bfloat16* Qg = static_cast<const __nv_bfloat16*>(a.Q) + hq0 * D;
+#pragma unroll
+  for (int nt = 0; nt < NTILE; ++nt) {
+    const int head = nt * 8 + g;
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      if (head < G) {
+        const uint32_t* qp = reinterpret_cast<const uint32_t*>(Qg + static_cast<int64_t>(head) * D + kk * 16 + 2 * c);
+        qf[nt][kk][0] = __ldg(qp);
+        qf[nt][kk][1] = __ldg(qp + 4);
+      } else {
+        qf[nt][kk][0] = 0u;
+        qf[nt][kk][1] = 0u;
+      }
+    }
+  }
+
+  const float scale_log2 = a.sm_scale * kLog2e;
+  float m_run[NTILE][2], l_run[NTILE][2];
+  float acc[KSTEPS][NTILE][4];
+#pragma unroll
+  for (int nt = 0; nt < NTILE; ++nt) {
+    m_run[nt][0] = m_run[nt][1] = -INFINITY;
+    l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+  }
+
+  const __nv_bfloat16* Kb = static_cast<const __nv_bfloat16*>(a.K) + b * a.ks[0] + h * a.ks[1];
+  const __nv_bfloat16* Vb = static_cast<const __nv_bfloat16*>(a.V) + b * a.vs[0] + h * a.vs[1];
+  const int nsub = (my_len + kSub - 1) / kSub;
+  const int my_count = (nsub > warp) ? (nsub - warp + kAttnWarps - 1) / kAttnWarps : 0;
+
+  auto token_at = [&](int j) -> int64_t {
+    if (j >= my_len) return -1;
+    return DENSE ? (win_start + my_lo + j) : static_cast<int64_t>(tok_s[j]);
+  };
+  auto issue = [&](int i) {  // i-th subtile of this warp into stage i % STAGES
+    const int sub = warp + i * kAttnWarps;
+    unsigned char* kbuf = ring + (i % STAGES) * Cfg::STAGE_BYTES;
+    unsigned char* vbuf = kbuf + Cfg::SUB_BYTES;
+#pragma unroll
+    for (int q = 0; q < (kSub * CPR) / 32; ++q) {
+      const int cid = lane + q * 32;
+      const int tin = cid / CPR, ch = cid % CPR;
+      const int64_t t = token_at(sub * kSub + tin);
+      const uint32_t nbytes = (t >= 0) ? 16u : 0u;
+      const int64_t tt = (t >= 0) ? t : 0;
+      const int soff = (tin * CPR + (ch ^ (tin & 7))) * 16;
+      cp_async16(kbuf + soff, Kb + tt * a.ks[2] + ch * 8, nbytes);
+      cp_async16(vbuf + soff, Vb + tt * a.vs[2] + ch * 8, nbytes);
+    }
+  };
+
+#pragma unroll
+  for (int s = 0; s < STAGES - 1; ++s) {
+    if (s < my_count) issue(s);
+    cp_async_commit();
+  }
+  for (int i = 0; i < my_count; ++i) {
+    if (i + STAGES - 1 < my_count) issue(i + STAGES - 1);
+    cp_async_commit();
+    cp_async_wait<STAGES - 1>();
+    __syncwarp();
+    const int sub = warp + i * kAttnWarps;
+    const unsigned char* kbuf = ring + (i % STAGES) * Cfg::STAGE_BYTES;
+    const unsigned char* vbuf = kbuf + Cfg::SUB_BYTES;
+
+    // ---- S^T = K_sub . Q^T
+    float sacc[NTILE][4];
+#pragma unroll
+    for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+    {
+      const int tin = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+        const int ch = 2 * kk + (lane >> 4);
+        uint32_t af[4];
+        ldmatrix_x4(af, kbuf + (tin * CPR + (ch ^ (tin & 7))) * 16);
+#pragma unroll
+        for (int nt = 0; nt < NTILE; ++nt) mma_bf16_16816(sacc[nt], af, qf[nt][kk][0], qf[nt][kk][1]);
+      }
+    }
+    // ---- online softmax over the 16 tokens of this subtile
+    const bool v0 = token_at(sub * kSub + g) >= 0;
+    const bool v1 = token_at(sub * kSub + g + 8) >= 0;
+    uint32_t bhi[NTILE][2], blo[NTILE][2];
+#pragma unroll
+    for (int nt = 0; nt < NTILE; ++nt) {
+      float x[4];
+      x[0] = v0 ? sacc[nt][0] * scale_log2 : -INFINITY;
+      x[1] = v0 ? sacc[nt][1] * scale_log2 : -INFINITY;
+      x[2] = v1 ? sacc[nt][2] * scale_log2 : -INFINITY;
+      x[3] = v1 ? sacc[nt][3] * scale_log2 : -INFINITY;
+      float p[4];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float mx = fmaxf(x[e], x[2 + e]);
+        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
+        const float m_new = fmaxf(m_run[nt][e], mx);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        const float alpha = exp2f(m_run[nt][e] - m_use);
+        p[e] = exp2f(x[e] - m_use);
+        p[2 + e] = exp2f(x[2 + e] - m_use);
+        l_run[nt][e] = l_run[nt][e] * alpha + p[e] + p[2 + e];
+        m_run[nt][e] = m_new;
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt) {
+          acc[mt][nt][e] *= alpha;
+          acc[mt][nt][2 + e] *= alpha;
+        }
+      }
+      // P^T as B fragments (tokens x heads) via an in-register 8x8 transpose
+      const uint32_t h0 = pack_bf16x2(p[0], p[1]);
+      const uint32_t h1 = pack_bf16x2(p[2], p[3]);
+      const uint32_t l0 = pack_bf16x2(p[0] - bf16_bits_to_float(h0 & 0xFFFFu), p[1] - bf16_bits_to_float(h0 >> 16));
+      const uint32_t l1 = pack_bf16x2(p[2] - bf16_bits_to_float(h1 & 0xFFFFu), p[3] - bf16_bits_to_float(h1 >> 16));
+      bhi[nt][0] = movmatrix_trans(h0);
+      bhi[nt][1] = movmatrix_trans(h1);
+      blo[nt][0] = movmatrix_trans(l0);
+      blo[nt][1] = movmatrix_trans(l1);
+    }
+    // ---- O^T += V_sub^T . P^T
+    {
+      const int tin = (lane & 7) + (lane >> 4) * 8;
+#pragma unroll
+      for (int mt = 0; mt < KSTEPS; ++mt) {
+        const int ch = 2 * mt + ((lane >> 3) & 1);
+        uint32_t vf[4];
+        ldmatrix_x4_trans(vf, vbuf + (tin * CPR + (ch ^ (tin & 7))) * 16);
+#pragma unroll
+        for (int nt = 0; nt < NTILE; ++nt) {
+          mma_bf16_16816(acc[mt][nt], vf, bhi[nt][0], bhi[nt][1]);
+          mma_bf16_16816(acc[mt][nt], vf, blo[nt][0], blo[nt][1]);
+        }
+      }
+    }
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+
+  // ---- merge the 4 warps' states in shared memory
+#pragma unroll
+  for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float l = l_run[nt][e];
+      l += __shfl_xor_sync(0xFFFFFFFFu, l, 4);
+      l += __shfl_xor_sync(0xFFFFFFFFu, l, 8);
+      l += __shfl_xor_sync(0xFFFFFFFFu, l, 16);
+      l_run[nt][e] = l;
+    }
+  __syncthreads();  // ring no longer needed
+  float* o_w = reinterpret_cast<float*>(smem_raw);           // [warps][16 heads][D]
+  float* m_w = o_w + kAttnWarps * 16 * D;                     // [warps][16]
+  float* l_w = m_w + kAttnWarps * 16;                         // [warps][16]
+#pragma unroll
+  for (int nt = 0; nt < NTILE; ++nt) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int head = nt * 8 + 2 * c + e;
+      if (g == 0) {
+        m_w[warp * 16 + head] = m_run[nt][e];
+        l_w[warp * 16 + head] = l_run[nt][e];
+      }
+#pragma unroll
+      for (int mt = 0; mt < KSTEPS; ++mt) {
+        o_w[(warp * 16 + head) * D + mt * 16 + g] = acc[mt][nt][e];
+        o_w[(warp * 16 + head) * D + mt * 16 + g + 8] = acc[mt][nt][2 + e];
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < G * D; i += kAttnThreads) {
+    const int head = i / D, dim = i % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, m_w[w * 16 + head]);
+    float o = 0.f, lse = -INFINITY;
+    if (M != -INFINITY) {
+      float L = 0.f;
+#pragma unroll
+      for (int w = 0; w < kAttnWarps; ++w) {
+        const float sc = exp2f(m_w[w * 16 + head] - M);
+        L += l_w[w * 16 + head] * sc;
+        o += o_w[(w * 16 + head) * D + dim] * sc;
+      }
+      o /= L;
+      lse = (M + log2f(L)) * kLn2;
+    }
+    a.part_o[((hq0 + head) * a.S + split) * D + dim] = o;
+    if (dim == 0) a.part_lse[(hq0 + head) * a.S + split] = lse;
+  }
+}
+
+// ------------------------------------------------------------------ LSE merge
+// O = sum_s w_s o_s / sum_s w_s with w_s = exp(lse_s - max lse); lse = max + log(sum w).
+__global__ void __launch_bounds__(256) merge_kernel(AttnArgs a) {
+  extern __shared__ float wsh[];  // [S]
+  __shared__ float sh_M, sh_L;
+  const int64_t q = blockIdx.x;   // b * Hq + hq
+  const int S = a.S, D = a.dv;
+  const float* lse_s = a.part_lse + q * S;
+  if (threadIdx.x == 0) {
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) M = fmaxf(M, lse_s[s]);
+    float L = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float w = (M == -INFINITY) ? 0.f : expf(lse_s[s] - M);
+      wsh[s] = w;
+      L += w;
+    }
+    sh_M = M;
+    sh_L = L;
+  }
+  __syncthreads();
+  const float M = sh_M, L = sh_L;
+  for (int dim = threadIdx.x; dim < D; dim += blockDim.x) {
+    float o = 0.f;
+    if (M != -INFINITY) {
+      for (int s = 0; s < S; ++s) o += wsh[s] * a.part_o[(q * S + s) * D + dim];
+      o /= L;
+    }
+    if (a.out_bf16) static_cast<__nv_bfloat16*>(a.O)[q * D + dim] = __float2bfloat16_rn(o);
+    else static_cast<float*>(a.O)[q * D + dim] = o;
+  }
+  if (a.lse && threadIdx.x == 0) a.lse[q] = (M == -INFINITY) ? -INFINITY : M + logf(L);
+}
+
+// ------------------------------------------------------------------ host side
+void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int num_sms, int* S_out, int* split_out) {
+  // Choose the split length (a multiple of the 16-token subtile, at least 64 tokens) that
+  // keeps the last wave of CTAs fullest; fewer splits win ties.  MLA splits are longer
+  // (each CTA amortises the 128-head query block over more tokens).
+  const int min_split = (mode == 1) ? 128 : 64;
+  const int slots = num_sms * ((mode == 1) ? 1 : 2);
+  if (list_max <= 0) { *S_out = 1; *split_out = min_split; return; }
+  int best_S = 0;
+  int64_t best_len = 0;
+  double best_eff = -1.0;
+  for (int S = 1; S <= 256; ++S) {
+    int64_t len = ceil_div(ceil_div(list_max, S), 16) * 16;
+    if (len < min_split) len = min_split;
+    const int64_t Sr = ceil_div(list_max, len);
+    if (Sr != S) continue;
+    if (indexed && mode != 1 && len > kMaxTokList) continue;  // the token list lives in shared memory
+    const int64_t ctas = static_cast<int64_t>(rows) * Sr;
+    const int64_t waves = ceil_div(ctas, slots);
+    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
+    if (eff > best_eff + 0.02) { best_eff = eff; best_S = S; best_len = len; }
+  }
+  if (best_S == 0) {  // only reachable for lists longer than 256 splits of the maximum length
+    best_len = ceil_div(ceil_div(list_max, 256), 16) * 16;
+    best_S = static_cast<int>(ceil_div(list_max, best_len));
+  }
+  *S_out = best_S;
+  *split_out = static_cast<int>(best_len);
+}
+
+template <int D, int NTILE, bool DENSE>
+static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
+  const size_t smem = attn_smem_bytes<D, DENSE>();
+  static int done[64] = {0};
+  cudaError_t e = set_smem_limit_once(attn_kernel<D, NTILE, DENSE>, smem, done);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.S, a.B * a.Hkv);
+  attn_kernel<D, NTILE, DENSE><<<grid, kAttnThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, bool DENSE>
+static cudaError_t launch_attn_d(const AttnArgs& a, cudaStream_t s) {
+  const int G = a.Hq / a.Hkv;
+  return (G <= 8) ? launch_attn_t<D, 1, DENSE>(a, s) : launch_attn_t<D, 2, DENSE>(a, s);
+}
+
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s) {
+  const bool dense = (a.idx == nullptr);
+  if (!dense && a.split_len > kMaxTokList) return cudaErrorInvalidValue;
+  switch (a.dk) {
+    case 64: return dense ? launch_attn_d<64, true>(a, s) : launch_attn_d<64, false>(a, s);
+    case 128: return dense ? launch_attn_d<128, true>(a, s) : launch_attn_d<128, false>(a, s);
+    case 256: return dense ? launch_attn_d<256, true>(a, s) : launch_attn_d<256, false>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_merge(const AttnArgs& a, cudaStream_t s) {
+  merge_kernel<<<a.B * a.Hq, 256, a.S * sizeof(float), s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace jssa

@@ -1,0 +1,89 @@
+// Internal launch interface between the C ABI layer (api.cu) and the kernel files.
+// Host-side only; every launcher enqueues on `stream` and returns the launch error.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace jssa {
+
+struct ProjectArgs {
+  const void* K;
+  int64_t ks[3];
+  const float* P;
+  void* Kp;
+  int64_t ps[3];
+  const int32_t* t_begin;   // nullable: then seq_lens[b] - n_tokens
+  const int32_t* seq_lens;
+  int64_t n_tokens;
+  int B, Hkv, d, r;
+  int64_t T_cap;
+  int* status;
+};
+cudaError_t launch_project_keys(const ProjectArgs& a, cudaStream_t s);
+
+struct QprojArgs {
+  const void* Q;  // [B, Hq, d]
+  const float* P; // [Hkv, d, r]
+  float* qs;      // [B*Hkv, r]
+  int B, Hq, Hkv, d, r;
+};
+cudaError_t launch_qproj(const QprojArgs& a, cudaStream_t s);
+
+struct ScoreArgs {
+  const void* Kp;
+  int64_t ps[3];
+  const float* qs;   // [B*Hkv, r]
+  float* scores;     // [B*Hkv, sc_ld]
+  int64_t sc_ld;
+  const int32_t* seq_lens;
+  int B, Hkv, r;
+  int64_t T_cap;
+  int window;
+  int* status;
+};
+cudaError_t launch_score(const ScoreArgs& a, int num_sms, cudaStream_t s);
+
+struct TopkArgs {
+  const float* scores;
+  int64_t sc_ld;
+  const int32_t* seq_lens;
+  int B, Hkv;
+  int64_t T_cap;
+  int k, window;
+  int32_t* idx;     // [B*Hkv, k]
+  int32_t* n_sel;   // [B*Hkv]
+  int* status;
+};
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
+
+struct AttnArgs {
+  const void* Q;    // [B, Hq, dk]
+  const void* K;
+  int64_t ks[3];
+  const void* V;
+  int64_t vs[3];
+  const int32_t* idx;    // nullable => dense range
+  int idx_ld;
+  const int32_t* n_sel;
+  const int32_t* seq_lens;
+  int B, Hq, Hkv, dk, dv;
+  int64_t T_cap;
+  int window;
+  float sm_scale;
+  int64_t list_max;  // host upper bound on the attended list length
+  float* part_o;     // [B, Hq, S, dv]
+  float* part_lse;   // [B, Hq, S]
+  int S, split_len;
+  void* O;           // [B, Hq, dv]
+  float* lse;        // nullable
+  int out_bf16;
+  int* status;
+};
+// Split policy shared by the workspace sizing and the launch.
+void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int num_sms, int* S, int* split_len);
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);   // GQA path
+cudaError_t launch_mla_attention(const AttnArgs& a, cudaStream_t s);  // MLA path
+cudaError_t launch_merge(const AttnArgs& a, cudaStream_t s);
+
+}  // namespace jssa

@@ -1,0 +1,109 @@
+// Projected scoring cache on write: Kp[t] = bf16(K[t] . P_h).
+//
+// "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", §3.1 and
+// §3.4 (a projected-key cache per layer and KV head, used for scoring only) and
+// §E.1 (the newly generated key is projected on write; at most 3.2 % of the step).
+//
+// The products K[t,i] * P[i,j] (bf16 x fp32) are exact in fp64 and are accumulated
+// in fp64, then rounded once to bf16 (nearest, ties to even), so the stored cache
+// equals the rounding of the exact product except when that product lies within
+// about 1e-16 relative of a rounding midpoint.  Per decode step this touches one
+// row per (sequence, KV head); the same kernel fills the whole cache at prefill.
+#include "common.cuh"
+#include "launch.h"
+
+namespace jssa {
+
+// Round a double to bf16, nearest with ties to even, in a single rounding step.
+// Written from the IEEE binary-format definition: bf16 keeps the fp32 exponent
+// range and 7 stored fraction bits; below 2^-126 its spacing is 2^-133.
+__device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
+  const unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(x));
+  const uint16_t sign = static_cast<uint16_t>((u >> 48) & 0x8000u);
+  const unsigned long long a = u & 0x7FFFFFFFFFFFFFFFull;
+  if (a >= 0x7FF0000000000000ull) return (a > 0x7FF0000000000000ull) ? uint16_t(0x7FC0) : uint16_t(sign | 0x7F80);
+  const int e = static_cast<int>(a >> 52) - 1023;
+  if (e >= -126) {
+    unsigned long long keep = a >> 45;  // exponent and the top 7 fraction bits
+    const unsigned long long rem = a & ((1ull << 45) - 1);
+    const unsigned long long half = 1ull << 44;
+    if (rem > half || (rem == half && (keep & 1ull))) keep += 1;
+    const double r = __longlong_as_double(static_cast<long long>(keep << 45));
+    if (r >= 0x1p128) return uint16_t(sign | 0x7F80);
+    return uint16_t(sign | (__float_as_uint(static_cast<float>(r)) >> 16));
+  }
+  const double q = rint(__longlong_as_double(static_cast<long long>(a)) * 0x1p133);  // whole quanta of 2^-133
+  return uint16_t(sign | static_cast<uint16_t>(q));
+}
+
+constexpr int kProjRows = 32;     // rows of K per CTA
+constexpr int kProjThreads = 256;
+
+__global__ void __launch_bounds__(kProjThreads) project_keys_kernel(ProjectArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  __nv_bfloat16* krows = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // [kProjRows][d]
+  const int b = blockIdx.z, h = blockIdx.y;
+  const int d = a.d, r = a.r;
+  int64_t tb;
+  if (a.t_begin) {
+    tb = a.t_begin[b];
+  } else {
+    int64_t T = a.seq_lens[b];
+    if (T < 0 || T > a.T_cap) {
+      if (threadIdx.x == 0) flag_error(a.status, DEVFLAG_BAD_SEQ_LEN);
+      T = T < 0 ? 0 : a.T_cap;
+    }
+    tb = T - a.n_tokens;
+  }
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kProjRows;  // offset within [0, n_tokens)
+  const int nrows = static_cast<int>(min64(kProjRows, a.n_tokens - row0));
+  const __nv_bfloat16* Kb = static_cast<const __nv_bfloat16*>(a.K) + b * a.ks[0] + h * a.ks[1];
+  // stage the rows (16-byte chunks); rows outside [0, T_cap) become zeros and are not stored
+  const int cpr = d / 8;
+  for (int c = threadIdx.x; c < nrows * cpr; c += blockDim.x) {
+    const int rr = c / cpr, ch = c % cpr;
+    const int64_t t = tb + row0 + rr;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (t >= 0 && t < a.T_cap) v = *reinterpret_cast<const uint4*>(Kb + t * a.ks[2] + ch * 8);
+    *reinterpret_cast<uint4*>(krows + rr * d + ch * 8) = v;
+  }
+  __syncthreads();
+  const int groups = kProjThreads / r;   // row groups
+  const int j = threadIdx.x % r, g = threadIdx.x / r;
+  const float* Ph = a.P + static_cast<int64_t>(h) * d * r;
+  constexpr int kMaxRowsPerThread = kProjRows / 4;   // r <= 64 -> at least 4 groups
+  double acc[kMaxRowsPerThread];
+#pragma unroll
+  for (int q = 0; q < kMaxRowsPerThread; ++q) acc[q] = 0.0;
+  const int my_rows = (nrows - g + groups - 1) / groups;  // rows g, g+groups, ...
+  for (int i = 0; i < d; ++i) {
+    const double p = static_cast<double>(__ldg(Ph + static_cast<int64_t>(i) * r + j));
+#pragma unroll
+    for (int q = 0; q < kMaxRowsPerThread; ++q)
+      if (q < my_rows) acc[q] = fma(static_cast<double>(__bfloat162float(krows[(g + q * groups) * d + i])), p, acc[q]);
+  }
+  __nv_bfloat16* Kpb = static_cast<__nv_bfloat16*>(a.Kp) + b * a.ps[0] + h * a.ps[1];
+#pragma unroll
+  for (int q = 0; q < kMaxRowsPerThread; ++q) {
+    if (q < my_rows) {
+      const int64_t t = tb + row0 + g + q * groups;
+      if (t >= 0 && t < a.T_cap) {
+        const uint16_t bits = f64_to_bf16_rne(acc[q]);
+        reinterpret_cast<uint16_t*>(Kpb)[t * a.ps[2] + j] = bits;
+      }
+    }
+  }
+}
+
+cudaError_t launch_project_keys(const ProjectArgs& a, cudaStream_t s) {
+  if (a.n_tokens <= 0) return cudaSuccess;
+  dim3 grid(static_cast<unsigned>(ceil_div(a.n_tokens, kProjRows)), a.Hkv, a.B);
+  const size_t smem = static_cast<size_t>(kProjRows) * a.d * sizeof(__nv_bfloat16);
+  static int done[64] = {0};
+  cudaError_t e = set_smem_limit_once(project_keys_kernel, smem, done);
+  if (e != cudaSuccess) return e;
+  project_keys_kernel<<<grid, kProjThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace jssa

@@ -1,0 +1,209 @@
+// Subspace scoring: projected group query and the full-context score scan.
+//
+// "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", Figure 1
+// and §3.1-§3.2: the group's query heads are projected with the same orthonormal
+// basis as the keys and score every cached position of the projected-key cache;
+// §E.1: this scan grows with batch size and dominates at large batch.
+//
+// qproj:  qs[b,h,:] = sum_g P_h^T q_{hG+g}   (fp32; the group sum is formed first)
+// score:  s[b,h,t]  = qs[b,h,:] . Kp[b,h,t,:] (fp32) for t in [0, T_b - W)
+//
+// The scan is HBM-bound (about r*2 bytes read and 4 bytes written per token).  A
+// persistent grid walks the flattened (row, token) space in 16 KB chunks; one
+// thread per CTA streams chunks into a 4-stage shared-memory ring with 1-D bulk
+// copies (TMA engine, L2 evict-first), completion tracked by mbarriers.  Each chunk
+// is consumed with 16-byte shared loads: r/8 consecutive threads share a token,
+// each holding a fixed 8-wide slice of qs in registers, and reduce by shuffles.
+#include "common.cuh"
+#include "launch.h"
+
+namespace jssa {
+
+// ---------------------------------------------------------------- query projection
+__global__ void __launch_bounds__(256) qproj_kernel(QprojArgs a) {
+  extern __shared__ float qsum[];  // [d]
+  const int row = blockIdx.x;
+  const int b = row / a.Hkv, h = row % a.Hkv;
+  const int G = a.Hq / a.Hkv;
+  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.Q) + (static_cast<int64_t>(b) * a.Hq + h * G) * a.d;
+  for (int i = threadIdx.x; i < a.d; i += blockDim.x) {
+    float s = 0.f;
+    for (int g = 0; g < G; ++g) s += __bfloat162float(Q[static_cast<int64_t>(g) * a.d + i]);
+    qsum[i] = s;
+  }
+  __syncthreads();
+  const float* Ph = a.P + static_cast<int64_t>(h) * a.d * a.r;
+  for (int j = threadIdx.x; j < a.r; j += blockDim.x) {
+    float acc = 0.f;
+    for (int i = 0; i < a.d; ++i) acc = fmaf(__ldg(Ph + static_cast<int64_t>(i) * a.r + j), qsum[i], acc);
+    a.qs[static_cast<int64_t>(row) * a.r + j] = acc;
+  }
+}
+
+cudaError_t launch_qproj(const QprojArgs& a, cudaStream_t s) {
+  qproj_kernel<<<a.B * a.Hkv, 256, a.d * sizeof(float), s>>>(a);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- score scan
+constexpr int kScoreThreads = 256;
+constexpr int kScoreStages = 4;
+constexpr int kChunkBytes = 16384;
+constexpr int kMaxBatch = 1024;
+
+struct ChunkLoc {
+  int row;
+  int64_t t0;
+  int cnt;
+};
+
+template <int R>
+__device__ __forceinline__ ChunkLoc locate_chunk(int64_t c, const int64_t* cum, const int64_t* nb, int B, int Hkv) {
+  constexpr int CH = kChunkBytes / (R * 2);
+  int lo = 0, hi = B - 1;  // last b with cum[b] <= c
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cum[mid] <= c) lo = mid; else hi = mid - 1;
+  }
+  const int b = lo;
+  const int64_t per_head = ceil_div(nb[b], CH);
+  const int64_t local = c - cum[b];
+  const int h = static_cast<int>(local / per_head);
+  const int64_t ci = local % per_head;
+  ChunkLoc L;
+  L.row = b * Hkv + h;
+  L.t0 = ci * CH;
+  L.cnt = static_cast<int>(min64(CH, nb[b] - L.t0));
+  return L;
+}
+
+template <int R>
+__global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreArgs a) {
+  constexpr int CH = kChunkBytes / (R * 2);  // tokens per chunk
+  constexpr int V = R / 8;                    // 16-byte vectors per token = threads per token
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  unsigned char* ring = smem_raw;                                           // [stages][16 KB]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + kScoreStages * kChunkBytes);
+  int64_t* cum = reinterpret_cast<int64_t*>(bars + kScoreStages);           // [B + 1]
+  int64_t* nb = cum + (a.B + 1);                                            // [B]
+
+  const int tid = threadIdx.x;
+  // candidate counts and chunk prefix per batch entry
+  for (int b = tid; b < a.B; b += blockDim.x) {
+    int64_t T = a.seq_lens[b];
+    if (T < 0 || T > a.T_cap) {
+      if (blockIdx.x == 0) flag_error(a.status, DEVFLAG_BAD_SEQ_LEN);
+      T = T < 0 ? 0 : a.T_cap;
+    }
+    const int64_t W = min64(max(a.window, 0), T);
+    nb[b] = T - W;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int64_t c = 0;
+    for (int b = 0; b < a.B; ++b) {
+      cum[b] = c;
+      c += static_cast<int64_t>(a.Hkv) * ceil_div(nb[b], CH);
+    }
+    cum[a.B] = c;
+    for (int s = 0; s < kScoreStages; ++s) mbar_init(&bars[s], 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  const int64_t total = cum[a.B];
+  const int64_t c_begin = total * blockIdx.x / gridDim.x;
+  const int64_t c_end = total * (blockIdx.x + 1) / gridDim.x;
+  const int64_t n_mine = c_end - c_begin;
+  if (n_mine <= 0) return;
+
+  const __nv_bfloat16* Kp = static_cast<const __nv_bfloat16*>(a.Kp);
+  uint64_t policy = 0;
+  auto issue = [&](int64_t it) {
+    const ChunkLoc L = locate_chunk<R>(c_begin + it, cum, nb, a.B, a.Hkv);
+    const int b = L.row / a.Hkv, h = L.row % a.Hkv;
+    const __nv_bfloat16* src = Kp + b * a.ps[0] + h * a.ps[1] + L.t0 * a.ps[2];
+    const uint32_t bytes = static_cast<uint32_t>(L.cnt) * R * 2;
+    const int s = static_cast<int>(it % kScoreStages);
+    mbar_arrive_expect_tx(&bars[s], bytes);
+    bulk_g2s(ring + s * kChunkBytes, src, bytes, &bars[s], policy);
+  };
+  if (tid == 0) {
+    policy = l2_policy_evict_first();
+    for (int64_t it = 0; it < min64(kScoreStages, n_mine); ++it) issue(it);
+  }
+
+  const int vec = tid % V;            // this thread's 8-wide slice of the token
+  float q[8];
+  int cur_row = -1;
+  int64_t it = 0;
+  bool aborted = false;
+  for (; it < n_mine; ++it) {
+    const int s = static_cast<int>(it % kScoreStages);
+    const uint32_t parity = static_cast<uint32_t>((it / kScoreStages) & 1);
+    const bool ok = mbar_wait_bounded(&bars[s], parity, a.status);
+    if (ok) {
+      const ChunkLoc L = locate_chunk<R>(c_begin + it, cum, nb, a.B, a.Hkv);
+      if (L.row != cur_row) {
+        cur_row = L.row;
+        const float4* qp = reinterpret_cast<const float4*>(a.qs + static_cast<int64_t>(cur_row) * R + vec * 8);
+        const float4 q0 = qp[0], q1 = qp[1];
+        q[0] = q0.x; q[1] = q0.y; q[2] = q0.z; q[3] = q0.w;
+        q[4] = q1.x; q[5] = q1.y; q[6] = q1.z; q[7] = q1.w;
+      }
+      const unsigned char* buf = ring + s * kChunkBytes;
+      float* out = a.scores + static_cast<int64_t>(L.row) * a.sc_ld + L.t0;
+#pragma unroll
+      for (int m = 0; m < (CH * V) / kScoreThreads; ++m) {
+        const int slot = tid + m * kScoreThreads;
+        const int tok = slot / V;
+        const uint4 raw = *reinterpret_cast<const uint4*>(buf + static_cast<size_t>(slot) * 16);
+        float acc = 0.f;
+        acc = fmaf(q[0], __uint_as_float(raw.x << 16), acc);
+        acc = fmaf(q[1], __uint_as_float(raw.x & 0xFFFF0000u), acc);
+        acc = fmaf(q[2], __uint_as_float(raw.y << 16), acc);
+        acc = fmaf(q[3], __uint_as_float(raw.y & 0xFFFF0000u), acc);
+        acc = fmaf(q[4], __uint_as_float(raw.z << 16), acc);
+        acc = fmaf(q[5], __uint_as_float(raw.z & 0xFFFF0000u), acc);
+        acc = fmaf(q[6], __uint_as_float(raw.w << 16), acc);
+        acc = fmaf(q[7], __uint_as_float(raw.w & 0xFFFF0000u), acc);
+#pragma unroll
+        for (int off = V / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+        if (vec == 0 && tok < L.cnt) out[tok] = acc;
+      }
+    }
+    // one barrier per chunk: everyone is done with stage s, and all agree on a timeout
+    if (__syncthreads_or(!ok)) { aborted = true; break; }
+    if (tid == 0 && it + kScoreStages < n_mine) issue(it + kScoreStages);
+  }
+  if (aborted && tid == 0) {
+    // give every copy still in flight a bounded chance to land before the CTA exits
+    for (int64_t j = it; j < min64(it + kScoreStages, n_mine); ++j) {
+      const int s = static_cast<int>(j % kScoreStages);
+      mbar_wait_bounded(&bars[s], static_cast<uint32_t>((j / kScoreStages) & 1), a.status, 100000000ull);
+    }
+  }
+}
+
+template <int R>
+static cudaError_t launch_score_r(const ScoreArgs& a, int num_sms, cudaStream_t s) {
+  const size_t smem = kScoreStages * kChunkBytes + kScoreStages * sizeof(uint64_t) + (2 * a.B + 1) * sizeof(int64_t);
+  static int done[64] = {0};
+  cudaError_t e = set_smem_limit_once(score_kernel<R>, smem, done);
+  if (e != cudaSuccess) return e;
+  const int grid = num_sms * 3;
+  score_kernel<R><<<grid, kScoreThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_score(const ScoreArgs& a, int num_sms, cudaStream_t s) {
+  if (a.B > kMaxBatch) return cudaErrorInvalidValue;
+  switch (a.r) {
+    case 8: return launch_score_r<8>(a, num_sms, s);
+    case 16: return launch_score_r<16>(a, num_sms, s);
+    case 32: return launch_score_r<32>(a, num_sms, s);
+    case 64: return launch_score_r<64>(a, num_sms, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace jssa
