@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark of the JSSA decode step on B200 (one JSON line on rank 0).
+
+Workload (default, ``--workload h128k``): the 128K headline GQA layer — B=4, Hq=32,
+Hkv=8, d=128, r=32, T=131072 cached tokens, top-k budget k=2048, bf16 K/V/Q, synthetic
+caches from the seeded generator (token_level_sparse_jssa_b200.synth).  One step =
+project the newest key into the scoring cache, project the group queries, scan all
+T projected keys, select the top-k per (sequence, KV head), attend over the selected
+rows in place and merge the split partials.  Every timed step uses a fresh query
+batch, so every step selects a different token set.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+
+N > 1 runs under torchrun: each rank owns an independent batch of sequences (weak
+scaling, no collective on the data path); time is the max over ranks.
+``--impl reference`` times the CPU oracle (fp64, single-threaded) on a bounded sample
+of the same workload on this host instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode steps/s and µs/step at 128K (1×B200); % of HBM roofline; × vs own dense kernel"
+UNIT = "steps/s"
+KERNELS_PER_STEP = 6  # project_keys, qproj, score, topk, attention, merge
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="jssa", choices=["jssa", "reference"])
+    ap.add_argument("--workload", default="h128k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------- helpers
+def byte_model(w, T, k, window, out_bytes=2):
+    """Algorithmic bytes of one step and of the dense step (HBM roofline numerator)."""
+    n = T - min(window, T)
+    keff = min(k, n)
+    rows = w.B * w.Hkv
+    kp = rows * n * w.r * 2
+    kv_row = (w.dk if w.mode == "mla" else w.dk + w.dv) * 2
+    sel = rows * (keff + min(window, T)) * kv_row
+    qo = w.B * w.Hq * (w.dk * 2 + w.dv * out_bytes)
+    dense = rows * T * kv_row + qo
+    return dict(kp=kp, selected=sel, qo=qo, step=kp + sel + qo, dense=dense, scores=rows * n * 4)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "token_level_sparse_jssa_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str, src_hash: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        d = json.load(open(p))
+        e = d[kernel][workload]
+        return e["bytes_per_launch"] if e.get("source_hash") == src_hash else None
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while the timed region runs."""
+
+    def __init__(self, dev_index: int, period=0.01):
+        self.period, self.samples, self.reasons = period, [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(dev_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = nv.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.nv = nv
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+            "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+            "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, bit in names.items():
+                    if r & bit and k != "gpu_idle":
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- workload setup
+class Setup:
+    def __init__(self, w, device, seed_offset=0):
+        import token_level_sparse_jssa_b200 as jssa
+        from token_level_sparse_jssa_b200 import synth
+        self.jssa, self.w = jssa, w
+        x = synth.make_inputs(w, device=device, seed=w.seed + seed_offset)
+        self.T_cap = x["T_cap"]
+        self.K = x["K"]
+        self.V = self.K[..., : w.dv] if w.mode == "mla" else x["V"]
+        self.P = x["P"].contiguous()
+        self.seq_lens = x["seq_lens"]
+        self.A = x["A"]
+        self.Kp = torch.empty(w.B, w.Hkv, self.T_cap, w.r, dtype=torch.bfloat16, device=device)
+        self.L = jssa.make_layout(self.K, self.V, self.Kp, w.Hq, w.r,
+                                  jssa.MODE_MLA if w.mode == "mla" else jssa.MODE_GQA, jssa.OUT_BF16)
+        tb = torch.zeros(w.B, dtype=torch.int32, device=device)
+        jssa.project_keys(self.L, self.K, self.P, self.Kp, self.T_cap, t_begin=tb)   # prefill fill
+        self.ws = jssa.alloc_workspace(self.L, w.k, w.window)
+        self.O = torch.empty(w.B, w.Hq, w.dv, dtype=torch.bfloat16, device=device)
+        self.idx = torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=device)
+        self.nsel = torch.empty(w.B, w.Hkv, dtype=torch.int32, device=device)
+        torch.cuda.synchronize()
+
+    def step(self, Q):
+        w = self.w
+        self.jssa.decode_step(self.L, Q, self.K, self.V, self.Kp, self.P, self.seq_lens, 1, w.k, w.window,
+                              w.sm_scale, self.O, None, self.idx, self.nsel, self.ws)
+
+    def dense(self, Q):
+        self.jssa.dense_decode(self.L, Q, self.K, self.V, self.seq_lens, 0, self.w.sm_scale, self.O, None, self.ws)
+
+
+def graph_of(fn, qs):
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for q in qs:
+                fn(q)
+    torch.cuda.current_stream().wait_stream(s)
+    return g
+
+
+def timed_graph(g, barrier):
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    return e0.elapsed_time(e1)
+
+
+def stage_times(st, Q, reps=50):
+    """Per-stage device time (eager launches, CUDA events on the launching stream)."""
+    jssa, w = st.jssa, st.w
+    scores = st.ws  # not used directly: the stage calls below use their own outputs
+    sc = torch.empty(w.B, w.Hkv, st.T_cap, device="cuda")
+    out = {}
+
+    def t(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1000.0 / reps
+
+    out["project_us"] = t(lambda: jssa.project_keys(st.L, st.K, st.P, st.Kp, 1, seq_lens=st.seq_lens))
+    out["score_us"] = t(lambda: jssa.score(st.L, Q, st.P, st.Kp, st.seq_lens, w.window, sc, st.ws))
+    out["topk_us"] = t(lambda: jssa.topk(st.L, sc, st.seq_lens, w.k, w.window, st.idx, st.nsel, st.ws))
+    out["attention_us"] = t(lambda: jssa.indexed_attn(st.L, Q, st.K, st.V, st.idx, w.k, st.nsel, st.seq_lens,
+                                                      w.window, w.sm_scale, st.O, None, st.ws))
+    return out
+
+
+# --------------------------------------------------------------------------- CPU oracle timing
+def cpu_oracle_rate(w, seconds: float, data=None):
+    """Time the fp64 oracle's decode step on sampled (sequence, KV head) rows of the workload
+    on this host (single thread) for about ``seconds``; returns (steps/s, description)."""
+    import numpy as np
+    import oracle
+    from token_level_sparse_jssa_b200 import synth
+    from tests._util import u16, f32
+    if data is None:
+        # a bounded sample of the workload: sequence 0 only (its Hkv rows)
+        x = synth.make_inputs(w.with_(B=1), device="cuda" if torch.cuda.is_available() else "cpu")
+        K, V, Q, P = x["K"], (x["K"][..., : w.dv] if w.mode == "mla" else x["V"]), x["Q"], x["P"]
+    else:
+        K, V, Q, P = data
+    rows = [(0, h) for h in range(min(2, w.Hkv))]
+    G, T = w.G, w.T
+    host = []
+    for (b, h) in rows:
+        Kh, Vh = u16(K[b, h, :T]), u16(V[b, h, :T])
+        Ph = f32(P[h])
+        Kp, _ = oracle.project_rows(Kh, Ph)       # cache state before the step (not timed)
+        host.append((u16(Q[b, h * G:(h + 1) * G]), Kh, Vh, Kp, Ph))
+    n, t0 = 0, time.perf_counter()
+    while True:
+        for (Qg, Kh, Vh, Kp, Ph) in host:
+            oracle.project_rows(Kh[T - 1:T], Ph)  # the newest key, projected on write
+            oracle.decode_head(Qg, Kh, Vh, Kp, Ph, T, w.k, w.window, w.sm_scale)
+            n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    per_row = el / n
+    step_s = per_row * w.B * w.Hkv
+    desc = (f"{n} (sequence, KV-head) problems of the {w.name} step ({len(rows)} distinct rows of sequence 0, "
+            f"T={T}, k={w.k}) in {el:.1f} s on 1 thread; one step = {w.B * w.Hkv} such problems")
+    return 1.0 / step_s, desc
+
+
+# --------------------------------------------------------------------------- arms
+def run_reference(args, w, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rate, desc = cpu_oracle_rate(w, max(5.0, args.cpu_seconds))
+    line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / rate, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+            "cpu_baseline": {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+            "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    from token_level_sparse_jssa_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    bm = byte_model(w, w.T, w.k, w.window)
+    cfg = {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} d_k={w.dk} d_v={w.dv} r={w.r} T={w.T} k={w.k}"
+                       + (f" W={w.window}" if w.window else "") + f" ({w.mode.upper()})",
+           "global_batch": w.B * max(world, args.gpus), "seq_len": w.T, "k": w.k, "r": w.r,
+           "parallelism": f"dp{max(world, args.gpus)} (independent sequences per rank, no collective)",
+           "l2": "inputs larger than L2 (the projected cache alone is %.0f MB per step) and a fresh query every step"
+                 % (bm["kp"] / 1e6)}
+    if args.impl == "reference":
+        return run_reference(args, w, cfg)
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    st = Setup(w, "cuda", seed_offset=rank)
+    nq = args.warmup + args.steps
+    Qs = synth.fresh_queries(w, nq, st.A, device="cuda", seed=7 + rank)
+    # warm-up (untimed), then exactly `steps` timed steps, each in one CUDA graph
+    g_warm = graph_of(st.step, [Qs[i] for i in range(args.warmup)])
+    g_warm.replay()
+    torch.cuda.synchronize()
+    g_timed = graph_of(st.step, [Qs[args.warmup + i] for i in range(args.steps)])
+    with ClockSampler(local) as clk:
+        ms = timed_graph(g_timed, barrier)
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = world * args.steps / (ms / 1000.0)
+    del g_warm, g_timed
+
+    # dense full-KV comparator at the same shape
+    nd = max(5, min(200, args.steps // 10))
+    g_dw = graph_of(st.dense, [Qs[i] for i in range(3)])
+    g_dw.replay()
+    g_d = graph_of(st.dense, [Qs[i % nq] for i in range(nd)])
+    dense_ms = timed_graph(g_d, barrier) / nd
+    del g_dw, g_d
+
+    stages = stage_times(st, Qs[0])
+    hbm, peak_kind = peaks()
+    score_bytes = bm["kp"] + bm["scores"]
+    score_s = stages["score_us"] * 1e-6
+    shash = source_hash("score.cu", "common.cuh")
+
+    # end to end through the public API with host buffers: per step, H2D of the query and of
+    # the newest token's K/V rows from pinned memory, the step, and D2H of the output
+    ne = max(10, min(500, args.steps // 4))
+    Qh = Qs[:ne].cpu().pin_memory()
+    newk = st.K[:, :, w.T - 1].contiguous().cpu().pin_memory()
+    newv = st.V[:, :, w.T - 1].contiguous().cpu().pin_memory() if w.mode != "mla" else None
+    Oh = torch.empty(st.O.shape, dtype=st.O.dtype).pin_memory()
+    Qd = torch.empty_like(Qs[0])
+    for i in range(3):
+        Qd.copy_(Qh[i], non_blocking=True)
+        st.step(Qd)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(ne):
+        Qd.copy_(Qh[i], non_blocking=True)
+        st.K[:, :, w.T - 1].copy_(newk, non_blocking=True)
+        if newv is not None:
+            st.V[:, :, w.T - 1].copy_(newv, non_blocking=True)
+        st.step(Qd)
+        Oh.copy_(st.O, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = Qd.numel() * 2 + newk.numel() * 2 + (newv.numel() * 2 if newv is not None else 0)
+    d2h = Oh.numel() * Oh.element_size()
+
+    code, flags = st.jssa.read_device_status(st.ws)
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            rate, desc = cpu_oracle_rate(w, args.cpu_seconds, data=(st.K, st.V, Qs[0], st.P))
+            cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+        achieved = score_bytes / score_s / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "us_per_step": ms_step * 1000.0, "tokens_per_s": value * w.B,
+            "bytes_per_step": bm["step"], "effective_GBps": bm["step"] / (ms_step * 1e-3) / 1e9,
+            "step_hbm_frac": bm["step"] / (ms_step * 1e-3) / 1e9 / hbm,
+            "dense_us_per_step": dense_ms * 1000.0, "speedup_vs_dense": dense_ms / ms_step,
+            "byte_ratio": bm["dense"] / bm["step"],
+            "dense_hbm_frac": bm["dense"] / (dense_ms * 1e-3) / 1e9 / hbm,
+            "stage_us": stages,
+            "roofline": {"kernel": "score_kernel", "bound": "hbm", "achieved": achieved, "peak": hbm,
+                         "unit": "GB/s", "frac": achieved / hbm, "peak_kind": peak_kind,
+                         "traffic": traffic_for("score_kernel", w.name, shash),
+                         "algorithmic_bytes_per_launch": score_bytes},
+            "cpu_baseline": cpu,
+            "e2e": {"value": ne / (e2e_ms / 1000.0) * world, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "clocks": clk.summary(),
+            "device_status": flags,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

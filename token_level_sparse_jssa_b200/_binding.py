@@ -76,6 +76,7 @@ def load(path: str = LIB_PATH):
 
 
 def _p(t):
+    """Device pointer of a cache tensor (strides are described by the layout)."""
     if t is None:
         return None
     if not isinstance(t, torch.Tensor):
@@ -83,6 +84,13 @@ def _p(t):
     if not t.is_cuda:
         raise ValueError("device tensor expected")
     return t.data_ptr()
+
+
+def _c(t):
+    """Device pointer of a tensor the C ABI reads as densely packed (Q, O, P, idx, ...)."""
+    if isinstance(t, torch.Tensor) and not t.is_contiguous():
+        raise ValueError(f"contiguous tensor expected, got strides {t.stride()} for shape {tuple(t.shape)}")
+    return _p(t)
 
 
 def _stream(stream):
@@ -141,41 +149,41 @@ def alloc_workspace(L: Layout, k: int, window: int = 0, device=None) -> torch.Te
 
 
 def project_keys(L, K, P, Kp, n_tokens: int, t_begin=None, seq_lens=None, stream=None):
-    _check("jssa_project_keys", load().jssa_project_keys(C.byref(L), _p(K), _p(P), _p(Kp), _p(t_begin),
-                                                         _p(seq_lens), n_tokens, _stream(stream)))
+    _check("jssa_project_keys", load().jssa_project_keys(C.byref(L), _p(K), _c(P), _p(Kp), _c(t_begin),
+                                                         _c(seq_lens), n_tokens, _stream(stream)))
 
 
 def score(L, Q, P, Kp, seq_lens, window: int, scores, ws, stream=None):
     w, n = _ws(ws)
-    _check("jssa_score", load().jssa_score(C.byref(L), _p(Q), _p(P), _p(Kp), _p(seq_lens), window, _p(scores),
+    _check("jssa_score", load().jssa_score(C.byref(L), _c(Q), _c(P), _p(Kp), _c(seq_lens), window, _c(scores),
                                            w, n, _stream(stream)))
 
 
 def topk(L, scores, seq_lens, k: int, window: int, idx, n_sel, ws=None, stream=None):
     w, n = _ws(ws)
-    _check("jssa_topk", load().jssa_topk(C.byref(L), _p(scores), _p(seq_lens), k, window, _p(idx), _p(n_sel),
+    _check("jssa_topk", load().jssa_topk(C.byref(L), _c(scores), _c(seq_lens), k, window, _c(idx), _c(n_sel),
                                          w, n, _stream(stream)))
 
 
 def indexed_attn(L, Q, K, V, idx, k: int, n_sel, seq_lens, window: int, sm_scale: float, O, lse, ws, stream=None):
     w, n = _ws(ws)
-    _check("jssa_indexed_attn", load().jssa_indexed_attn(C.byref(L), _p(Q), _p(K), _p(V), _p(idx), k, _p(n_sel),
-                                                         _p(seq_lens), window, sm_scale, _p(O), _p(lse), w, n,
+    _check("jssa_indexed_attn", load().jssa_indexed_attn(C.byref(L), _c(Q), _p(K), _p(V), _c(idx), k, _c(n_sel),
+                                                         _c(seq_lens), window, sm_scale, _c(O), _c(lse), w, n,
                                                          _stream(stream)))
 
 
 def decode_step(L, Q, K, V, Kp, P, seq_lens, n_new: int, k: int, window: int, sm_scale: float, O, lse=None,
                 idx_out=None, n_sel_out=None, ws=None, stream=None):
     w, n = _ws(ws)
-    _check("jssa_decode_step", load().jssa_decode_step(C.byref(L), _p(Q), _p(K), _p(V), _p(Kp), _p(P),
-                                                       _p(seq_lens), n_new, k, window, sm_scale, _p(O), _p(lse),
-                                                       _p(idx_out), _p(n_sel_out), w, n, _stream(stream)))
+    _check("jssa_decode_step", load().jssa_decode_step(C.byref(L), _c(Q), _p(K), _p(V), _p(Kp), _c(P),
+                                                       _c(seq_lens), n_new, k, window, sm_scale, _c(O), _c(lse),
+                                                       _c(idx_out), _c(n_sel_out), w, n, _stream(stream)))
 
 
 def dense_decode(L, Q, K, V, seq_lens, window: int, sm_scale: float, O, lse=None, ws=None, stream=None):
     w, n = _ws(ws)
-    _check("jssa_dense_decode", load().jssa_dense_decode(C.byref(L), _p(Q), _p(K), _p(V), _p(seq_lens), window,
-                                                         sm_scale, _p(O), _p(lse), w, n, _stream(stream)))
+    _check("jssa_dense_decode", load().jssa_dense_decode(C.byref(L), _c(Q), _p(K), _p(V), _c(seq_lens), window,
+                                                         sm_scale, _c(O), _c(lse), w, n, _stream(stream)))
 
 
 def workspace_init(ws, stream=None):

@@ -139,20 +139,33 @@ def make_inputs(w: Workload, device="cpu", T_cap: int | None = None, seq_lens=No
         Ah = A.repeat_interleave(G, dim=0)                      # [Hq, R, d]
         q = torch.einsum("bhr,hrd->bhd", zq, Ah) + 0.3 * torch.randn(B, Hq, d, generator=g, **f32)
         Q = (q / math.sqrt(d)).to(torch.bfloat16)
+    Q = Q.contiguous()
     P = torch.stack([orthonormal_basis(w.dk, w.r, seed * 1000 + h) for h in range(Hkv)]).to(device)
     if seq_lens is None:
         seq_lens = [min(w.T, T_cap)] * B
     sl = torch.as_tensor(seq_lens, dtype=torch.int32, device=device)
-    return dict(Q=Q, K=K, V=V, P=P, seq_lens=sl, T_cap=T_cap)
+    return dict(Q=Q, K=K, V=V, P=P, seq_lens=sl, T_cap=T_cap, A=A)
 
 
-def fresh_queries(w: Workload, n: int, device="cpu", seed: int = 0) -> torch.Tensor:
-    """``n`` independent query batches [n, B, Hq, dk] (bf16) with the workload's statistics
-    in the subspace-free part only (isotropic N(0,1)/sqrt(dk)); used to vary the query
-    from step to step so that every timed step selects a different set."""
+def fresh_queries(w: Workload, n: int, A: torch.Tensor, device="cpu", seed: int = 0) -> torch.Tensor:
+    """``n`` further query batches [n, B, Hq, dk] (bf16) drawn with the workload's query
+    recipe and latent bases ``A`` (as returned by make_inputs); used to vary the query
+    from step to step so that every timed step selects a different token set."""
     g = _gen(device, seed)
-    q = torch.randn(n, w.B, w.Hq, w.dk, generator=g, device=device, dtype=torch.float32)
-    return (q / math.sqrt(w.dk)).to(torch.bfloat16)
+    f32 = dict(device=device, dtype=torch.float32)
+    B, Hq = w.B, w.Hq
+    A = A.to(device)
+    if w.mode == "mla":
+        dl = w.dv
+        zq = torch.randn(n, B, Hq, w.R, generator=g, **f32)
+        qlat = zq @ A + 0.3 * torch.randn(n, B, Hq, dl, generator=g, **f32)
+        qrope = torch.randn(n, B, Hq, w.dk - dl, generator=g, **f32)
+        q = torch.cat([qlat, qrope], dim=3)
+    else:
+        Ah = A.repeat_interleave(w.G, dim=0)                     # [Hq, R, d]
+        zq = torch.randn(n, B, Hq, w.R, generator=g, **f32)
+        q = torch.einsum("nbhr,hrd->nbhd", zq, Ah) + 0.3 * torch.randn(n, B, Hq, w.dk, generator=g, **f32)
+    return (q / math.sqrt(w.dk)).to(torch.bfloat16).contiguous()
 
 
 def random_scores(rows: int, n: int, device="cpu", seed: int = 0, ties: int = 0,
@@ -166,7 +179,7 @@ def random_scores(rows: int, n: int, device="cpu", seed: int = 0, ties: int = 0,
         for _ in range(ties):
             m = int(torch.randint(2, 9, (1,), generator=g))
             pos = torch.randperm(n, generator=g)[:m]
-            s[i, pos] = s[i, pos[0]]
+            s[i, pos] = float(s[i, pos[0]])
         if zeros:
             pos = torch.randperm(n, generator=g)[:zeros]
             s[i, pos] = 0.0
