@@ -35,7 +35,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode steps/s and µs/step at 128K (1×B200); % of HBM roofline; × vs own dense kernel"
 UNIT = "steps/s"
-KERNELS_PER_STEP = 6  # project_keys, qproj, score, topk, attention, merge
+KERNELS_PER_STEP = 5  # prologue (qs + newest key), score, topk, attention, merge
 
 
 def parse():

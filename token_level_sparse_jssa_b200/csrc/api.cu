@@ -14,6 +14,7 @@ namespace {
 constexpr size_t kAlign = 256;
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxK = 1 << 24;
+constexpr int kMaxPrologueRows = 16;  // appended rows projected inside the step prologue
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -148,19 +149,30 @@ ProjectArgs project_args(const jssa_layout* L, const void* K, const float* P, vo
   return a;
 }
 
-jssa_status run_score(const jssa_layout* L, const void* Q, const float* P, const void* Kp, const int32_t* seq_lens,
-                      int window, float* scores, int64_t sc_ld, const Workspace& w, cudaStream_t s) {
-  QprojArgs q{};
+jssa_status run_prologue(const jssa_layout* L, const void* Q, const float* P, const void* K, void* Kp,
+                         const int32_t* seq_lens, int n_new, const Workspace& w, cudaStream_t s) {
+  PrologueArgs q{};
   q.Q = Q;
   q.P = P;
   q.qs = w.qs;
+  q.K = K;
+  memcpy(q.ks, L->k_stride, sizeof q.ks);
+  q.Kp = Kp;
+  memcpy(q.ps, L->kp_stride, sizeof q.ps);
+  q.seq_lens = seq_lens;
+  q.n_new = n_new;
   q.B = L->B;
   q.Hq = L->Hq;
   q.Hkv = L->Hkv;
   q.d = L->d_k;
   q.r = L->r;
-  jssa_status st = cu(launch_qproj(q, s));
-  if (st != JSSA_OK) return st;
+  q.T_cap = L->T_cap;
+  q.status = w.status;
+  return cu(launch_step_prologue(q, s));
+}
+
+jssa_status run_score(const jssa_layout* L, const void* Kp, const int32_t* seq_lens, int window, float* scores,
+                      int64_t sc_ld, const Workspace& w, cudaStream_t s) {
   ScoreArgs a{};
   a.Kp = Kp;
   memcpy(a.ps, L->kp_stride, sizeof a.ps);
@@ -285,7 +297,10 @@ jssa_status jssa_score(const jssa_layout* L, const void* Q, const float* P, cons
   Workspace w{};
   st = get_ws(L, 1, window, workspace, ws_bytes, &w);
   if (st != JSSA_OK) return st;
-  return run_score(L, Q, P, Kp, seq_lens, window, scores, L->T_cap, w, static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = run_prologue(L, Q, P, nullptr, nullptr, seq_lens, 0, w, s);
+  if (st != JSSA_OK) return st;
+  return run_score(L, Kp, seq_lens, window, scores, L->T_cap, w, s);
 }
 
 jssa_status jssa_topk(const jssa_layout* L, const float* scores, const int32_t* seq_lens, int32_t k, int32_t window,
@@ -336,12 +351,14 @@ jssa_status jssa_decode_step(const jssa_layout* L, const void* Q, const void* K,
   st = get_ws(L, k, window, workspace, ws_bytes, &w);
   if (st != JSSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (n_new > 0) {
+  if (n_new > kMaxPrologueRows) {  // long appends go through the bulk projection kernel
     ProjectArgs pa = project_args(L, K, P, Kp, nullptr, seq_lens, n_new, w.status);
     st = cu(launch_project_keys(pa, s));
     if (st != JSSA_OK) return st;
   }
-  st = run_score(L, Q, P, Kp, seq_lens, window, w.scores, L->T_cap, w, s);
+  st = run_prologue(L, Q, P, K, Kp, seq_lens, n_new > kMaxPrologueRows ? 0 : n_new, w, s);
+  if (st != JSSA_OK) return st;
+  st = run_score(L, Kp, seq_lens, window, w.scores, L->T_cap, w, s);
   if (st != JSSA_OK) return st;
   int32_t* idx = idx_out ? idx_out : w.idx;
   int32_t* nsel = n_sel_out ? n_sel_out : w.n_sel;

@@ -22,13 +22,23 @@ struct ProjectArgs {
 };
 cudaError_t launch_project_keys(const ProjectArgs& a, cudaStream_t s);
 
-struct QprojArgs {
+// Per-step prologue: projected group queries qs, plus the projection of the newest
+// n_new (<= 16) rows of each sequence into Kp.
+struct PrologueArgs {
   const void* Q;  // [B, Hq, d]
   const float* P; // [Hkv, d, r]
   float* qs;      // [B*Hkv, r]
+  const void* K;
+  int64_t ks[3];
+  void* Kp;
+  int64_t ps[3];
+  const int32_t* seq_lens;
+  int n_new;
   int B, Hq, Hkv, d, r;
+  int64_t T_cap;
+  int* status;
 };
-cudaError_t launch_qproj(const QprojArgs& a, cudaStream_t s);
+cudaError_t launch_step_prologue(const PrologueArgs& a, cudaStream_t s);
 
 struct ScoreArgs {
   const void* Kp;

@@ -1,14 +1,24 @@
-// Projected scoring cache on write: Kp[t] = bf16(K[t] . P_h).
+// Projected scoring cache on write, and the step prologue.
 //
 // "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", §3.1 and
-// §3.4 (a projected-key cache per layer and KV head, used for scoring only) and
-// §E.1 (the newly generated key is projected on write; at most 3.2 % of the step).
+// §3.4 (a projected-key cache per layer and KV head, used for scoring only), §3.2
+// (one basis for queries and keys) and §E.1 (the newly generated key is projected on
+// write; at most 3.2 % of the step).
 //
-// The products K[t,i] * P[i,j] (bf16 x fp32) are exact in fp64 and are accumulated
-// in fp64, then rounded once to bf16 (nearest, ties to even), so the stored cache
-// equals the rounding of the exact product except when that product lies within
-// about 1e-16 relative of a rounding midpoint.  Per decode step this touches one
-// row per (sequence, KV head); the same kernel fills the whole cache at prefill.
+// Kp[t] = bf16(K[t] . P_h): the products K[t,i] * P[i,j] (bf16 x fp32) are exact in
+// fp64 and are accumulated in fp64, then rounded once to bf16 (nearest, ties to
+// even), so the stored cache equals the rounding of the exact product except when
+// that product lies within about 1e-16 relative of a rounding midpoint.
+//
+// Two kernels:
+//   project_keys_kernel  — many rows (the prefill fill of the cache): 32 rows per CTA,
+//                          P_h and the rows staged in shared memory.
+//   step_prologue_kernel — one CTA per (sequence, KV head) per decode step: stages
+//                          P_h once, forms the projected group query
+//                          qs = sum_g P_h^T q_g (fp32; the group sum first) and
+//                          projects the newest row(s) into Kp; every output column is
+//                          split over 256/r threads whose partial sums are added in a
+//                          fixed order.
 #include "common.cuh"
 #include "launch.h"
 
@@ -36,14 +46,22 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
   return uint16_t(sign | static_cast<uint16_t>(q));
 }
 
+// Stage P_h [d][r] (fp32) into shared memory with 16-byte loads.
+__device__ __forceinline__ void stage_basis(float* Psm, const float* Ph, int n) {
+  const float4* src = reinterpret_cast<const float4*>(Ph);
+  float4* dst = reinterpret_cast<float4*>(Psm);
+  for (int i = threadIdx.x; i < n / 4; i += blockDim.x) dst[i] = __ldg(src + i);
+}
+
 constexpr int kProjRows = 32;     // rows of K per CTA
 constexpr int kProjThreads = 256;
 
 __global__ void __launch_bounds__(kProjThreads) project_keys_kernel(ProjectArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  __nv_bfloat16* krows = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // [kProjRows][d]
-  const int b = blockIdx.z, h = blockIdx.y;
   const int d = a.d, r = a.r;
+  float* Psm = reinterpret_cast<float*>(smem_raw);                                 // [d][r]
+  __nv_bfloat16* krows = reinterpret_cast<__nv_bfloat16*>(Psm + d * r);          // [kProjRows][d]
+  const int b = blockIdx.z, h = blockIdx.y;
   int64_t tb;
   if (a.t_begin) {
     tb = a.t_begin[b];
@@ -55,6 +73,7 @@ __global__ void __launch_bounds__(kProjThreads) project_keys_kernel(ProjectArgs 
     }
     tb = T - a.n_tokens;
   }
+  stage_basis(Psm, a.P + static_cast<int64_t>(h) * d * r, d * r);
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kProjRows;  // offset within [0, n_tokens)
   const int nrows = static_cast<int>(min64(kProjRows, a.n_tokens - row0));
   const __nv_bfloat16* Kb = static_cast<const __nv_bfloat16*>(a.K) + b * a.ks[0] + h * a.ks[1];
@@ -70,14 +89,14 @@ __global__ void __launch_bounds__(kProjThreads) project_keys_kernel(ProjectArgs 
   __syncthreads();
   const int groups = kProjThreads / r;   // row groups
   const int j = threadIdx.x % r, g = threadIdx.x / r;
-  const float* Ph = a.P + static_cast<int64_t>(h) * d * r;
   constexpr int kMaxRowsPerThread = kProjRows / 4;   // r <= 64 -> at least 4 groups
   double acc[kMaxRowsPerThread];
 #pragma unroll
   for (int q = 0; q < kMaxRowsPerThread; ++q) acc[q] = 0.0;
   const int my_rows = (nrows - g + groups - 1) / groups;  // rows g, g+groups, ...
+#pragma unroll 4
   for (int i = 0; i < d; ++i) {
-    const double p = static_cast<double>(__ldg(Ph + static_cast<int64_t>(i) * r + j));
+    const double p = static_cast<double>(Psm[i * r + j]);
 #pragma unroll
     for (int q = 0; q < kMaxRowsPerThread; ++q)
       if (q < my_rows) acc[q] = fma(static_cast<double>(__bfloat162float(krows[(g + q * groups) * d + i])), p, acc[q]);
@@ -87,10 +106,7 @@ __global__ void __launch_bounds__(kProjThreads) project_keys_kernel(ProjectArgs 
   for (int q = 0; q < kMaxRowsPerThread; ++q) {
     if (q < my_rows) {
       const int64_t t = tb + row0 + g + q * groups;
-      if (t >= 0 && t < a.T_cap) {
-        const uint16_t bits = f64_to_bf16_rne(acc[q]);
-        reinterpret_cast<uint16_t*>(Kpb)[t * a.ps[2] + j] = bits;
-      }
+      if (t >= 0 && t < a.T_cap) reinterpret_cast<uint16_t*>(Kpb)[t * a.ps[2] + j] = f64_to_bf16_rne(acc[q]);
     }
   }
 }
@@ -98,11 +114,85 @@ __global__ void __launch_bounds__(kProjThreads) project_keys_kernel(ProjectArgs 
 cudaError_t launch_project_keys(const ProjectArgs& a, cudaStream_t s) {
   if (a.n_tokens <= 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>(ceil_div(a.n_tokens, kProjRows)), a.Hkv, a.B);
-  const size_t smem = static_cast<size_t>(kProjRows) * a.d * sizeof(__nv_bfloat16);
+  const size_t smem = static_cast<size_t>(a.d) * a.r * sizeof(float) +
+                      static_cast<size_t>(kProjRows) * a.d * sizeof(__nv_bfloat16);
   static int done[64] = {0};
   cudaError_t e = set_smem_limit_once(project_keys_kernel, smem, done);
   if (e != cudaSuccess) return e;
   project_keys_kernel<<<grid, kProjThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ step prologue
+constexpr int kPrologueThreads = 256;
+constexpr int kMaxNewRowsInPrologue = 16;
+
+__global__ void __launch_bounds__(kPrologueThreads) step_prologue_kernel(PrologueArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int d = a.d, r = a.r;
+  float* Psm = reinterpret_cast<float*>(smem_raw);              // [d][r]
+  float* vec = Psm + d * r;                                      // [d]  group-summed query / key row
+  double* red = reinterpret_cast<double*>(vec + d + (d & 1));    // [parts][r] partial sums
+  const int row = blockIdx.x;
+  const int b = row / a.Hkv, h = row % a.Hkv;
+  const int G = a.Hq / a.Hkv;
+  const int tid = threadIdx.x;
+  stage_basis(Psm, a.P + static_cast<int64_t>(h) * d * r, d * r);
+  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.Q) + (static_cast<int64_t>(b) * a.Hq + h * G) * d;
+  for (int i = tid; i < d; i += blockDim.x) {
+    float s = 0.f;
+#pragma unroll 8
+    for (int g = 0; g < G; ++g) s += __bfloat162float(Q[static_cast<int64_t>(g) * d + i]);
+    vec[i] = s;
+  }
+  __syncthreads();
+  // output column j = tid % r; this thread sums i = part, part + parts, ... (conflict-free
+  // shared loads: a warp reads consecutive columns of one row of P)
+  const int parts = kPrologueThreads / r, j = tid % r, part = tid / r;
+  {
+    float acc = 0.f;
+    for (int i = part; i < d; i += parts) acc = fmaf(Psm[i * r + j], vec[i], acc);
+    red[part * r + j] = acc;
+    __syncthreads();
+    if (tid < r) {
+      float s = 0.f;
+      for (int q = 0; q < parts; ++q) s += static_cast<float>(red[q * r + tid]);
+      a.qs[static_cast<int64_t>(row) * r + tid] = s;
+    }
+  }
+  if (a.n_new <= 0) return;
+  // project the newest n_new rows [T_b - n_new, T_b) of this (sequence, KV head)
+  int64_t T = a.seq_lens[b];
+  if (T < 0 || T > a.T_cap) {
+    if (tid == 0) flag_error(a.status, DEVFLAG_BAD_SEQ_LEN);
+    T = T < 0 ? 0 : a.T_cap;
+  }
+  const __nv_bfloat16* Kb = static_cast<const __nv_bfloat16*>(a.K) + b * a.ks[0] + h * a.ks[1];
+  uint16_t* Kpb = reinterpret_cast<uint16_t*>(a.Kp) + b * a.ps[0] + h * a.ps[1];
+  for (int64_t t = max64(0, T - a.n_new); t < T; ++t) {
+    __syncthreads();  // vec and red are free again
+    for (int i = tid; i < d; i += blockDim.x) vec[i] = __bfloat162float(Kb[t * a.ks[2] + i]);
+    __syncthreads();
+    double acc = 0.0;
+    for (int i = part; i < d; i += parts) acc = fma(static_cast<double>(vec[i]), static_cast<double>(Psm[i * r + j]), acc);
+    red[part * r + j] = acc;
+    __syncthreads();
+    if (tid < r) {
+      double s = 0.0;
+      for (int q = 0; q < parts; ++q) s += red[q * r + tid];
+      Kpb[t * a.ps[2] + tid] = f64_to_bf16_rne(s);
+    }
+  }
+}
+
+cudaError_t launch_step_prologue(const PrologueArgs& a, cudaStream_t s) {
+  if (a.n_new > kMaxNewRowsInPrologue) return cudaErrorInvalidValue;
+  const size_t smem = static_cast<size_t>(a.d) * a.r * sizeof(float) + static_cast<size_t>(a.d + 1) * sizeof(float) +
+                      static_cast<size_t>(kPrologueThreads) * sizeof(double);
+  static int done[64] = {0};
+  cudaError_t e = set_smem_limit_once(step_prologue_kernel, smem, done);
+  if (e != cudaSuccess) return e;
+  step_prologue_kernel<<<a.B * a.Hkv, kPrologueThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -1,12 +1,12 @@
-// Subspace scoring: projected group query and the full-context score scan.
+// Subspace scoring: the full-context score scan.
 //
 // "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", Figure 1
 // and §3.1-§3.2: the group's query heads are projected with the same orthonormal
 // basis as the keys and score every cached position of the projected-key cache;
 // §E.1: this scan grows with batch size and dominates at large batch.
 //
-// qproj:  qs[b,h,:] = sum_g P_h^T q_{hG+g}   (fp32; the group sum is formed first)
-// score:  s[b,h,t]  = qs[b,h,:] . Kp[b,h,t,:] (fp32) for t in [0, T_b - W)
+// score:  s[b,h,t] = qs[b,h,:] . Kp[b,h,t,:] (fp32) for t in [0, T_b - W), with the
+//         projected group query qs formed by the step prologue (project.cu).
 //
 // The scan is HBM-bound (about r*2 bytes read and 4 bytes written per token).  A
 // persistent grid walks the flattened (row, token) space in 16 KB chunks; one
@@ -18,32 +18,6 @@
 #include "launch.h"
 
 namespace jssa {
-
-// ---------------------------------------------------------------- query projection
-__global__ void __launch_bounds__(256) qproj_kernel(QprojArgs a) {
-  extern __shared__ float qsum[];  // [d]
-  const int row = blockIdx.x;
-  const int b = row / a.Hkv, h = row % a.Hkv;
-  const int G = a.Hq / a.Hkv;
-  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.Q) + (static_cast<int64_t>(b) * a.Hq + h * G) * a.d;
-  for (int i = threadIdx.x; i < a.d; i += blockDim.x) {
-    float s = 0.f;
-    for (int g = 0; g < G; ++g) s += __bfloat162float(Q[static_cast<int64_t>(g) * a.d + i]);
-    qsum[i] = s;
-  }
-  __syncthreads();
-  const float* Ph = a.P + static_cast<int64_t>(h) * a.d * a.r;
-  for (int j = threadIdx.x; j < a.r; j += blockDim.x) {
-    float acc = 0.f;
-    for (int i = 0; i < a.d; ++i) acc = fmaf(__ldg(Ph + static_cast<int64_t>(i) * a.r + j), qsum[i], acc);
-    a.qs[static_cast<int64_t>(row) * a.r + j] = acc;
-  }
-}
-
-cudaError_t launch_qproj(const QprojArgs& a, cudaStream_t s) {
-  qproj_kernel<<<a.B * a.Hkv, 256, a.d * sizeof(float), s>>>(a);
-  return cudaGetLastError();
-}
 
 // ---------------------------------------------------------------- score scan
 constexpr int kScoreThreads = 256;
