@@ -35,7 +35,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode steps/s and µs/step at 128K (1×B200); % of HBM roofline; × vs own dense kernel"
 UNIT = "steps/s"
-KERNELS_PER_STEP = 5  # prologue (qs + newest key), score, topk, attention, merge
+KERNELS_PER_STEP = 4  # prologue (qs + newest key + resets), score (+ digit-1 histogram), topk, attention (+ merge)
 
 
 def parse():
@@ -206,29 +206,28 @@ def timed_graph(g, barrier):
 
 
 def stage_times(st, Q, reps=50):
-    """Per-stage device time (eager launches, CUDA events on the launching stream)."""
+    """Device time of the public entry points that make up the step, each replayed from a
+    CUDA graph of `reps` calls (CUDA events on the replay stream).  score = prologue +
+    score scan; topk = standalone selection (builds its own first-digit histogram);
+    attention = indexed attention with its fused merge."""
     jssa, w = st.jssa, st.w
-    scores = st.ws  # not used directly: the stage calls below use their own outputs
     sc = torch.empty(w.B, w.Hkv, st.T_cap, device="cuda")
+    calls = {
+        "score_us": lambda: jssa.score(st.L, Q, st.P, st.Kp, st.seq_lens, w.window, sc, st.ws),
+        "topk_us": lambda: jssa.topk(st.L, sc, st.seq_lens, w.k, w.window, st.idx, st.nsel, st.ws),
+        "attention_us": lambda: jssa.indexed_attn(st.L, Q, st.K, st.V, st.idx, w.k, st.nsel, st.seq_lens,
+                                                  w.window, w.sm_scale, st.O, None, st.ws),
+        "dense_us": lambda: st.dense(Q),
+    }
     out = {}
-
-    def t(fn):
-        for _ in range(3):
-            fn()
+    for name, fn in calls.items():
+        fn()
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(reps):
-            fn()
-        e1.record()
+        g = graph_of(lambda _q: fn(), [None] * reps)
+        g.replay()
         torch.cuda.synchronize()
-        return e0.elapsed_time(e1) * 1000.0 / reps
-
-    out["project_us"] = t(lambda: jssa.project_keys(st.L, st.K, st.P, st.Kp, 1, seq_lens=st.seq_lens))
-    out["score_us"] = t(lambda: jssa.score(st.L, Q, st.P, st.Kp, st.seq_lens, w.window, sc, st.ws))
-    out["topk_us"] = t(lambda: jssa.topk(st.L, sc, st.seq_lens, w.k, w.window, st.idx, st.nsel, st.ws))
-    out["attention_us"] = t(lambda: jssa.indexed_attn(st.L, Q, st.K, st.V, st.idx, w.k, st.nsel, st.seq_lens,
-                                                      w.window, w.sm_scale, st.O, None, st.ws))
+        out[name] = timed_graph(g, lambda: None) * 1000.0 / reps
+        del g
     return out
 
 
@@ -345,7 +344,7 @@ def main():
     stages = stage_times(st, Qs[0])
     hbm, peak_kind = peaks()
     score_bytes = bm["kp"] + bm["scores"]
-    score_s = stages["score_us"] * 1e-6
+    score_s = stages["score_us"] * 1e-6   # includes the (tiny) prologue launched with it
     shash = source_hash("score.cu", "common.cuh")
 
     # end to end through the public API with host buffers: per step, H2D of the query and of
@@ -399,7 +398,7 @@ def main():
             "byte_ratio": bm["dense"] / bm["step"],
             "dense_hbm_frac": bm["dense"] / (dense_ms * 1e-3) / 1e9 / hbm,
             "stage_us": stages,
-            "roofline": {"kernel": "score_kernel", "bound": "hbm", "achieved": achieved, "peak": hbm,
+            "roofline": {"kernel": "score_kernel (timed together with its step prologue)", "bound": "hbm", "achieved": achieved, "peak": hbm,
                          "unit": "GB/s", "frac": achieved / hbm, "peak_kind": peak_kind,
                          "traffic": traffic_for("score_kernel", w.name, shash),
                          "algorithmic_bytes_per_launch": score_bytes},

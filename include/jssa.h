@@ -148,7 +148,8 @@ JSSA_API jssa_status jssa_score(const jssa_layout* L, const void* Q, const float
  *   idx[b, h, :]  the k_eff = min(k, T_b - W) positions of largest score, ties to the
  *                 lower index, ascending; slots >= k_eff are -1      (device int32 [B, Hkv, k])
  *   n_sel[b, h]   k_eff                                               (device int32 [B, Hkv])
- * Scores must be finite.
+ * scores: device fp32 [B, Hkv, T_cap]; must be finite.  The workspace (required) holds
+ * the per-row first-digit histogram this call builds before selecting.
  */
 JSSA_API jssa_status jssa_topk(const jssa_layout* L, const float* scores, const int32_t* seq_lens,
                       int32_t k, int32_t window, int32_t* idx, int32_t* n_sel,

@@ -125,8 +125,10 @@ def test_topk_is_bit_exact(rows_T, k, seq, window, ties):
     sl = torch.tensor(seq, dtype=torch.int32, device="cuda")
     idx = torch.full((B, Hkv, k), -7, dtype=torch.int32, device="cuda")
     nsel = torch.full((B, Hkv), -7, dtype=torch.int32, device="cuda")
-    jssa.topk(L, scores, sl, k, window, idx, nsel)
+    ws = jssa.alloc_workspace(L, k, window)
+    jssa.topk(L, scores, sl, k, window, idx, nsel, ws)
     torch.cuda.synchronize()
+    _assert_status_clean(ws)
     s_host = scores.cpu().numpy().astype(np.float64)
     for b in range(B):
         n = seq[b] - min(window, seq[b])

@@ -65,9 +65,12 @@ jssa_status check_layout(const jssa_layout* L) {
 struct Workspace {
   int* status;
   float* qs;
-  float* scores;
+  uint32_t* hist;   // [rows, 4096] first radix digit of the selection
+  float* scores;    // [rows, sc_ld]
+  int64_t sc_ld;
   int32_t* idx;
   int32_t* n_sel;
+  int* counters;    // [rows] split arrival counters of the attention
   float* part_lse;
   float* part_o;
   int S_cap;
@@ -97,9 +100,12 @@ jssa_status carve(const jssa_layout* L, int64_t k, int64_t window, void* base, W
   };
   const size_t o_status = take(sizeof(int));
   const size_t o_qs = take(sizeof(float) * rows * L->r);
-  const size_t o_scores = take(sizeof(float) * static_cast<size_t>(rows) * L->T_cap);
+  const size_t o_hist = take(sizeof(uint32_t) * static_cast<size_t>(rows) * 4096);
+  const int64_t sc_ld = ceil_div(L->T_cap, 32) * 32;  // 128-byte aligned rows for bulk staging
+  const size_t o_scores = take(sizeof(float) * static_cast<size_t>(rows) * sc_ld);
   const size_t o_idx = take(sizeof(int32_t) * static_cast<size_t>(rows) * k);
   const size_t o_nsel = take(sizeof(int32_t) * rows);
+  const size_t o_cnt = take(sizeof(int) * rows);
   const size_t o_lse = take(sizeof(float) * static_cast<size_t>(L->B) * L->Hq * S_cap);
   const size_t o_po = take(sizeof(float) * static_cast<size_t>(L->B) * L->Hq * S_cap * L->d_v);
   w->bytes = off;
@@ -107,9 +113,12 @@ jssa_status carve(const jssa_layout* L, int64_t k, int64_t window, void* base, W
   char* p = static_cast<char*>(base);
   w->status = p ? reinterpret_cast<int*>(p + o_status) : nullptr;
   w->qs = p ? reinterpret_cast<float*>(p + o_qs) : nullptr;
+  w->hist = p ? reinterpret_cast<uint32_t*>(p + o_hist) : nullptr;
   w->scores = p ? reinterpret_cast<float*>(p + o_scores) : nullptr;
+  w->sc_ld = sc_ld;
   w->idx = p ? reinterpret_cast<int32_t*>(p + o_idx) : nullptr;
   w->n_sel = p ? reinterpret_cast<int32_t*>(p + o_nsel) : nullptr;
+  w->counters = p ? reinterpret_cast<int*>(p + o_cnt) : nullptr;
   w->part_lse = p ? reinterpret_cast<float*>(p + o_lse) : nullptr;
   w->part_o = p ? reinterpret_cast<float*>(p + o_po) : nullptr;
   return JSSA_OK;
@@ -160,6 +169,8 @@ jssa_status run_prologue(const jssa_layout* L, const void* Q, const float* P, co
   q.Kp = Kp;
   memcpy(q.ps, L->kp_stride, sizeof q.ps);
   q.seq_lens = seq_lens;
+  q.hist = w.hist;
+  q.counters = w.counters;
   q.n_new = n_new;
   q.B = L->B;
   q.Hq = L->Hq;
@@ -179,6 +190,7 @@ jssa_status run_score(const jssa_layout* L, const void* Kp, const int32_t* seq_l
   a.qs = w.qs;
   a.scores = scores;
   a.sc_ld = sc_ld;
+  a.hist = w.hist;
   a.seq_lens = seq_lens;
   a.B = L->B;
   a.Hkv = L->Hkv;
@@ -190,10 +202,11 @@ jssa_status run_score(const jssa_layout* L, const void* Kp, const int32_t* seq_l
 }
 
 jssa_status run_topk(const jssa_layout* L, const float* scores, int64_t sc_ld, const int32_t* seq_lens, int k,
-                     int window, int32_t* idx, int32_t* n_sel, int* status, cudaStream_t s) {
+                     int window, int32_t* idx, int32_t* n_sel, const Workspace& w, bool build_hist, cudaStream_t s) {
   TopkArgs a{};
   a.scores = scores;
   a.sc_ld = sc_ld;
+  a.hist = w.hist;
   a.seq_lens = seq_lens;
   a.B = L->B;
   a.Hkv = L->Hkv;
@@ -202,13 +215,23 @@ jssa_status run_topk(const jssa_layout* L, const float* scores, int64_t sc_ld, c
   a.window = window;
   a.idx = idx;
   a.n_sel = n_sel;
-  a.status = status;
+  a.status = w.status;
+  if (build_hist) {  // standalone selection: the first-digit histogram is not there yet
+    jssa_status st = cu(cudaMemsetAsync(w.hist, 0, sizeof(uint32_t) * 4096 * L->B * L->Hkv, s));
+    if (st != JSSA_OK) return st;
+    st = cu(launch_topk_histogram(a, num_sms_current(), s));
+    if (st != JSSA_OK) return st;
+  }
   return cu(launch_topk(a, s));
 }
 
 jssa_status run_attention(const jssa_layout* L, const void* Q, const void* K, const void* V, const int32_t* idx,
                           int idx_ld, const int32_t* n_sel, const int32_t* seq_lens, int window, float sm_scale,
-                          void* O, float* lse, const Workspace& w, cudaStream_t s) {
+                          void* O, float* lse, const Workspace& w, bool counters_zeroed, cudaStream_t s) {
+  if (!counters_zeroed) {
+    jssa_status st = cu(cudaMemsetAsync(w.counters, 0, sizeof(int) * L->B * L->Hkv, s));
+    if (st != JSSA_OK) return st;
+  }
   AttnArgs a{};
   a.Q = Q;
   a.K = K;
@@ -234,13 +257,17 @@ jssa_status run_attention(const jssa_layout* L, const void* Q, const void* K, co
   if (a.S > w.S_cap) return JSSA_ERR_WORKSPACE;
   a.part_o = w.part_o;
   a.part_lse = w.part_lse;
+  a.counters = w.counters;
   a.O = O;
   a.lse = lse;
   a.out_bf16 = (L->out_dtype == JSSA_OUT_BF16);
   a.status = w.status;
-  jssa_status st = cu(L->mode == JSSA_MODE_MLA ? launch_mla_attention(a, s) : launch_attention(a, s));
-  if (st != JSSA_OK) return st;
-  return cu(launch_merge(a, s));
+  if (L->mode == JSSA_MODE_MLA) {
+    jssa_status st = cu(launch_mla_attention(a, s));
+    if (st != JSSA_OK) return st;
+    return cu(launch_merge(a, s));
+  }
+  return cu(launch_attention(a, s));  // merges in its last CTA per row
 }
 
 }  // namespace
@@ -309,14 +336,10 @@ jssa_status jssa_topk(const jssa_layout* L, const float* scores, const int32_t* 
   if (st != JSSA_OK) return st;
   if (!scores || !seq_lens || !idx || !n_sel || k < 1 || k > kMaxK || window < 0) return JSSA_ERR_INVALID_ARG;
   if (!aligned(scores, 4) || !aligned(idx, 4) || !aligned(n_sel, 4)) return JSSA_ERR_INVALID_ARG;
-  int* status = nullptr;
-  if (workspace) {
-    Workspace w{};
-    st = get_ws(L, k, window, workspace, ws_bytes, &w);
-    if (st != JSSA_OK) return st;
-    status = w.status;
-  }
-  return run_topk(L, scores, L->T_cap, seq_lens, k, window, idx, n_sel, status, static_cast<cudaStream_t>(stream));
+  Workspace w{};
+  st = get_ws(L, k, window, workspace, ws_bytes, &w);
+  if (st != JSSA_OK) return st;
+  return run_topk(L, scores, L->T_cap, seq_lens, k, window, idx, n_sel, w, true, static_cast<cudaStream_t>(stream));
 }
 
 jssa_status jssa_indexed_attn(const jssa_layout* L, const void* Q, const void* K, const void* V, const int32_t* idx,
@@ -331,7 +354,7 @@ jssa_status jssa_indexed_attn(const jssa_layout* L, const void* Q, const void* K
   Workspace w{};
   st = get_ws(L, k, window, workspace, ws_bytes, &w);
   if (st != JSSA_OK) return st;
-  return run_attention(L, Q, K, V, idx, k, n_sel, seq_lens, window, sm_scale, O, lse, w,
+  return run_attention(L, Q, K, V, idx, k, n_sel, seq_lens, window, sm_scale, O, lse, w, false,
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -358,13 +381,13 @@ jssa_status jssa_decode_step(const jssa_layout* L, const void* Q, const void* K,
   }
   st = run_prologue(L, Q, P, K, Kp, seq_lens, n_new > kMaxPrologueRows ? 0 : n_new, w, s);
   if (st != JSSA_OK) return st;
-  st = run_score(L, Kp, seq_lens, window, w.scores, L->T_cap, w, s);
+  st = run_score(L, Kp, seq_lens, window, w.scores, w.sc_ld, w, s);
   if (st != JSSA_OK) return st;
   int32_t* idx = idx_out ? idx_out : w.idx;
   int32_t* nsel = n_sel_out ? n_sel_out : w.n_sel;
-  st = run_topk(L, w.scores, L->T_cap, seq_lens, k, window, idx, nsel, w.status, s);
+  st = run_topk(L, w.scores, w.sc_ld, seq_lens, k, window, idx, nsel, w, false, s);
   if (st != JSSA_OK) return st;
-  return run_attention(L, Q, K, V, idx, k, nsel, seq_lens, window, sm_scale, O, lse, w, s);
+  return run_attention(L, Q, K, V, idx, k, nsel, seq_lens, window, sm_scale, O, lse, w, true, s);
 }
 
 jssa_status jssa_dense_decode(const jssa_layout* L, const void* Q, const void* K, const void* V,
@@ -377,7 +400,7 @@ jssa_status jssa_dense_decode(const jssa_layout* L, const void* Q, const void* K
   Workspace w{};
   st = get_ws(L, 1, window, workspace, ws_bytes, &w);
   if (st != JSSA_OK) return st;
-  return run_attention(L, Q, K, V, nullptr, 0, nullptr, seq_lens, window, sm_scale, O, lse, w,
+  return run_attention(L, Q, K, V, nullptr, 0, nullptr, seq_lens, window, sm_scale, O, lse, w, false,
                        static_cast<cudaStream_t>(stream));
 }
 

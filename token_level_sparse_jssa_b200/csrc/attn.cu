@@ -18,7 +18,8 @@
 //   O^T[d x 8 heads]     += V_sub^T . P^T               (P split into bf16 hi + lo parts,
 //                                                        so the weights keep ~16 bits)
 // The 4 warps' states are merged in shared memory and the CTA writes one normalised
-// partial (o, lse) per query head; the merge kernel combines the splits.
+// partial (o, lse) per query head; the last CTA of each (sequence, KV head) row to
+// finish (a per-row arrival counter) combines the row's partials by log-sum-exp.
 #include <cmath>
 
 #include "common.cuh"
@@ -47,6 +48,53 @@ struct AttnCfg {
 template <int D, bool DENSE>
 static size_t attn_smem_bytes() {
   return AttnCfg<D>::MAIN_BYTES + (DENSE ? 0 : kMaxTokList * sizeof(int32_t));
+}
+
+// Combine the S split partials of query heads [hq0, hq0 + G) into O (and lse):
+// O = sum_s w_s o_s / sum_s w_s with w_s = exp(lse_s - max lse); lse = max + log(sum w).
+// Run by the last CTA of a row to finish, on partials every CTA made visible with a
+// device-scope fence before counting itself in.
+template <int D>
+__device__ __forceinline__ void merge_row(const AttnArgs& a, int64_t hq0, int G) {
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+    const int head = i / D, dim = i % D;
+    const float* lse_s = a.part_lse + (hq0 + head) * a.S;
+    const float* o_s = a.part_o + (hq0 + head) * a.S * D + dim;
+    float M = -INFINITY;
+    for (int s = 0; s < a.S; ++s) M = fmaxf(M, __ldcg(lse_s + s));
+    float o = 0.f, L = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll 4
+      for (int s = 0; s < a.S; ++s) {
+        const float w = expf(__ldcg(lse_s + s) - M);
+        L += w;
+        o += w * __ldcg(o_s + static_cast<int64_t>(s) * D);
+      }
+      o /= L;
+    }
+    const int64_t q = hq0 + head;
+    if (a.out_bf16) static_cast<__nv_bfloat16*>(a.O)[q * D + dim] = __float2bfloat16_rn(o);
+    else static_cast<float*>(a.O)[q * D + dim] = o;
+    if (a.lse && dim == 0) a.lse[q] = (M == -INFINITY) ? -INFINITY : M + logf(L);
+  }
+}
+
+// Count this CTA's finished partial in; the CTA that completes the row merges it and
+// re-arms the counter for the next call.
+template <int D>
+__device__ __forceinline__ void finish_split(const AttnArgs& a, int row, int64_t hq0, int G) {
+  __shared__ int is_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int prev = atomicAdd(a.counters + row, 1);
+    is_last = (prev == a.S - 1);
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  merge_row<D>(a, hq0, G);
+  if (threadIdx.x == 0) a.counters[row] = 0;
 }
 
 template <int D, int NTILE, bool DENSE>
@@ -94,6 +142,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
       a.part_o[((hq0 + head) * a.S + split) * D + dim] = 0.f;
       if (dim == 0) a.part_lse[(hq0 + head) * a.S + split] = -INFINITY;
     }
+    finish_split<D>(a, row, hq0, G);
     return;
   }
   if (!DENSE) {
@@ -316,6 +365,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
     a.part_o[((hq0 + head) * a.S + split) * D + dim] = o;
     if (dim == 0) a.part_lse[(hq0 + head) * a.S + split] = lse;
   }
+  finish_split<D>(a, row, hq0, G);
 }
 
 // ------------------------------------------------------------------ LSE merge

@@ -33,6 +33,8 @@ struct PrologueArgs {
   void* Kp;
   int64_t ps[3];
   const int32_t* seq_lens;
+  uint32_t* hist;   // nullable: [B*Hkv, 4096] zeroed here for the score scan
+  int* counters;    // nullable: [B*Hkv] attention arrival counters zeroed here
   int n_new;
   int B, Hq, Hkv, d, r;
   int64_t T_cap;
@@ -46,6 +48,7 @@ struct ScoreArgs {
   const float* qs;   // [B*Hkv, r]
   float* scores;     // [B*Hkv, sc_ld]
   int64_t sc_ld;
+  uint32_t* hist;    // nullable: [B*Hkv, 4096] histogram of key bits [31:20], pre-zeroed
   const int32_t* seq_lens;
   int B, Hkv, r;
   int64_t T_cap;
@@ -57,6 +60,7 @@ cudaError_t launch_score(const ScoreArgs& a, int num_sms, cudaStream_t s);
 struct TopkArgs {
   const float* scores;
   int64_t sc_ld;
+  uint32_t* hist;   // [B*Hkv, 4096] per-row histogram of key bits [31:20] (from the score scan)
   const int32_t* seq_lens;
   int B, Hkv;
   int64_t T_cap;
@@ -66,6 +70,8 @@ struct TopkArgs {
   int* status;
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
+// Standalone path: build the per-row first-digit histogram (hist must be zeroed).
+cudaError_t launch_topk_histogram(const TopkArgs& a, int num_sms, cudaStream_t s);
 
 struct AttnArgs {
   const void* Q;    // [B, Hq, dk]
@@ -84,6 +90,7 @@ struct AttnArgs {
   int64_t list_max;  // host upper bound on the attended list length
   float* part_o;     // [B, Hq, S, dv]
   float* part_lse;   // [B, Hq, S]
+  int* counters;     // [B*Hkv] per-row arrival counters, zero on entry, re-armed on exit
   int S, split_len;
   void* O;           // [B, Hq, dv]
   float* lse;        // nullable

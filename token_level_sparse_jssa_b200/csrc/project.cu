@@ -138,6 +138,11 @@ __global__ void __launch_bounds__(kPrologueThreads) step_prologue_kernel(Prologu
   const int G = a.Hq / a.Hkv;
   const int tid = threadIdx.x;
   stage_basis(Psm, a.P + static_cast<int64_t>(h) * d * r, d * r);
+  if (a.hist) {  // this row's first-digit histogram, filled by the score scan that follows
+    uint4* g = reinterpret_cast<uint4*>(a.hist + static_cast<int64_t>(row) * 4096);
+    for (int i = tid; i < 4096 / 4; i += blockDim.x) g[i] = make_uint4(0, 0, 0, 0);
+  }
+  if (a.counters && tid == 0) a.counters[row] = 0;
   const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.Q) + (static_cast<int64_t>(b) * a.Hq + h * G) * d;
   for (int i = tid; i < d; i += blockDim.x) {
     float s = 0.f;

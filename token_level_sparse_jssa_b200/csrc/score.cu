@@ -7,6 +7,11 @@
 //
 // score:  s[b,h,t] = qs[b,h,:] . Kp[b,h,t,:] (fp32) for t in [0, T_b - W), with the
 //         projected group query qs formed by the step prologue (project.cu).
+// The scan also builds, per (sequence, KV head) row, the histogram of the top 12 bits
+// of the order-preserving score keys (the first radix digit of the top-k selection):
+// a shared-memory histogram per CTA, flushed to the row's global histogram with one
+// atomic add per non-zero bin whenever the CTA moves to another row.  The ALU work is
+// hidden under the memory stream.
 //
 // The scan is HBM-bound (about r*2 bytes read and 4 bytes written per token).  A
 // persistent grid walks the flattened (row, token) space in 16 KB chunks; one
@@ -24,6 +29,7 @@ constexpr int kScoreThreads = 256;
 constexpr int kScoreStages = 4;
 constexpr int kChunkBytes = 16384;
 constexpr int kMaxBatch = 1024;
+constexpr int kHistBins = 4096;  // first radix digit of the selection: key bits [31:20]
 
 struct ChunkLoc {
   int row;
@@ -58,10 +64,12 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreArgs a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   unsigned char* ring = smem_raw;                                           // [stages][16 KB]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + kScoreStages * kChunkBytes);
-  int64_t* cum = reinterpret_cast<int64_t*>(bars + kScoreStages);           // [B + 1]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(bars + kScoreStages);        // [kHistBins]
+  int64_t* cum = reinterpret_cast<int64_t*>(hist + kHistBins);              // [B + 1]
   int64_t* nb = cum + (a.B + 1);                                            // [B]
 
   const int tid = threadIdx.x;
+  for (int i = tid; i < kHistBins; i += blockDim.x) hist[i] = 0;
   // candidate counts and chunk prefix per batch entry
   for (int b = tid; b < a.B; b += blockDim.x) {
     int64_t T = a.seq_lens[b];
@@ -109,21 +117,33 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreArgs a) {
   const int vec = tid % V;            // this thread's 8-wide slice of the token
   float q[8];
   int cur_row = -1;
+  // add this CTA's histogram of row `row` into the global one and clear it (block-uniform)
+  auto flush = [&](int row) {
+    if (a.hist) {
+      uint32_t* g = a.hist + static_cast<int64_t>(row) * kHistBins;
+      for (int i = tid; i < kHistBins; i += blockDim.x) {
+        const uint32_t v = hist[i];
+        if (v) { atomicAdd(g + i, v); hist[i] = 0; }
+      }
+    }
+    __syncthreads();
+  };
   int64_t it = 0;
   bool aborted = false;
   for (; it < n_mine; ++it) {
     const int s = static_cast<int>(it % kScoreStages);
     const uint32_t parity = static_cast<uint32_t>((it / kScoreStages) & 1);
+    const ChunkLoc L = locate_chunk<R>(c_begin + it, cum, nb, a.B, a.Hkv);
+    if (L.row != cur_row) {
+      if (cur_row >= 0) flush(cur_row);
+      cur_row = L.row;
+      const float4* qp = reinterpret_cast<const float4*>(a.qs + static_cast<int64_t>(cur_row) * R + vec * 8);
+      const float4 q0 = qp[0], q1 = qp[1];
+      q[0] = q0.x; q[1] = q0.y; q[2] = q0.z; q[3] = q0.w;
+      q[4] = q1.x; q[5] = q1.y; q[6] = q1.z; q[7] = q1.w;
+    }
     const bool ok = mbar_wait_bounded(&bars[s], parity, a.status);
     if (ok) {
-      const ChunkLoc L = locate_chunk<R>(c_begin + it, cum, nb, a.B, a.Hkv);
-      if (L.row != cur_row) {
-        cur_row = L.row;
-        const float4* qp = reinterpret_cast<const float4*>(a.qs + static_cast<int64_t>(cur_row) * R + vec * 8);
-        const float4 q0 = qp[0], q1 = qp[1];
-        q[0] = q0.x; q[1] = q0.y; q[2] = q0.z; q[3] = q0.w;
-        q[4] = q1.x; q[5] = q1.y; q[6] = q1.z; q[7] = q1.w;
-      }
       const unsigned char* buf = ring + s * kChunkBytes;
       float* out = a.scores + static_cast<int64_t>(L.row) * a.sc_ld + L.t0;
 #pragma unroll
@@ -142,29 +162,37 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreArgs a) {
         acc = fmaf(q[7], __uint_as_float(raw.w & 0xFFFF0000u), acc);
 #pragma unroll
         for (int off = V / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-        if (vec == 0 && tok < L.cnt) out[tok] = acc;
+        if (vec == 0 && tok < L.cnt) {
+          out[tok] = acc;
+          atomicAdd(&hist[float_to_ordered(acc) >> 20], 1u);
+        }
       }
     }
     // one barrier per chunk: everyone is done with stage s, and all agree on a timeout
     if (__syncthreads_or(!ok)) { aborted = true; break; }
     if (tid == 0 && it + kScoreStages < n_mine) issue(it + kScoreStages);
   }
-  if (aborted && tid == 0) {
-    // give every copy still in flight a bounded chance to land before the CTA exits
-    for (int64_t j = it; j < min64(it + kScoreStages, n_mine); ++j) {
-      const int s = static_cast<int>(j % kScoreStages);
-      mbar_wait_bounded(&bars[s], static_cast<uint32_t>((j / kScoreStages) & 1), a.status, 100000000ull);
+  if (aborted) {
+    if (tid == 0) {
+      // give every copy still in flight a bounded chance to land before the CTA exits
+      for (int64_t j = it; j < min64(it + kScoreStages, n_mine); ++j) {
+        const int s = static_cast<int>(j % kScoreStages);
+        mbar_wait_bounded(&bars[s], static_cast<uint32_t>((j / kScoreStages) & 1), a.status, 100000000ull);
+      }
     }
+    return;
   }
+  if (cur_row >= 0) flush(cur_row);
 }
 
 template <int R>
 static cudaError_t launch_score_r(const ScoreArgs& a, int num_sms, cudaStream_t s) {
-  const size_t smem = kScoreStages * kChunkBytes + kScoreStages * sizeof(uint64_t) + (2 * a.B + 1) * sizeof(int64_t);
+  const size_t smem = kScoreStages * kChunkBytes + kScoreStages * sizeof(uint64_t) + kHistBins * sizeof(uint32_t) +
+                      (2 * a.B + 1) * sizeof(int64_t);
   static int done[64] = {0};
   cudaError_t e = set_smem_limit_once(score_kernel<R>, smem, done);
   if (e != cudaSuccess) return e;
-  const int grid = num_sms * 3;
+  const int grid = num_sms * 2;
   score_kernel<R><<<grid, kScoreThreads, smem, s>>>(a);
   return cudaGetLastError();
 }

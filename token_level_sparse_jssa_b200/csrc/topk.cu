@@ -4,16 +4,26 @@
 // (top-B positions per KV head), §A.3 / §E.3 (independent selections per KV head
 // and sequence), §E.1 (top-B selection dominates the step at small batch).
 //
-// Exact radix select on order-preserving 32-bit keys, one thread-block cluster per
-// (sequence, KV head) row.  Each CTA of the cluster owns a contiguous slice of the
-// row, staged once from L2 into shared memory.  Three histogram passes (12, 12 and
-// 8 key bits) find the k-th largest key K*: each CTA histograms its slice, pushes
-// the non-zero bins into rank 0's shared memory (distributed shared memory atomics),
-// and rank 0 finds the digit and broadcasts it.  A last pass compacts, in index
-// order, every key > K* plus the lowest-indexed keys == K* up to the quota, using
-// warp ballots; per-CTA and per-warp counts give each output position, so the
-// selection comes out sorted ascending.  Cluster barriers are hardware barriers
-// over co-scheduled CTAs, so no wait here can hang.
+// Exact radix select on order-preserving 32-bit keys (larger score -> larger key,
+// -0 == +0), one thread-block cluster per (sequence, KV head) row; ties go to the
+// lower token index and the selection is written in ascending index order.
+//
+//   digit 1 (key bits 31..20): from the row's histogram, which the score scan builds
+//           as it streams the projected cache (or topk_hist_kernel for standalone
+//           calls); every CTA finds the digit itself.
+//   digits 2 and 3 (bits 19..10, 9..0): each CTA histograms the keys of its slice that
+//           match the prefix so far, adds the non-zero bins into rank 0's shared memory
+//           (distributed shared memory atomics), and after a cluster barrier every CTA
+//           reads the totals back and finds the digit.
+//   compaction: every key > K* plus, in index order, the first `need` keys == K*.  Each
+//           warp owns a contiguous piece of the slice; ballots give in-warp order, and
+//           per-warp / per-CTA counts exchanged across the cluster give each output
+//           position.
+//
+// Each CTA's slice of scores is staged once into shared memory with one bulk copy
+// (TMA engine).  Four cluster barriers in total; cluster barriers are hardware
+// barriers over co-scheduled CTAs, so no wait here can hang; the bulk-copy wait is
+// bounded in time.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -25,11 +35,14 @@ namespace jssa {
 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kBins = 4096;
+constexpr int kBins1 = 4096;   // digit 1: key bits [31:20]
+constexpr int kBins2 = 1024;   // digits 2 and 3: bits [19:10] and [9:0]
 constexpr int kMaxCluster = 8;
+constexpr int kSliceTarget = 16384;   // keys per CTA the cluster size aims for
+constexpr int kMaxStaged = 40960;     // keys per CTA that still fit in shared memory
 
-// Exclusive prefix sum over the block (every thread contributes v); returns the
-// sum of the values of lower-numbered threads and writes the block total.
+// Exclusive prefix sum over the block; returns the sum over lower-numbered threads and
+// writes the block total.
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_tmp, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t x = v;
@@ -51,10 +64,42 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
   }
   __syncthreads();
   const uint32_t warp_base = (warp > 0) ? warp_tmp[warp - 1] : 0;
-  const uint32_t res = warp_base + x - v;
-  if (total) *total = warp_tmp[kTopkWarps - 1];
+  *total = warp_tmp[kTopkWarps - 1];
   __syncthreads();
-  return res;
+  return warp_base + x - v;
+}
+
+// Given a histogram (any address space, generic pointer) and the number of keys still
+// to select, find the digit D whose suffix count (bins >= D) first reaches krem.  Writes
+// D and the count still to take inside bin D to *digit / *krem_out (shared memory).
+template <int NB>
+__device__ __forceinline__ void find_digit(const uint32_t* hist, uint32_t krem, uint32_t* scan_tmp,
+                                           uint32_t* digit, uint32_t* krem_out) {
+  constexpr int PER = (NB + kTopkThreads - 1) / kTopkThreads;
+  const int b0 = threadIdx.x * PER;
+  uint32_t c[PER];
+  uint32_t s = 0;
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    c[q] = (b0 + q < NB) ? hist[b0 + q] : 0u;
+    s += c[q];
+  }
+  uint32_t total;
+  const uint32_t below = block_exclusive_scan(s, scan_tmp, &total);
+  const uint32_t above = total - below - s;  // keys in the bins above this thread's group
+  if (b0 < NB && above < krem && above + s >= krem) {
+    uint32_t acc = above;
+#pragma unroll
+    for (int q = PER - 1; q >= 0; --q) {
+      if (acc + c[q] >= krem) {
+        *digit = static_cast<uint32_t>(b0 + q);
+        *krem_out = krem - acc;
+        break;
+      }
+      acc += c[q];
+    }
+  }
+  __syncthreads();
 }
 
 template <bool STAGED>
@@ -62,11 +107,13 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   cg::cluster_group cluster = cg::this_cluster();
   const int C = static_cast<int>(cluster.num_blocks());
   const int crank = static_cast<int>(cluster.block_rank());
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);  // [kBins] this CTA's histogram
-  uint32_t* tot = hist + kBins;                             // [kBins] cluster total (rank 0)
-  uint32_t* keys = tot + kBins;                             // [per_cap] staged keys
-  __shared__ uint32_t bc_digit, bc_krem;                    // written by rank 0
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  float* fs = reinterpret_cast<float*>(smem_raw);                      // [per_cap] staged scores
+  uint32_t* hloc = reinterpret_cast<uint32_t*>(fs + per_cap);          // [kBins2] this CTA's histogram
+  uint32_t* totA = hloc + kBins2;                                       // [kBins2] digit-2 totals (rank 0)
+  uint32_t* totB = totA + kBins2;                                       // [kBins2] digit-3 totals (rank 0)
+  __shared__ uint64_t bar;
+  __shared__ uint32_t dig, krem_s;
   __shared__ uint32_t cta_gt[kMaxCluster], cta_eq[kMaxCluster];
   __shared__ uint32_t warp_gt[kTopkWarps], warp_eq[kTopkWarps];
   __shared__ uint32_t scan_tmp[32];
@@ -92,72 +139,68 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   }
 
   // this CTA's slice [lo, lo + len)
-  const int64_t per = ceil_div(n, C);
+  const int64_t per = ceil_div(ceil_div(n, C), 4) * 4;
   const int64_t lo = crank * per;
   const int len = static_cast<int>(max64(0, min64(n, lo + per) - lo));
   const float* srow = a.scores + static_cast<int64_t>(row) * a.sc_ld + lo;
+  bool staged_ok = true;
   if (STAGED) {
-    for (int i = tid; i < len; i += kTopkThreads) keys[i] = float_to_ordered(__ldg(srow + i));
-  }
-  auto key_at = [&](int i) -> uint32_t { return STAGED ? keys[i] : float_to_ordered(__ldg(srow + i)); };
-
-  uint32_t prefix = 0, mask = 0, krem = static_cast<uint32_t>(k_eff);
-  for (int i = tid; i < kBins; i += kTopkThreads) tot[i] = 0;
-  uint32_t* tot0 = cluster.map_shared_rank(tot, 0);
-#pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = (pass == 0) ? 20 : (pass == 1) ? 8 : 0;
-    const int nb = (pass == 2) ? 256 : kBins;
-    for (int i = tid; i < nb; i += kTopkThreads) hist[i] = 0;
-    if (pass == 0) cluster.sync();  // every CTA runs and rank 0's totals are zero
-    else __syncthreads();
-    for (int i = tid; i < len; i += kTopkThreads) {
-      const uint32_t key = key_at(i);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+    const bool bulk = (reinterpret_cast<uintptr_t>(srow) & 15u) == 0;
+    const int nbulk = bulk ? (len & ~3) : 0;
+    if (tid == 0) {
+      mbar_init(&bar, 1);
+      fence_mbarrier_init();
     }
     __syncthreads();
-    for (int i = tid; i < nb; i += kTopkThreads) {
-      const uint32_t v = hist[i];
+    if (tid == 0 && nbulk > 0) {
+      mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nbulk) * 4u);
+      bulk_g2s(fs, srow, static_cast<uint32_t>(nbulk) * 4u, &bar, l2_policy_evict_first());
+    }
+    for (int i = nbulk + tid; i < len; i += kTopkThreads) fs[i] = __ldg(srow + i);
+    if (nbulk > 0) staged_ok = mbar_wait_bounded(&bar, 0, a.status);
+  }
+  auto key_at = [&](int i) -> uint32_t { return float_to_ordered(STAGED ? fs[i] : __ldg(srow + i)); };
+
+  if (crank == 0)
+    for (int i = tid; i < kBins2; i += kTopkThreads) { totA[i] = 0; totB[i] = 0; }
+  // digit 1 from the global histogram (every CTA computes the same digit)
+  find_digit<kBins1>(a.hist + static_cast<int64_t>(row) * kBins1, static_cast<uint32_t>(k_eff), scan_tmp, &dig,
+                     &krem_s);
+  uint32_t prefix = dig << 20, mask = 0xFFF00000u, krem = krem_s;
+  const bool aborted = __syncthreads_or(!staged_ok);
+  cluster.sync();  // rank 0's totals are zero and every CTA of the cluster is running
+
+  uint32_t* totA0 = cluster.map_shared_rank(totA, 0);
+  uint32_t* totB0 = cluster.map_shared_rank(totB, 0);
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const int shift = (pass == 0) ? 10 : 0;
+    uint32_t* tot0 = (pass == 0) ? totA0 : totB0;
+    for (int i = tid; i < kBins2; i += kTopkThreads) hloc[i] = 0;
+    __syncthreads();
+    if (!aborted) {
+      for (int i = tid; i < len; i += kTopkThreads) {
+        const uint32_t key = key_at(i);
+        if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kBins2 - 1)], 1u);
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < kBins2; i += kTopkThreads) {
+      const uint32_t v = hloc[i];
       if (v) atomicAdd(&tot0[i], v);
     }
     cluster.sync();
-    if (crank == 0) {
-      // digit D: the largest bin whose suffix count (bins >= D) reaches krem
-      const int per_t = (nb + kTopkThreads - 1) / kTopkThreads;
-      const int b0 = tid * per_t, b1 = min(nb, b0 + per_t);
-      uint32_t s = 0;
-      for (int i = b0; i < b1; ++i) s += tot[i];
-      // count in the bins above this thread's range: total - inclusive prefix
-      uint32_t total;
-      const uint32_t below = block_exclusive_scan(s, scan_tmp, &total);
-      const uint32_t above = total - below - s;
-      if (b0 < b1 && above < krem && above + s >= krem) {
-        uint32_t acc = above;
-        for (int i = b1 - 1; i >= b0; --i) {
-          if (acc + tot[i] >= krem) {
-            for (int c = 0; c < C; ++c) {
-              *cluster.map_shared_rank(&bc_digit, c) = static_cast<uint32_t>(i);
-              *cluster.map_shared_rank(&bc_krem, c) = krem - acc;
-            }
-            break;
-          }
-          acc += tot[i];
-        }
-      }
-      __syncthreads();
-      for (int i = tid; i < nb; i += kTopkThreads) tot[i] = 0;
-    }
-    cluster.sync();
-    prefix |= bc_digit << shift;
-    mask |= static_cast<uint32_t>(nb - 1) << shift;
-    krem = bc_krem;
+    find_digit<kBins2>(tot0, krem, scan_tmp, &dig, &krem_s);
+    prefix |= dig << shift;
+    mask |= static_cast<uint32_t>(kBins2 - 1) << shift;
+    krem = krem_s;
   }
   const uint32_t kstar = prefix;  // the k-th largest key
   const uint32_t need = krem;     // keys equal to kstar to take, lowest index first
 
   // ---- ordered compaction: warp w owns [w*wc, min(len, (w+1)*wc))
   const int wc = static_cast<int>(ceil_div(ceil_div(len, kTopkWarps), 32) * 32);
-  const int w_lo = warp * wc, w_hi = min(len, w_lo + wc);
+  const int w_lo = warp * wc, w_hi = aborted ? w_lo : min(len, w_lo + wc);
   uint32_t ngt = 0, neq = 0;
   for (int base = w_lo; base < w_hi; base += 32) {
     const int i = base + lane;
@@ -174,7 +217,10 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     *cluster.map_shared_rank(&cta_eq[crank], tid) = e;
   }
   cluster.sync();  // last access to another CTA's shared memory
-  // output base of this CTA and its quota of equal keys
+  if (aborted) {  // the staging copy never completed (flagged): report an empty selection
+    for (int64_t j = crank * kTopkThreads + tid; j < k_eff; j += static_cast<int64_t>(C) * kTopkThreads) out[j] = -1;
+    return;
+  }
   uint32_t base_out = 0, eq_before = 0;
   for (int c = 0; c < crank; ++c) {
     const uint32_t q = (need > eq_before) ? min(cta_eq[c], need - eq_before) : 0u;
@@ -182,7 +228,6 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     eq_before += cta_eq[c];
   }
   const uint32_t quota = (need > eq_before) ? min(cta_eq[crank], need - eq_before) : 0u;
-  // this warp's base and its first equal-key rank inside the CTA
   uint32_t pos = base_out, eq_rank = 0;
   for (int w = 0; w < warp; ++w) {
     const uint32_t q = (quota > eq_rank) ? min(warp_eq[w], quota - eq_rank) : 0u;
@@ -208,14 +253,43 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   }
 }
 
+// Standalone path: histogram of key bits [31:20] per row, 8192 scores per CTA.
+constexpr int kHistChunk = 8192;
+__global__ void __launch_bounds__(256) topk_hist_kernel(TopkArgs a) {
+  __shared__ uint32_t h[kBins1];
+  const int row = blockIdx.y;
+  const int b = row / a.Hkv;
+  int64_t T = a.seq_lens[b];
+  T = T < 0 ? 0 : (T > a.T_cap ? a.T_cap : T);
+  const int64_t n = T - min64(max64(a.window, 0), T);
+  const int64_t lo = static_cast<int64_t>(blockIdx.x) * kHistChunk;
+  if (lo >= n) return;
+  const int64_t hi = min64(n, lo + kHistChunk);
+  for (int i = threadIdx.x; i < kBins1; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  const float* srow = a.scores + static_cast<int64_t>(row) * a.sc_ld;
+  for (int64_t t = lo + threadIdx.x; t < hi; t += blockDim.x)
+    atomicAdd(&h[float_to_ordered(__ldg(srow + t)) >> 20], 1u);
+  __syncthreads();
+  uint32_t* g = a.hist + static_cast<int64_t>(row) * kBins1;
+  for (int i = threadIdx.x; i < kBins1; i += blockDim.x)
+    if (h[i]) atomicAdd(g + i, h[i]);
+}
+
+cudaError_t launch_topk_histogram(const TopkArgs& a, int, cudaStream_t s) {
+  dim3 grid(static_cast<unsigned>(ceil_div(a.T_cap, kHistChunk)), a.B * a.Hkv);
+  topk_hist_kernel<<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   const int64_t n_max = a.T_cap;
   int C = 1;
-  while (C < kMaxCluster && ceil_div(n_max, C) > 16384) C *= 2;
-  const int64_t per = ceil_div(n_max, C);
-  const bool staged = per <= 40960;
+  while (C < kMaxCluster && ceil_div(n_max, C) > kSliceTarget) C *= 2;
+  const int64_t per = ceil_div(ceil_div(n_max, C), 4) * 4;
+  const bool staged = per <= kMaxStaged;
   const int per_cap = staged ? static_cast<int>(per) : 0;
-  const size_t smem = 2 * kBins * sizeof(uint32_t) + static_cast<size_t>(per_cap) * sizeof(uint32_t);
+  const size_t smem = static_cast<size_t>(per_cap) * sizeof(float) + 3 * kBins2 * sizeof(uint32_t);
   void (*kern)(TopkArgs, int) = staged ? topk_kernel<true> : topk_kernel<false>;
   static int done_staged[64] = {0}, done_plain[64] = {0};
   cudaError_t e = set_smem_limit_once(kern, smem, staged ? done_staged : done_plain);
