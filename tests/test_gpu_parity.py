@@ -107,7 +107,9 @@ def test_score_within_fp32_error_bound(name, kw, seq, window):
     ((4, 131072), 2048, None, 0, 200),                    # 8-CTA clusters
     ((2, 65536), 1024, [65536, 40000], 1024, 100),        # window shrinks the candidates
     ((2, 4096), 4096, [4096, 100], 0, 10),                # k >= n: select everything
-    ((1, 400000), 777, [400000], 0, 100),                 # slice larger than shared memory
+    ((1, 400000), 777, [400000], 0, 100),                 # 16-CTA cluster, large staged slices
+    ((1, 600000), 3000, [599999], 0, 100),                # slice larger than shared memory
+    ((2, 50000), 1000, [50000, 49000], 0, 30000),         # many exact ties
     ((2, 5000), 1, [5000, 1], 0, 2),
 ])
 def test_topk_is_bit_exact(rows_T, k, seq, window, ties):
@@ -133,6 +135,40 @@ def test_topk_is_bit_exact(rows_T, k, seq, window, ties):
     for b in range(B):
         n = seq[b] - min(window, seq[b])
         ref, k_eff = oracle.topk(s_host[b, :n], k)
+        assert int(nsel[b, 0]) == k_eff
+        np.testing.assert_array_equal(idx[b, 0].cpu().numpy(), ref)
+
+
+def _topk_layout(B, T):
+    L = jssa.Layout()
+    L.mode, L.B, L.Hq, L.Hkv, L.d_k, L.d_v, L.r, L.out_dtype, L.T_cap = 0, B, 4, 1, 128, 128, 16, 0, T
+    for i, v in enumerate((T * 128, T * 128, 128)):
+        L.k_stride[i] = v
+        L.v_stride[i] = v
+    for i, v in enumerate((T * 16, T * 16, 16)):
+        L.kp_stride[i] = v
+    return L
+
+
+@pytest.mark.parametrize("T,k,levels", [(131072, 2048, 1), (131072, 5000, 3), (70000, 300, 2)])
+def test_topk_with_few_distinct_values(T, k, levels):
+    # every key of a slice falls in one digit-1 bin: the candidate list overflows and the
+    # CTAs scan their whole slices instead; ties resolve to the lowest indices
+    B = 2
+    g = torch.Generator().manual_seed(T + k)
+    vals = torch.tensor([1.5, -0.25, 7.0][:levels])
+    scores = vals[torch.randint(0, levels, (B, T), generator=g)].float().cuda()
+    L = _topk_layout(B, T)
+    sl = torch.tensor([T, T - 17], dtype=torch.int32, device="cuda")
+    idx = torch.empty((B, 1, k), dtype=torch.int32, device="cuda")
+    nsel = torch.empty((B, 1), dtype=torch.int32, device="cuda")
+    ws = jssa.alloc_workspace(L, k, 0)
+    jssa.topk(L, scores, sl, k, 0, idx, nsel, ws)
+    torch.cuda.synchronize()
+    _assert_status_clean(ws)
+    s_host = scores.cpu().numpy().astype(np.float64)
+    for b in range(B):
+        ref, k_eff = oracle.topk(s_host[b, :int(sl[b])], k)
         assert int(nsel[b, 0]) == k_eff
         np.testing.assert_array_equal(idx[b, 0].cpu().numpy(), ref)
 

@@ -10,85 +10,93 @@
 // The scan also builds, per (sequence, KV head) row, the histogram of the top 12 bits
 // of the order-preserving score keys (the first radix digit of the top-k selection):
 // a shared-memory histogram per CTA, flushed to the row's global histogram with one
-// atomic add per non-zero bin whenever the CTA moves to another row.  The ALU work is
-// hidden under the memory stream.
+// atomic add per non-zero bin whenever the CTA moves to another row.
 //
-// The scan is HBM-bound (about r*2 bytes read and 4 bytes written per token).  A
-// persistent grid walks the flattened (row, token) space in 16 KB chunks; one
-// thread per CTA streams chunks into a 4-stage shared-memory ring with 1-D bulk
-// copies (TMA engine, L2 evict-first), completion tracked by mbarriers.  Each chunk
-// is consumed with 16-byte shared loads: r/8 consecutive threads share a token,
-// each holding a fixed 8-wide slice of qs in registers, and reduce by shuffles.
+// The scan is HBM-bound (r*2 bytes read and 4 bytes written per token).  A persistent
+// grid walks the flattened (row, token) space in 16 KB chunks, each CTA a contiguous
+// range of chunks.  One producer warp streams chunks into a shared-memory ring with
+// 1-D bulk copies (TMA engine, L2 evict-first) and full/empty mbarrier pairs; eight
+// consumer warps score them without any block-wide barrier.  A consumer thread owns
+// whole tokens (two threads per token for r = 64): it reads a token's 16-byte
+// vectors in a per-thread rotated order, so that every 8-thread phase of a 16-byte
+// shared load touches 8 different bank groups, and holds the matching rotated slice
+// of qs in registers.  Chunk bookkeeping advances incrementally (no divisions).
 #include "common.cuh"
 #include "launch.h"
 
 namespace jssa {
 
-// ---------------------------------------------------------------- score scan
-constexpr int kScoreThreads = 256;
-constexpr int kScoreStages = 4;
+constexpr int kScoreConsumers = 256;                 // 8 consumer warps
+constexpr int kScoreThreads = kScoreConsumers + 32;  // + 1 producer warp
+constexpr int kScoreStages = 3;
 constexpr int kChunkBytes = 16384;
 constexpr int kMaxBatch = 1024;
 constexpr int kHistBins = 4096;  // first radix digit of the selection: key bits [31:20]
 
-struct ChunkLoc {
-  int row;
-  int64_t t0;
-  int cnt;
+// Position in the flattened chunk space: sequence b, KV head h, chunk ci of the row.
+struct ChunkIter {
+  int b, h;
+  int64_t ci;
 };
 
-template <int R>
-__device__ __forceinline__ ChunkLoc locate_chunk(int64_t c, const int64_t* cum, const int64_t* nb, int B, int Hkv) {
-  constexpr int CH = kChunkBytes / (R * 2);
-  int lo = 0, hi = B - 1;  // last b with cum[b] <= c
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (cum[mid] <= c) lo = mid; else hi = mid - 1;
-  }
-  const int b = lo;
-  const int64_t per_head = ceil_div(nb[b], CH);
-  const int64_t local = c - cum[b];
-  const int h = static_cast<int>(local / per_head);
-  const int64_t ci = local % per_head;
-  ChunkLoc L;
-  L.row = b * Hkv + h;
-  L.t0 = ci * CH;
-  L.cnt = static_cast<int>(min64(CH, nb[b] - L.t0));
-  return L;
+__device__ __forceinline__ void chunk_advance(ChunkIter& c, const int64_t* per_head, int B, int Hkv) {
+  if (++c.ci < per_head[c.b]) return;
+  c.ci = 0;
+  if (++c.h < Hkv) return;
+  c.h = 0;
+  do { ++c.b; } while (c.b < B && per_head[c.b] == 0);
+}
+
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kScoreConsumers) : "memory"); }
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 template <int R>
 __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreArgs a) {
-  constexpr int CH = kChunkBytes / (R * 2);  // tokens per chunk
-  constexpr int V = R / 8;                    // 16-byte vectors per token = threads per token
+  constexpr int CH = kChunkBytes / (R * 2);           // tokens per chunk
+  constexpr int V = R / 8;                            // 16-byte vectors per token
+  constexpr int TPT = (R >= 64) ? 2 : 1;              // threads per token
+  constexpr int VPT = V / TPT;                        // vectors per thread (<= 4)
+  constexpr int TOK_PER_PASS = kScoreConsumers / TPT;
+  constexpr int PASSES = CH / TOK_PER_PASS;
+  static_assert(PASSES >= 1 && CH % TOK_PER_PASS == 0, "chunk / thread mapping");
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  unsigned char* ring = smem_raw;                                           // [stages][16 KB]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + kScoreStages * kChunkBytes);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(bars + kScoreStages);        // [kHistBins]
-  int64_t* cum = reinterpret_cast<int64_t*>(hist + kHistBins);              // [B + 1]
-  int64_t* nb = cum + (a.B + 1);                                            // [B]
+  unsigned char* ring = smem_raw;                                                   // [stages][16 KB]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + kScoreStages * kChunkBytes);
+  uint64_t* empty = full + kScoreStages;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(empty + kScoreStages);               // [kHistBins]
+  int64_t* cum = reinterpret_cast<int64_t*>(hist + kHistBins);                      // [B + 1] chunk prefix
+  int64_t* per_head = cum + (a.B + 1);                                              // [B] chunks per row
+  int64_t* nb = per_head + a.B;                                                     // [B] candidates
+  __shared__ int aborted;
 
   const int tid = threadIdx.x;
+  const bool producer = tid >= kScoreConsumers;
   for (int i = tid; i < kHistBins; i += blockDim.x) hist[i] = 0;
-  // candidate counts and chunk prefix per batch entry
   for (int b = tid; b < a.B; b += blockDim.x) {
     int64_t T = a.seq_lens[b];
     if (T < 0 || T > a.T_cap) {
       if (blockIdx.x == 0) flag_error(a.status, DEVFLAG_BAD_SEQ_LEN);
       T = T < 0 ? 0 : a.T_cap;
     }
-    const int64_t W = min64(max(a.window, 0), T);
-    nb[b] = T - W;
+    nb[b] = T - min64(max64(a.window, 0), T);
+    per_head[b] = ceil_div(nb[b], CH);
   }
   __syncthreads();
   if (tid == 0) {
+    aborted = 0;
     int64_t c = 0;
     for (int b = 0; b < a.B; ++b) {
       cum[b] = c;
-      c += static_cast<int64_t>(a.Hkv) * ceil_div(nb[b], CH);
+      c += static_cast<int64_t>(a.Hkv) * per_head[b];
     }
     cum[a.B] = c;
-    for (int s = 0; s < kScoreStages; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s < kScoreStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kScoreConsumers / 32);
+    }
     fence_mbarrier_init();
   }
   __syncthreads();
@@ -98,101 +106,138 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreArgs a) {
   const int64_t n_mine = c_end - c_begin;
   if (n_mine <= 0) return;
 
-  const __nv_bfloat16* Kp = static_cast<const __nv_bfloat16*>(a.Kp);
-  uint64_t policy = 0;
-  auto issue = [&](int64_t it) {
-    const ChunkLoc L = locate_chunk<R>(c_begin + it, cum, nb, a.B, a.Hkv);
-    const int b = L.row / a.Hkv, h = L.row % a.Hkv;
-    const __nv_bfloat16* src = Kp + b * a.ps[0] + h * a.ps[1] + L.t0 * a.ps[2];
-    const uint32_t bytes = static_cast<uint32_t>(L.cnt) * R * 2;
-    const int s = static_cast<int>(it % kScoreStages);
-    mbar_arrive_expect_tx(&bars[s], bytes);
-    bulk_g2s(ring + s * kChunkBytes, src, bytes, &bars[s], policy);
-  };
-  if (tid == 0) {
-    policy = l2_policy_evict_first();
-    for (int64_t it = 0; it < min64(kScoreStages, n_mine); ++it) issue(it);
+  // iterator at c_begin (the only divisions of the kernel)
+  ChunkIter it0;
+  {
+    int b = 0;
+    while (b + 1 < a.B && cum[b + 1] <= c_begin) ++b;
+    const int64_t local = c_begin - cum[b];
+    it0.b = b;
+    it0.h = static_cast<int>(local / per_head[b]);
+    it0.ci = local % per_head[b];
   }
 
-  const int vec = tid % V;            // this thread's 8-wide slice of the token
-  float q[8];
-  int cur_row = -1;
-  // add this CTA's histogram of row `row` into the global one and clear it (block-uniform)
-  auto flush = [&](int row) {
-    if (a.hist) {
-      uint32_t* g = a.hist + static_cast<int64_t>(row) * kHistBins;
-      for (int i = tid; i < kHistBins; i += blockDim.x) {
-        const uint32_t v = hist[i];
-        if (v) { atomicAdd(g + i, v); hist[i] = 0; }
+  if (producer) {
+    if ((tid & 31) == 0) {
+      const uint64_t policy = l2_policy_evict_first();
+      const __nv_bfloat16* Kp = static_cast<const __nv_bfloat16*>(a.Kp);
+      ChunkIter c = it0;
+      for (int64_t it = 0; it < n_mine; ++it) {
+        const int s = static_cast<int>(it % kScoreStages);
+        if (it >= kScoreStages &&
+            !mbar_wait_bounded(&empty[s], static_cast<uint32_t>((it / kScoreStages - 1) & 1), a.status)) {
+          atomicExch(&aborted, 1);
+          break;
+        }
+        const int64_t t0 = c.ci * CH;
+        const uint32_t cnt = static_cast<uint32_t>(min64(CH, nb[c.b] - t0));
+        const __nv_bfloat16* src = Kp + c.b * a.ps[0] + c.h * a.ps[1] + t0 * a.ps[2];
+        mbar_arrive_expect_tx(&full[s], cnt * R * 2);
+        bulk_g2s(ring + s * kChunkBytes, src, cnt * R * 2, &full[s], policy);
+        chunk_advance(c, per_head, a.B, a.Hkv);
       }
     }
-    __syncthreads();
-  };
-  int64_t it = 0;
-  bool aborted = false;
-  for (; it < n_mine; ++it) {
-    const int s = static_cast<int>(it % kScoreStages);
-    const uint32_t parity = static_cast<uint32_t>((it / kScoreStages) & 1);
-    const ChunkLoc L = locate_chunk<R>(c_begin + it, cum, nb, a.B, a.Hkv);
-    if (L.row != cur_row) {
-      if (cur_row >= 0) flush(cur_row);
-      cur_row = L.row;
-      const float4* qp = reinterpret_cast<const float4*>(a.qs + static_cast<int64_t>(cur_row) * R + vec * 8);
-      const float4 q0 = qp[0], q1 = qp[1];
-      q[0] = q0.x; q[1] = q0.y; q[2] = q0.z; q[3] = q0.w;
-      q[4] = q1.x; q[5] = q1.y; q[6] = q1.z; q[7] = q1.w;
-    }
-    const bool ok = mbar_wait_bounded(&bars[s], parity, a.status);
-    if (ok) {
-      const unsigned char* buf = ring + s * kChunkBytes;
-      float* out = a.scores + static_cast<int64_t>(L.row) * a.sc_ld + L.t0;
+  } else {
+    // this thread's token within a pass, its slice of the token and its rotation
+    const int sub = (TPT == 2) ? (tid & 1) : 0;
+    const int tok_in_pass = tid / TPT;
+    const int rot = (V == 1) ? 0 : (TPT == 2 ? ((tid >> 1) & 3) : ((tid >> (V == 2 ? 2 : 1)) & (V - 1)));
+    float q[VPT][8];
+    ChunkIter c = it0;
+    int cur_row = -1;
+    bool dead = false;  // a wait gave up: keep the loop's barrier structure, skip the work
+    for (int64_t it = 0; it < n_mine; ++it) {
+      const int s = static_cast<int>(it % kScoreStages);
+      const int row = c.b * a.Hkv + c.h;
+      if (row != cur_row) {
+        if (cur_row >= 0) {  // flush the finished row's histogram (all consumers)
+          consumers_sync();
+          if (a.hist) {
+            uint32_t* g = a.hist + static_cast<int64_t>(cur_row) * kHistBins;
+            for (int i = tid; i < kHistBins; i += kScoreConsumers) {
+              const uint32_t v = hist[i];
+              if (v) { atomicAdd(g + i, v); hist[i] = 0; }
+            }
+          }
+          consumers_sync();
+        }
+        cur_row = row;
 #pragma unroll
-      for (int m = 0; m < (CH * V) / kScoreThreads; ++m) {
-        const int slot = tid + m * kScoreThreads;
-        const int tok = slot / V;
-        const uint4 raw = *reinterpret_cast<const uint4*>(buf + static_cast<size_t>(slot) * 16);
-        float acc = 0.f;
-        acc = fmaf(q[0], __uint_as_float(raw.x << 16), acc);
-        acc = fmaf(q[1], __uint_as_float(raw.x & 0xFFFF0000u), acc);
-        acc = fmaf(q[2], __uint_as_float(raw.y << 16), acc);
-        acc = fmaf(q[3], __uint_as_float(raw.y & 0xFFFF0000u), acc);
-        acc = fmaf(q[4], __uint_as_float(raw.z << 16), acc);
-        acc = fmaf(q[5], __uint_as_float(raw.z & 0xFFFF0000u), acc);
-        acc = fmaf(q[6], __uint_as_float(raw.w << 16), acc);
-        acc = fmaf(q[7], __uint_as_float(raw.w & 0xFFFF0000u), acc);
-#pragma unroll
-        for (int off = V / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-        if (vec == 0 && tok < L.cnt) {
-          out[tok] = acc;
-          atomicAdd(&hist[float_to_ordered(acc) >> 20], 1u);
+        for (int j = 0; j < VPT; ++j) {
+          const float4* qp = reinterpret_cast<const float4*>(a.qs + static_cast<int64_t>(row) * R +
+                                                             (sub * VPT + (j + rot) % VPT) * 8);
+          const float4 q0 = qp[0], q1 = qp[1];
+          q[j][0] = q0.x; q[j][1] = q0.y; q[j][2] = q0.z; q[j][3] = q0.w;
+          q[j][4] = q1.x; q[j][5] = q1.y; q[j][6] = q1.z; q[j][7] = q1.w;
         }
       }
+      if (!dead && !mbar_wait_bounded(&full[s], static_cast<uint32_t>((it / kScoreStages) & 1), a.status)) {
+        dead = true;
+        atomicExch(&aborted, 1);
+      }
+      if (!dead) {
+        const int64_t t0 = c.ci * CH;
+        const int cnt = static_cast<int>(min64(CH, nb[c.b] - t0));
+        const unsigned char* buf = ring + s * kChunkBytes;
+        float* out = a.scores + static_cast<int64_t>(row) * a.sc_ld + t0;
+#pragma unroll
+        for (int p = 0; p < PASSES; ++p) {
+          const int tok = p * TOK_PER_PASS + tok_in_pass;
+          const unsigned char* trow = buf + tok * (R * 2);
+          float acc[VPT];
+#pragma unroll
+          for (int j = 0; j < VPT; ++j) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(trow + (sub * VPT + (j + rot) % VPT) * 16);
+            float x = q[j][0] * __uint_as_float(raw.x << 16);
+            x = fmaf(q[j][1], __uint_as_float(raw.x & 0xFFFF0000u), x);
+            x = fmaf(q[j][2], __uint_as_float(raw.y << 16), x);
+            x = fmaf(q[j][3], __uint_as_float(raw.y & 0xFFFF0000u), x);
+            x = fmaf(q[j][4], __uint_as_float(raw.z << 16), x);
+            x = fmaf(q[j][5], __uint_as_float(raw.z & 0xFFFF0000u), x);
+            x = fmaf(q[j][6], __uint_as_float(raw.w << 16), x);
+            x = fmaf(q[j][7], __uint_as_float(raw.w & 0xFFFF0000u), x);
+            acc[j] = x;
+          }
+          float sc = acc[0];
+#pragma unroll
+          for (int j = 1; j < VPT; ++j) sc += acc[j];
+          if (TPT == 2) sc += __shfl_xor_sync(0xFFFFFFFFu, sc, 1);
+          if (sub == 0 && tok < cnt) {
+            out[tok] = sc;
+            atomicAdd(&hist[float_to_ordered(sc) >> 20], 1u);
+          }
+        }
+      }
+      __syncwarp();
+      if ((tid & 31) == 0) mbar_arrive(&empty[s]);
+      chunk_advance(c, per_head, a.B, a.Hkv);
     }
-    // one barrier per chunk: everyone is done with stage s, and all agree on a timeout
-    if (__syncthreads_or(!ok)) { aborted = true; break; }
-    if (tid == 0 && it + kScoreStages < n_mine) issue(it + kScoreStages);
-  }
-  if (aborted) {
-    if (tid == 0) {
-      // give every copy still in flight a bounded chance to land before the CTA exits
-      for (int64_t j = it; j < min64(it + kScoreStages, n_mine); ++j) {
-        const int s = static_cast<int>(j % kScoreStages);
-        mbar_wait_bounded(&bars[s], static_cast<uint32_t>((j / kScoreStages) & 1), a.status, 100000000ull);
+    consumers_sync();
+    if (a.hist && cur_row >= 0) {
+      uint32_t* g = a.hist + static_cast<int64_t>(cur_row) * kHistBins;
+      for (int i = tid; i < kHistBins; i += kScoreConsumers) {
+        const uint32_t v = hist[i];
+        if (v) atomicAdd(g + i, v);
       }
     }
-    return;
   }
-  if (cur_row >= 0) flush(cur_row);
+  __syncthreads();
+  if (aborted && tid == kScoreConsumers) {
+    // give every copy still in flight a bounded chance to land before the CTA exits
+    for (int s = 0; s < kScoreStages; ++s) {
+      for (int par = 0; par < 2; ++par) mbar_wait_bounded(&full[s], par, nullptr, 50000000ull);
+    }
+  }
 }
 
 template <int R>
 static cudaError_t launch_score_r(const ScoreArgs& a, int num_sms, cudaStream_t s) {
-  const size_t smem = kScoreStages * kChunkBytes + kScoreStages * sizeof(uint64_t) + kHistBins * sizeof(uint32_t) +
-                      (2 * a.B + 1) * sizeof(int64_t);
+  const size_t smem = kScoreStages * kChunkBytes + 2 * kScoreStages * sizeof(uint64_t) +
+                      kHistBins * sizeof(uint32_t) + (3 * a.B + 1) * sizeof(int64_t);
   static int done[64] = {0};
   cudaError_t e = set_smem_limit_once(score_kernel<R>, smem, done);
   if (e != cudaSuccess) return e;
-  const int grid = num_sms * 2;
+  const int grid = num_sms * 3;
   score_kernel<R><<<grid, kScoreThreads, smem, s>>>(a);
   return cudaGetLastError();
 }

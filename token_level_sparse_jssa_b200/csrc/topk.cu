@@ -11,17 +11,21 @@
 //   digit 1 (key bits 31..20): from the row's histogram, which the score scan builds
 //           as it streams the projected cache (or topk_hist_kernel for standalone
 //           calls); every CTA finds the digit itself.
-//   digits 2 and 3 (bits 19..10, 9..0): each CTA histograms the keys of its slice that
-//           match the prefix so far, adds the non-zero bins into rank 0's shared memory
+//   scan 1 (whole slice): each warp counts its keys above bin D1 and appends the keys
+//           inside bin D1 (about 1 % of them for the workloads here) to a candidate list.
+//   digits 2 and 3 (bits 19..10, 9..0): each CTA histograms the candidates matching the
+//           prefix so far, adds the non-zero bins into rank 0's shared memory
 //           (distributed shared memory atomics), and after a cluster barrier every CTA
-//           reads the totals back and finds the digit.
-//   compaction: every key > K* plus, in index order, the first `need` keys == K*.  Each
-//           warp owns a contiguous piece of the slice; ballots give in-warp order, and
-//           per-warp / per-CTA counts exchanged across the cluster give each output
-//           position.
+//           reads the totals back and finds the digit.  A CTA whose candidates overflow
+//           the list scans its whole slice instead (same barriers, same result).
+//   write scan (whole slice): every key > K* plus, in index order, the first `need`
+//           keys == K*.  Each warp owns a contiguous piece of the slice; ballots give
+//           in-warp order, and per-warp / per-CTA counts exchanged across the cluster
+//           give each output position.
 //
 // Each CTA's slice of scores is staged once into shared memory with one bulk copy
-// (TMA engine).  Four cluster barriers in total; cluster barriers are hardware
+// (TMA engine); rows of 128K tokens use 16-CTA clusters (8192 keys per CTA) where
+// the device can co-schedule them.  Four cluster barriers in total; cluster barriers are hardware
 // barriers over co-scheduled CTAs, so no wait here can hang; the bulk-copy wait is
 // bounded in time.
 #include <cooperative_groups.h>
@@ -37,9 +41,10 @@ constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kBins1 = 4096;   // digit 1: key bits [31:20]
 constexpr int kBins2 = 1024;   // digits 2 and 3: bits [19:10] and [9:0]
-constexpr int kMaxCluster = 8;
-constexpr int kSliceTarget = 16384;   // keys per CTA the cluster size aims for
-constexpr int kMaxStaged = 40960;     // keys per CTA that still fit in shared memory
+constexpr int kMaxCluster = 16;
+constexpr int kSliceTarget = 8192;    // keys per CTA the cluster size aims for
+constexpr int kMaxStaged = 32768;     // keys per CTA that still fit in shared memory
+constexpr int kMaxCand = 4096;        // keys of the digit-1 bin kept as candidates per CTA
 
 // Exclusive prefix sum over the block; returns the sum over lower-numbered threads and
 // writes the block total.
@@ -112,8 +117,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   uint32_t* hloc = reinterpret_cast<uint32_t*>(fs + per_cap);          // [kBins2] this CTA's histogram
   uint32_t* totA = hloc + kBins2;                                       // [kBins2] digit-2 totals (rank 0)
   uint32_t* totB = totA + kBins2;                                       // [kBins2] digit-3 totals (rank 0)
+  uint32_t* cand = totB + kBins2;                                       // [kMaxCand] slice offsets in bin D1
   __shared__ uint64_t bar;
-  __shared__ uint32_t dig, krem_s;
+  __shared__ uint32_t dig, krem_s, ncand;
   __shared__ uint32_t cta_gt[kMaxCluster], cta_eq[kMaxCluster];
   __shared__ uint32_t warp_gt[kTopkWarps], warp_eq[kTopkWarps];
   __shared__ uint32_t scan_tmp[32];
@@ -127,31 +133,35 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     T = T < 0 ? 0 : a.T_cap;
   }
   const int64_t W = min64(max64(a.window, 0), T);
-  const int64_t n = T - W;
-  const int64_t k_eff = min64(a.k, n);
+  const int n = static_cast<int>(T - W);
+  const int k_eff = static_cast<int>(min64(a.k, n));
   int32_t* out = a.idx + static_cast<int64_t>(row) * a.k;
-  if (crank == 0 && tid == 0) a.n_sel[row] = static_cast<int32_t>(k_eff);
-  for (int64_t j = k_eff + crank * kTopkThreads + tid; j < a.k; j += static_cast<int64_t>(C) * kTopkThreads) out[j] = -1;
+  if (crank == 0 && tid == 0) a.n_sel[row] = k_eff;
+  for (int j = k_eff + crank * kTopkThreads + tid; j < a.k; j += C * kTopkThreads) out[j] = -1;
   if (k_eff == n) {  // everything is selected (includes n == 0)
-    for (int64_t j = crank * kTopkThreads + tid; j < n; j += static_cast<int64_t>(C) * kTopkThreads)
-      out[j] = static_cast<int32_t>(j);
+    for (int j = crank * kTopkThreads + tid; j < n; j += C * kTopkThreads) out[j] = j;
     return;
   }
 
-  // this CTA's slice [lo, lo + len)
-  const int64_t per = ceil_div(ceil_div(n, C), 4) * 4;
-  const int64_t lo = crank * per;
-  const int len = static_cast<int>(max64(0, min64(n, lo + per) - lo));
+  // this CTA's slice [lo, lo + len); warp w owns [w * wc, min(len, (w + 1) * wc))
+  const int per = (((n + C - 1) / C) + 3) & ~3;
+  const int lo = crank * per;
+  const int len = max(0, min(n, lo + per) - lo);
+  const int wc = ((len + kTopkWarps - 1) / kTopkWarps + 31) & ~31;
   const float* srow = a.scores + static_cast<int64_t>(row) * a.sc_ld + lo;
   bool staged_ok = true;
-  if (STAGED) {
-    const bool bulk = (reinterpret_cast<uintptr_t>(srow) & 15u) == 0;
-    const int nbulk = bulk ? (len & ~3) : 0;
-    if (tid == 0) {
+  if (tid == 0) {
+    ncand = 0;
+    if (STAGED) {
       mbar_init(&bar, 1);
       fence_mbarrier_init();
     }
-    __syncthreads();
+  }
+  if (tid < kTopkWarps) { warp_gt[tid] = 0; warp_eq[tid] = 0; }
+  __syncthreads();
+  if (STAGED) {
+    const bool bulk = (reinterpret_cast<uintptr_t>(srow) & 15u) == 0;
+    const int nbulk = bulk ? (len & ~3) : 0;
     if (tid == 0 && nbulk > 0) {
       mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nbulk) * 4u);
       bulk_g2s(fs, srow, static_cast<uint32_t>(nbulk) * 4u, &bar, l2_policy_evict_first());
@@ -163,22 +173,54 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
 
   if (crank == 0)
     for (int i = tid; i < kBins2; i += kTopkThreads) { totA[i] = 0; totB[i] = 0; }
-  // digit 1 from the global histogram (every CTA computes the same digit)
+  // digit 1 from the row's global histogram (every CTA computes the same digit)
   find_digit<kBins1>(a.hist + static_cast<int64_t>(row) * kBins1, static_cast<uint32_t>(k_eff), scan_tmp, &dig,
                      &krem_s);
-  uint32_t prefix = dig << 20, mask = 0xFFF00000u, krem = krem_s;
+  const uint32_t d1 = dig;
+  uint32_t krem = krem_s;
   const bool aborted = __syncthreads_or(!staged_ok);
+
+  // scan 1: per warp, the keys above bin d1; the keys inside bin d1 become candidates
+  const int w_lo = warp * wc, w_hi = aborted ? w_lo : min(len, w_lo + wc);
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  {
+    uint32_t above = 0;
+    for (int base = w_lo; base < w_hi; base += 32) {
+      const int i = base + lane;
+      const uint32_t key = (i < w_hi) ? key_at(i) : 0u;
+      const uint32_t dk = key >> 20;
+      above += __popc(__ballot_sync(0xFFFFFFFFu, i < w_hi && dk > d1));
+      const uint32_t m = __ballot_sync(0xFFFFFFFFu, i < w_hi && dk == d1);
+      if (m) {
+        uint32_t off = 0;
+        if (lane == 0) off = atomicAdd(&ncand, __popc(m));
+        off = __shfl_sync(0xFFFFFFFFu, off, 0);
+        const uint32_t p = off + __popc(m & lt_mask);
+        if (((m >> lane) & 1u) && p < kMaxCand) cand[p] = static_cast<uint32_t>(i);
+      }
+    }
+    if (lane == 0) warp_gt[warp] = above;
+  }
+  __syncthreads();
+  const int nc = static_cast<int>(ncand);
+  const bool overflow = nc > kMaxCand;   // fall back to scanning the whole slice
   cluster.sync();  // rank 0's totals are zero and every CTA of the cluster is running
 
   uint32_t* totA0 = cluster.map_shared_rank(totA, 0);
   uint32_t* totB0 = cluster.map_shared_rank(totB, 0);
+  uint32_t prefix = d1 << 20, mask = 0xFFF00000u;
 #pragma unroll 1
   for (int pass = 0; pass < 2; ++pass) {
     const int shift = (pass == 0) ? 10 : 0;
     uint32_t* tot0 = (pass == 0) ? totA0 : totB0;
     for (int i = tid; i < kBins2; i += kTopkThreads) hloc[i] = 0;
     __syncthreads();
-    if (!aborted) {
+    if (!overflow) {
+      for (int j = tid; j < nc; j += kTopkThreads) {
+        const uint32_t key = key_at(static_cast<int>(cand[j]));
+        if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kBins2 - 1)], 1u);
+      }
+    } else if (!aborted) {
       for (int i = tid; i < len; i += kTopkThreads) {
         const uint32_t key = key_at(i);
         if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kBins2 - 1)], 1u);
@@ -198,17 +240,24 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   const uint32_t kstar = prefix;  // the k-th largest key
   const uint32_t need = krem;     // keys equal to kstar to take, lowest index first
 
-  // ---- ordered compaction: warp w owns [w*wc, min(len, (w+1)*wc))
-  const int wc = static_cast<int>(ceil_div(ceil_div(len, kTopkWarps), 32) * 32);
-  const int w_lo = warp * wc, w_hi = aborted ? w_lo : min(len, w_lo + wc);
-  uint32_t ngt = 0, neq = 0;
-  for (int base = w_lo; base < w_hi; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = (i < w_hi) ? key_at(i) : 0u;
-    ngt += __popc(__ballot_sync(0xFFFFFFFFu, i < w_hi && key > kstar));
-    neq += __popc(__ballot_sync(0xFFFFFFFFu, i < w_hi && key == kstar));
+  // per-warp counts of keys > kstar and == kstar
+  if (!overflow) {
+    for (int j = tid; j < nc; j += kTopkThreads) {
+      const int i = static_cast<int>(cand[j]);
+      const uint32_t key = key_at(i);
+      if (key > kstar) atomicAdd(&warp_gt[i / wc], 1u);
+      else if (key == kstar) atomicAdd(&warp_eq[i / wc], 1u);
+    }
+  } else {
+    uint32_t ngt = 0, neq = 0;
+    for (int base = w_lo; base < w_hi; base += 32) {
+      const int i = base + lane;
+      const uint32_t key = (i < w_hi) ? key_at(i) : 0u;
+      ngt += __popc(__ballot_sync(0xFFFFFFFFu, i < w_hi && key > kstar && (key >> 20) == d1));
+      neq += __popc(__ballot_sync(0xFFFFFFFFu, i < w_hi && key == kstar));
+    }
+    if (lane == 0) { warp_gt[warp] += ngt; warp_eq[warp] = neq; }
   }
-  if (lane == 0) { warp_gt[warp] = ngt; warp_eq[warp] = neq; }
   __syncthreads();
   if (tid < C) {
     uint32_t g = 0, e = 0;
@@ -218,7 +267,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   }
   cluster.sync();  // last access to another CTA's shared memory
   if (aborted) {  // the staging copy never completed (flagged): report an empty selection
-    for (int64_t j = crank * kTopkThreads + tid; j < k_eff; j += static_cast<int64_t>(C) * kTopkThreads) out[j] = -1;
+    for (int j = crank * kTopkThreads + tid; j < k_eff; j += C * kTopkThreads) out[j] = -1;
     return;
   }
   uint32_t base_out = 0, eq_before = 0;
@@ -234,7 +283,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     pos += warp_gt[w] + q;
     eq_rank += warp_eq[w];
   }
-  const uint32_t lt_mask = (1u << lane) - 1u;
+  // write scan: every key > kstar, and keys == kstar while the quota lasts, in index order
   for (int base = w_lo; base < w_hi; base += 32) {
     const int i = base + lane;
     const uint32_t key = (i < w_hi) ? key_at(i) : 0u;
@@ -245,7 +294,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     const uint32_t sel_m = __ballot_sync(0xFFFFFFFFu, sel);
     if (sel) {
       const uint32_t p = pos + __popc(sel_m & lt_mask);
-      if (p < static_cast<uint32_t>(k_eff)) out[p] = static_cast<int32_t>(lo + i);
+      if (p < static_cast<uint32_t>(k_eff)) out[p] = lo + i;
       else flag_error(a.status, DEVFLAG_BAD_INDEX);  // unreachable when the counts are consistent
     }
     pos += __popc(sel_m);
@@ -282,18 +331,62 @@ cudaError_t launch_topk_histogram(const TopkArgs& a, int, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// Largest cluster size (power of two, <= kMaxCluster) that the device can co-schedule
+// for this kernel and shared-memory size, cached per device.
+static int max_cluster_for(void (*kern)(TopkArgs, int), size_t smem) {
+  static int cache[64][2] = {{0}};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
+  const int slot = (kern == topk_kernel<true>) ? 0 : 1;
+  if (cache[dev][slot]) return cache[dev][slot];
+  int best = 8;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) == cudaSuccess &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kMaxCluster, 1, 1);
+    cfg.blockDim = dim3(kTopkThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kMaxCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) best = kMaxCluster;
+  }
+  cudaGetLastError();  // clear a refused query
+  cache[dev][slot] = best;
+  return best;
+}
+
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   const int64_t n_max = a.T_cap;
+  void (*kern)(TopkArgs, int) = nullptr;
   int C = 1;
-  while (C < kMaxCluster && ceil_div(n_max, C) > kSliceTarget) C *= 2;
-  const int64_t per = ceil_div(ceil_div(n_max, C), 4) * 4;
+  while (C < 8 && ceil_div(n_max, C) > kSliceTarget) C *= 2;
+  int64_t per = ceil_div(ceil_div(n_max, C), 4) * 4;
+  // the staged slice must fit in shared memory; prefer a larger cluster when allowed
+  const size_t fixed = (3 * kBins2 + kMaxCand) * sizeof(uint32_t);
+  if (per > kSliceTarget) {
+    const int cmax = max_cluster_for(topk_kernel<true>, fixed + sizeof(float) * ceil_div(ceil_div(n_max, kMaxCluster), 4) * 4);
+    if (cmax >= kMaxCluster) {
+      C = kMaxCluster;
+      per = ceil_div(ceil_div(n_max, C), 4) * 4;
+    }
+  }
   const bool staged = per <= kMaxStaged;
+  kern = staged ? topk_kernel<true> : topk_kernel<false>;
   const int per_cap = staged ? static_cast<int>(per) : 0;
-  const size_t smem = static_cast<size_t>(per_cap) * sizeof(float) + 3 * kBins2 * sizeof(uint32_t);
-  void (*kern)(TopkArgs, int) = staged ? topk_kernel<true> : topk_kernel<false>;
+  const size_t smem = fixed + static_cast<size_t>(per_cap) * sizeof(float);
   static int done_staged[64] = {0}, done_plain[64] = {0};
   cudaError_t e = set_smem_limit_once(kern, smem, staged ? done_staged : done_plain);
   if (e != cudaSuccess) return e;
+  if (C > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, a.B * a.Hkv, 1);
   cfg.blockDim = dim3(kTopkThreads, 1, 1);
