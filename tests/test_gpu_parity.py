@@ -150,6 +150,23 @@ def _topk_layout(B, T):
     return L
 
 
+def test_topk_with_the_winners_bunched_together():
+    # increasing scores: all winners sit in the last warps' ranges (their lists overflow)
+    B, T, k = 2, 131072, 3000
+    scores = torch.arange(B * T, dtype=torch.float32).view(B, T).cuda() / 7.0
+    scores[1] = scores[1].flip(0)
+    L = _topk_layout(B, T)
+    sl = torch.tensor([T, T - 5], dtype=torch.int32, device="cuda")
+    idx = torch.empty((B, 1, k), dtype=torch.int32, device="cuda")
+    nsel = torch.empty((B, 1), dtype=torch.int32, device="cuda")
+    ws = jssa.alloc_workspace(L, k, 0)
+    jssa.topk(L, scores, sl, k, 0, idx, nsel, ws)
+    torch.cuda.synchronize()
+    _assert_status_clean(ws)
+    np.testing.assert_array_equal(idx[0, 0].cpu().numpy(), np.arange(T - k, T))
+    np.testing.assert_array_equal(idx[1, 0].cpu().numpy(), np.arange(k))
+
+
 @pytest.mark.parametrize("T,k,levels", [(131072, 2048, 1), (131072, 5000, 3), (70000, 300, 2)])
 def test_topk_with_few_distinct_values(T, k, levels):
     # every key of a slice falls in one digit-1 bin: the candidate list overflows and the

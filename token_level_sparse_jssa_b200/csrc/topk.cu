@@ -11,21 +11,21 @@
 //   digit 1 (key bits 31..20): from the row's histogram, which the score scan builds
 //           as it streams the projected cache (or topk_hist_kernel for standalone
 //           calls); every CTA finds the digit itself.
-//   scan 1 (whole slice): each warp counts its keys above bin D1 and appends the keys
-//           inside bin D1 (about 1 % of them for the workloads here) to a candidate list.
+//   scan 1 (the only pass over the whole slice): each warp lists, in index order, its
+//           keys above bin D1 ("definites", all selected) and inside bin D1
+//           ("candidates", about 1 % of the keys for the workloads here).
 //   digits 2 and 3 (bits 19..10, 9..0): each CTA histograms the candidates matching the
 //           prefix so far, adds the non-zero bins into rank 0's shared memory
 //           (distributed shared memory atomics), and after a cluster barrier every CTA
-//           reads the totals back and finds the digit.  A CTA whose candidates overflow
-//           the list scans its whole slice instead (same barriers, same result).
-//   write scan (whole slice): every key > K* plus, in index order, the first `need`
-//           keys == K*.  Each warp owns a contiguous piece of the slice; ballots give
-//           in-warp order, and per-warp / per-CTA counts exchanged across the cluster
-//           give each output position.
+//           reads the totals back and finds the digit.  A warp whose candidates overflow
+//           its list rescans its own range instead (same barriers, same result).
+//   output: every key > K* plus, in index order, the first `need` keys == K*.  Per-warp
+//           and per-CTA counts exchanged across the cluster give each warp its output
+//           position; a warp marks its selected offsets in a bitmap and emits them in
+//           order (or, with overflowing lists, rescans its range with ballots).
 //
 // Each CTA's slice of scores is staged once into shared memory with one bulk copy
-// (TMA engine); rows of 128K tokens use 16-CTA clusters (8192 keys per CTA) where
-// the device can co-schedule them.  Four cluster barriers in total; cluster barriers are hardware
+// (TMA engine).  Four cluster barriers in total; cluster barriers are hardware
 // barriers over co-scheduled CTAs, so no wait here can hang; the bulk-copy wait is
 // bounded in time.
 #include <cooperative_groups.h>
@@ -41,10 +41,11 @@ constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kBins1 = 4096;   // digit 1: key bits [31:20]
 constexpr int kBins2 = 1024;   // digits 2 and 3: bits [19:10] and [9:0]
-constexpr int kMaxCluster = 16;
-constexpr int kSliceTarget = 8192;    // keys per CTA the cluster size aims for
+constexpr int kMaxCluster = 8;
+constexpr int kSliceTarget = 16384;   // keys per CTA the cluster size aims for
 constexpr int kMaxStaged = 32768;     // keys per CTA that still fit in shared memory
-constexpr int kMaxCand = 4096;        // keys of the digit-1 bin kept as candidates per CTA
+constexpr int kCapW = 64;             // per-warp capacity of the definite and candidate lists
+constexpr int kMaskWords = 64;        // per-warp output bitmap: ranges of up to 2048 keys
 
 // Exclusive prefix sum over the block; returns the sum over lower-numbered threads and
 // writes the block total.
@@ -117,9 +118,11 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   uint32_t* hloc = reinterpret_cast<uint32_t*>(fs + per_cap);          // [kBins2] this CTA's histogram
   uint32_t* totA = hloc + kBins2;                                       // [kBins2] digit-2 totals (rank 0)
   uint32_t* totB = totA + kBins2;                                       // [kBins2] digit-3 totals (rank 0)
-  uint32_t* cand = totB + kBins2;                                       // [kMaxCand] slice offsets in bin D1
+  uint32_t* defs = totB + kBins2;                                       // [warps][kCapW] keys above bin D1
+  uint32_t* cands = defs + kTopkWarps * kCapW;                          // [warps][kCapW] keys inside bin D1
+  uint32_t* masks = cands + kTopkWarps * kCapW;                         // [warps][kMaskWords] output bitmaps
   __shared__ uint64_t bar;
-  __shared__ uint32_t dig, krem_s, ncand;
+  __shared__ uint32_t dig, krem_s;
   __shared__ uint32_t cta_gt[kMaxCluster], cta_eq[kMaxCluster];
   __shared__ uint32_t warp_gt[kTopkWarps], warp_eq[kTopkWarps];
   __shared__ uint32_t scan_tmp[32];
@@ -143,21 +146,17 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     return;
   }
 
-  // this CTA's slice [lo, lo + len); warp w owns [w * wc, min(len, (w + 1) * wc))
+  // this CTA's slice [lo, lo + len); warp w owns slice offsets [w * wc, min(len, (w + 1) * wc))
   const int per = (((n + C - 1) / C) + 3) & ~3;
   const int lo = crank * per;
   const int len = max(0, min(n, lo + per) - lo);
   const int wc = ((len + kTopkWarps - 1) / kTopkWarps + 31) & ~31;
   const float* srow = a.scores + static_cast<int64_t>(row) * a.sc_ld + lo;
   bool staged_ok = true;
-  if (tid == 0) {
-    ncand = 0;
-    if (STAGED) {
-      mbar_init(&bar, 1);
-      fence_mbarrier_init();
-    }
+  if (STAGED && tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
   }
-  if (tid < kTopkWarps) { warp_gt[tid] = 0; warp_eq[tid] = 0; }
   __syncthreads();
   if (STAGED) {
     const bool bulk = (reinterpret_cast<uintptr_t>(srow) & 15u) == 0;
@@ -180,30 +179,32 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   uint32_t krem = krem_s;
   const bool aborted = __syncthreads_or(!staged_ok);
 
-  // scan 1: per warp, the keys above bin d1; the keys inside bin d1 become candidates
+  // scan 1, the only pass over the whole slice: each warp lists (in index order) its keys
+  // above bin d1 ("definites", all selected) and inside bin d1 ("candidates")
   const int w_lo = warp * wc, w_hi = aborted ? w_lo : min(len, w_lo + wc);
   const uint32_t lt_mask = (1u << lane) - 1u;
-  {
-    uint32_t above = 0;
-    for (int base = w_lo; base < w_hi; base += 32) {
-      const int i = base + lane;
-      const uint32_t key = (i < w_hi) ? key_at(i) : 0u;
-      const uint32_t dk = key >> 20;
-      above += __popc(__ballot_sync(0xFFFFFFFFu, i < w_hi && dk > d1));
-      const uint32_t m = __ballot_sync(0xFFFFFFFFu, i < w_hi && dk == d1);
-      if (m) {
-        uint32_t off = 0;
-        if (lane == 0) off = atomicAdd(&ncand, __popc(m));
-        off = __shfl_sync(0xFFFFFFFFu, off, 0);
-        const uint32_t p = off + __popc(m & lt_mask);
-        if (((m >> lane) & 1u) && p < kMaxCand) cand[p] = static_cast<uint32_t>(i);
-      }
+  uint32_t* my_defs = defs + warp * kCapW;
+  uint32_t* my_cands = cands + warp * kCapW;
+  uint32_t nd = 0, nca = 0;
+  for (int base = w_lo; base < w_hi; base += 32) {
+    const int i = base + lane;
+    const bool valid = i < w_hi;
+    const uint32_t dk = valid ? (key_at(i) >> 20) : 0u;
+    const bool isdef = valid && dk > d1, iscand = valid && dk == d1;
+    const uint32_t mdef = __ballot_sync(0xFFFFFFFFu, isdef);
+    const uint32_t mcan = __ballot_sync(0xFFFFFFFFu, iscand);
+    if (isdef) {
+      const uint32_t p = nd + __popc(mdef & lt_mask);
+      if (p < kCapW) my_defs[p] = static_cast<uint32_t>(i);
     }
-    if (lane == 0) warp_gt[warp] = above;
+    if (iscand) {
+      const uint32_t p = nca + __popc(mcan & lt_mask);
+      if (p < kCapW) my_cands[p] = static_cast<uint32_t>(i);
+    }
+    nd += __popc(mdef);
+    nca += __popc(mcan);
   }
-  __syncthreads();
-  const int nc = static_cast<int>(ncand);
-  const bool overflow = nc > kMaxCand;   // fall back to scanning the whole slice
+  const bool cand_list = nca <= kCapW;   // warp-uniform: else this warp rescans its range
   cluster.sync();  // rank 0's totals are zero and every CTA of the cluster is running
 
   uint32_t* totA0 = cluster.map_shared_rank(totA, 0);
@@ -215,13 +216,13 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     uint32_t* tot0 = (pass == 0) ? totA0 : totB0;
     for (int i = tid; i < kBins2; i += kTopkThreads) hloc[i] = 0;
     __syncthreads();
-    if (!overflow) {
-      for (int j = tid; j < nc; j += kTopkThreads) {
-        const uint32_t key = key_at(static_cast<int>(cand[j]));
+    if (cand_list) {
+      for (int j = lane; j < static_cast<int>(nca); j += 32) {
+        const uint32_t key = key_at(static_cast<int>(my_cands[j]));
         if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kBins2 - 1)], 1u);
       }
-    } else if (!aborted) {
-      for (int i = tid; i < len; i += kTopkThreads) {
+    } else {
+      for (int i = w_lo + lane; i < w_hi; i += 32) {
         const uint32_t key = key_at(i);
         if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kBins2 - 1)], 1u);
       }
@@ -240,23 +241,25 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   const uint32_t kstar = prefix;  // the k-th largest key
   const uint32_t need = krem;     // keys equal to kstar to take, lowest index first
 
-  // per-warp counts of keys > kstar and == kstar
-  if (!overflow) {
-    for (int j = tid; j < nc; j += kTopkThreads) {
-      const int i = static_cast<int>(cand[j]);
-      const uint32_t key = key_at(i);
-      if (key > kstar) atomicAdd(&warp_gt[i / wc], 1u);
-      else if (key == kstar) atomicAdd(&warp_eq[i / wc], 1u);
+  // per-warp counts of keys > kstar (all definites + candidates above) and == kstar
+  {
+    uint32_t ngt = nd, neq = 0;
+    if (cand_list) {
+      for (int j0 = 0; j0 < static_cast<int>(nca); j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t key = (j < static_cast<int>(nca)) ? key_at(static_cast<int>(my_cands[j])) : 0u;
+        ngt += __popc(__ballot_sync(0xFFFFFFFFu, j < static_cast<int>(nca) && key > kstar));
+        neq += __popc(__ballot_sync(0xFFFFFFFFu, j < static_cast<int>(nca) && key == kstar));
+      }
+    } else {
+      for (int base = w_lo; base < w_hi; base += 32) {
+        const int i = base + lane;
+        const uint32_t key = (i < w_hi) ? key_at(i) : 0u;
+        ngt += __popc(__ballot_sync(0xFFFFFFFFu, i < w_hi && key > kstar && (key >> 20) == d1));
+        neq += __popc(__ballot_sync(0xFFFFFFFFu, i < w_hi && key == kstar));
+      }
     }
-  } else {
-    uint32_t ngt = 0, neq = 0;
-    for (int base = w_lo; base < w_hi; base += 32) {
-      const int i = base + lane;
-      const uint32_t key = (i < w_hi) ? key_at(i) : 0u;
-      ngt += __popc(__ballot_sync(0xFFFFFFFFu, i < w_hi && key > kstar && (key >> 20) == d1));
-      neq += __popc(__ballot_sync(0xFFFFFFFFu, i < w_hi && key == kstar));
-    }
-    if (lane == 0) { warp_gt[warp] += ngt; warp_eq[warp] = neq; }
+    if (lane == 0) { warp_gt[warp] = ngt; warp_eq[warp] = neq; }
   }
   __syncthreads();
   if (tid < C) {
@@ -270,6 +273,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     for (int j = crank * kTopkThreads + tid; j < k_eff; j += C * kTopkThreads) out[j] = -1;
     return;
   }
+  // output base and quota of keys == kstar: of this CTA, then of this warp
   uint32_t base_out = 0, eq_before = 0;
   for (int c = 0; c < crank; ++c) {
     const uint32_t q = (need > eq_before) ? min(cta_eq[c], need - eq_before) : 0u;
@@ -283,22 +287,74 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     pos += warp_gt[w] + q;
     eq_rank += warp_eq[w];
   }
-  // write scan: every key > kstar, and keys == kstar while the quota lasts, in index order
-  for (int base = w_lo; base < w_hi; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = (i < w_hi) ? key_at(i) : 0u;
-    const bool gt = i < w_hi && key > kstar;
-    const bool eq = i < w_hi && key == kstar;
-    const uint32_t eq_m = __ballot_sync(0xFFFFFFFFu, eq);
-    const bool sel = gt || (eq && (eq_rank + __popc(eq_m & lt_mask)) < quota);
-    const uint32_t sel_m = __ballot_sync(0xFFFFFFFFu, sel);
-    if (sel) {
-      const uint32_t p = pos + __popc(sel_m & lt_mask);
-      if (p < static_cast<uint32_t>(k_eff)) out[p] = lo + i;
-      else flag_error(a.status, DEVFLAG_BAD_INDEX);  // unreachable when the counts are consistent
+  const uint32_t wquota = (quota > eq_rank) ? min(warp_eq[warp], quota - eq_rank) : 0u;
+  const int words = wc / 32;
+  if (cand_list && nd <= kCapW && words <= kMaskWords) {
+    // mark the selected offsets of this warp's range in a bitmap, then emit them in order
+    uint32_t* m = masks + warp * kMaskWords;
+    for (int j = lane; j < words; j += 32) m[j] = 0u;
+    __syncwarp();
+    for (int j = lane; j < static_cast<int>(nd); j += 32) {
+      const uint32_t o = my_defs[j] - static_cast<uint32_t>(w_lo);
+      atomicOr(&m[o >> 5], 1u << (o & 31));
     }
-    pos += __popc(sel_m);
-    eq_rank += __popc(eq_m);
+    uint32_t eq_run = 0;
+    for (int j0 = 0; j0 < static_cast<int>(nca); j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t i = (j < static_cast<int>(nca)) ? my_cands[j] : 0u;
+      const uint32_t key = (j < static_cast<int>(nca)) ? key_at(static_cast<int>(i)) : 0u;
+      const bool gt = j < static_cast<int>(nca) && key > kstar;
+      const bool eq = j < static_cast<int>(nca) && key == kstar;
+      const uint32_t eq_m = __ballot_sync(0xFFFFFFFFu, eq);
+      if (gt || (eq && (eq_run + __popc(eq_m & lt_mask)) < wquota)) {
+        const uint32_t o = i - static_cast<uint32_t>(w_lo);
+        atomicOr(&m[o >> 5], 1u << (o & 31));
+      }
+      eq_run += __popc(eq_m);
+    }
+    __syncwarp();
+    const uint32_t w0 = (lane < words) ? m[lane] : 0u;
+    const uint32_t w1 = (lane + 32 < words) ? m[lane + 32] : 0u;
+    uint32_t c0 = __popc(w0), c1 = __popc(w1);
+    uint32_t x0 = c0, x1 = c1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y0 = __shfl_up_sync(0xFFFFFFFFu, x0, off);
+      const uint32_t y1 = __shfl_up_sync(0xFFFFFFFFu, x1, off);
+      if (lane >= off) { x0 += y0; x1 += y1; }
+    }
+    const uint32_t tot0 = __shfl_sync(0xFFFFFFFFu, x0, 31);
+    uint32_t p0 = pos + x0 - c0, p1 = pos + tot0 + x1 - c1;
+    const int gbase = lo + w_lo;
+    for (uint32_t v = w0; v; v &= v - 1) {
+      if (p0 < static_cast<uint32_t>(k_eff)) out[p0] = gbase + lane * 32 + (__ffs(v) - 1);
+      else flag_error(a.status, DEVFLAG_BAD_INDEX);  // unreachable when the counts are consistent
+      ++p0;
+    }
+    for (uint32_t v = w1; v; v &= v - 1) {
+      if (p1 < static_cast<uint32_t>(k_eff)) out[p1] = gbase + (lane + 32) * 32 + (__ffs(v) - 1);
+      else flag_error(a.status, DEVFLAG_BAD_INDEX);
+      ++p1;
+    }
+  } else {
+    // long lists: rescan this warp's range and compact with ballots
+    uint32_t eq_run = 0;
+    for (int base = w_lo; base < w_hi; base += 32) {
+      const int i = base + lane;
+      const uint32_t key = (i < w_hi) ? key_at(i) : 0u;
+      const bool gt = i < w_hi && key > kstar;
+      const bool eq = i < w_hi && key == kstar;
+      const uint32_t eq_m = __ballot_sync(0xFFFFFFFFu, eq);
+      const bool sel = gt || (eq && (eq_run + __popc(eq_m & lt_mask)) < wquota);
+      const uint32_t sel_m = __ballot_sync(0xFFFFFFFFu, sel);
+      if (sel) {
+        const uint32_t p = pos + __popc(sel_m & lt_mask);
+        if (p < static_cast<uint32_t>(k_eff)) out[p] = lo + i;
+        else flag_error(a.status, DEVFLAG_BAD_INDEX);
+      }
+      pos += __popc(sel_m);
+      eq_run += __popc(eq_m);
+    }
   }
 }
 
@@ -331,62 +387,19 @@ cudaError_t launch_topk_histogram(const TopkArgs& a, int, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-// Largest cluster size (power of two, <= kMaxCluster) that the device can co-schedule
-// for this kernel and shared-memory size, cached per device.
-static int max_cluster_for(void (*kern)(TopkArgs, int), size_t smem) {
-  static int cache[64][2] = {{0}};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
-  const int slot = (kern == topk_kernel<true>) ? 0 : 1;
-  if (cache[dev][slot]) return cache[dev][slot];
-  int best = 8;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) == cudaSuccess &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kMaxCluster, 1, 1);
-    cfg.blockDim = dim3(kTopkThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kMaxCluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) best = kMaxCluster;
-  }
-  cudaGetLastError();  // clear a refused query
-  cache[dev][slot] = best;
-  return best;
-}
-
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   const int64_t n_max = a.T_cap;
-  void (*kern)(TopkArgs, int) = nullptr;
   int C = 1;
-  while (C < 8 && ceil_div(n_max, C) > kSliceTarget) C *= 2;
-  int64_t per = ceil_div(ceil_div(n_max, C), 4) * 4;
-  // the staged slice must fit in shared memory; prefer a larger cluster when allowed
-  const size_t fixed = (3 * kBins2 + kMaxCand) * sizeof(uint32_t);
-  if (per > kSliceTarget) {
-    const int cmax = max_cluster_for(topk_kernel<true>, fixed + sizeof(float) * ceil_div(ceil_div(n_max, kMaxCluster), 4) * 4);
-    if (cmax >= kMaxCluster) {
-      C = kMaxCluster;
-      per = ceil_div(ceil_div(n_max, C), 4) * 4;
-    }
-  }
+  while (C < kMaxCluster && ceil_div(n_max, C) > kSliceTarget) C *= 2;
+  const int64_t per = ceil_div(ceil_div(n_max, C), 4) * 4;
   const bool staged = per <= kMaxStaged;
-  kern = staged ? topk_kernel<true> : topk_kernel<false>;
+  void (*kern)(TopkArgs, int) = staged ? topk_kernel<true> : topk_kernel<false>;
   const int per_cap = staged ? static_cast<int>(per) : 0;
-  const size_t smem = fixed + static_cast<size_t>(per_cap) * sizeof(float);
+  const size_t smem = static_cast<size_t>(per_cap) * sizeof(float) +
+                      (3 * kBins2 + 2 * kTopkWarps * kCapW + kTopkWarps * kMaskWords) * sizeof(uint32_t);
   static int done_staged[64] = {0}, done_plain[64] = {0};
   cudaError_t e = set_smem_limit_once(kern, smem, staged ? done_staged : done_plain);
   if (e != cudaSuccess) return e;
-  if (C > 8) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, a.B * a.Hkv, 1);
   cfg.blockDim = dim3(kTopkThreads, 1, 1);
