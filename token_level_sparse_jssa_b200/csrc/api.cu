@@ -4,7 +4,7 @@
 #include <cstdio>
 #include <cstring>
 
-#include "../../include/jssa.h"
+#include "jssa.h"
 #include "common.cuh"
 #include "launch.h"
 

@@ -51,38 +51,68 @@ static size_t attn_smem_bytes() {
 }
 
 // Combine the S split partials of query heads [hq0, hq0 + G) into O (and lse):
-// O = sum_s w_s o_s / sum_s w_s with w_s = exp(lse_s - max lse); lse = max + log(sum w).
-// Run by the last CTA of a row to finish, on partials every CTA made visible with a
-// device-scope fence before counting itself in.
+// O = sum_s w_s o_s with w_s = exp(lse_s - M) / sum_s' exp(lse_s' - M), M = max lse;
+// lse = M + log(sum exp(lse_s - M)).  Run by the last CTA of a row to finish, on
+// partials every CTA made visible with a device-scope fence before counting itself
+// in.  The split weights go through shared memory (wsm: G * S floats); every thread
+// then issues all the loads of two outputs (up to 16 splits each) before using them,
+// so the merge costs about one memory round trip per two outputs.
+constexpr int kMergeUnroll = 16;
 template <int D>
-__device__ __forceinline__ void merge_row(const AttnArgs& a, int64_t hq0, int G) {
-  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-    const int head = i / D, dim = i % D;
-    const float* lse_s = a.part_lse + (hq0 + head) * a.S;
-    const float* o_s = a.part_o + (hq0 + head) * a.S * D + dim;
+__device__ __forceinline__ void merge_row(const AttnArgs& a, int64_t hq0, int G, float* wsm) {
+  const int S = a.S;
+  for (int i = threadIdx.x; i < G * S; i += blockDim.x) wsm[i] = __ldcg(a.part_lse + (hq0 + i / S) * S + i % S);
+  __syncthreads();
+  if (threadIdx.x < G) {
+    float* w = wsm + threadIdx.x * S;
     float M = -INFINITY;
-    for (int s = 0; s < a.S; ++s) M = fmaxf(M, __ldcg(lse_s + s));
-    float o = 0.f, L = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll 4
-      for (int s = 0; s < a.S; ++s) {
-        const float w = expf(__ldcg(lse_s + s) - M);
-        L += w;
-        o += w * __ldcg(o_s + static_cast<int64_t>(s) * D);
+    for (int s = 0; s < S; ++s) M = fmaxf(M, w[s]);
+    float L = 0.f;
+    if (M != -INFINITY)
+      for (int s = 0; s < S; ++s) { w[s] = expf(w[s] - M); L += w[s]; }
+    const float inv = (M != -INFINITY) ? 1.f / L : 0.f;
+    for (int s = 0; s < S; ++s) w[s] = (M != -INFINITY) ? w[s] * inv : 0.f;
+    if (a.lse) a.lse[hq0 + threadIdx.x] = (M == -INFINITY) ? -INFINITY : M + logf(L);
+  }
+  __syncthreads();
+  for (int i0 = threadIdx.x; i0 < G * D; i0 += 2 * blockDim.x) {
+    const int i1 = i0 + blockDim.x;
+    const bool has1 = i1 < G * D;
+    const int h0 = i0 / D, d0 = i0 % D, h1 = has1 ? i1 / D : h0, d1 = has1 ? i1 % D : d0;
+    const float* o0 = a.part_o + (hq0 + h0) * S * D + d0;
+    const float* o1 = a.part_o + (hq0 + h1) * S * D + d1;
+    float acc0 = 0.f, acc1 = 0.f;
+    for (int s0 = 0; s0 < S; s0 += kMergeUnroll) {
+      float v0[kMergeUnroll], v1[kMergeUnroll];
+#pragma unroll
+      for (int u = 0; u < kMergeUnroll; ++u) {
+        const bool ok = s0 + u < S;
+        v0[u] = ok ? __ldcg(o0 + static_cast<int64_t>(s0 + u) * D) : 0.f;
+        v1[u] = (ok && has1) ? __ldcg(o1 + static_cast<int64_t>(s0 + u) * D) : 0.f;
       }
-      o /= L;
+#pragma unroll
+      for (int u = 0; u < kMergeUnroll; ++u) {
+        if (s0 + u < S) {
+          acc0 = fmaf(wsm[h0 * S + s0 + u], v0[u], acc0);
+          acc1 = fmaf(wsm[h1 * S + s0 + u], v1[u], acc1);
+        }
+      }
     }
-    const int64_t q = hq0 + head;
-    if (a.out_bf16) static_cast<__nv_bfloat16*>(a.O)[q * D + dim] = __float2bfloat16_rn(o);
-    else static_cast<float*>(a.O)[q * D + dim] = o;
-    if (a.lse && dim == 0) a.lse[q] = (M == -INFINITY) ? -INFINITY : M + logf(L);
+    const int64_t q0 = hq0 + h0, q1 = hq0 + h1;
+    if (a.out_bf16) {
+      static_cast<__nv_bfloat16*>(a.O)[q0 * D + d0] = __float2bfloat16_rn(acc0);
+      if (has1) static_cast<__nv_bfloat16*>(a.O)[q1 * D + d1] = __float2bfloat16_rn(acc1);
+    } else {
+      static_cast<float*>(a.O)[q0 * D + d0] = acc0;
+      if (has1) static_cast<float*>(a.O)[q1 * D + d1] = acc1;
+    }
   }
 }
 
 // Count this CTA's finished partial in; the CTA that completes the row merges it and
 // re-arms the counter for the next call.
 template <int D>
-__device__ __forceinline__ void finish_split(const AttnArgs& a, int row, int64_t hq0, int G) {
+__device__ __forceinline__ void finish_split(const AttnArgs& a, int row, int64_t hq0, int G, float* wsm) {
   __shared__ int is_last;
   __threadfence();
   __syncthreads();
@@ -93,7 +123,7 @@ __device__ __forceinline__ void finish_split(const AttnArgs& a, int row, int64_t
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  merge_row<D>(a, hq0, G);
+  merge_row<D>(a, hq0, G, wsm);
   if (threadIdx.x == 0) a.counters[row] = 0;
 }
 
@@ -111,59 +141,23 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
   const int split = blockIdx.x, row = blockIdx.y;
   const int b = row / a.Hkv, h = row % a.Hkv;
   const int G = a.Hq / a.Hkv;
-  int64_t T = a.seq_lens[b];
-  if (T < 0 || T > a.T_cap) {
-    if (split == 0 && threadIdx.x == 0) flag_error(a.status, DEVFLAG_BAD_SEQ_LEN);
-    T = T < 0 ? 0 : a.T_cap;
-  }
-  int64_t list_len, win_start;
-  int64_t nsel = 0;
-  if (DENSE) {
-    win_start = (a.window > 0) ? max64(0, T - a.window) : 0;
-    list_len = T - win_start;
-  } else {
-    const int64_t Wc = min64(max64(a.window, 0), T);
-    win_start = T - Wc;
-    nsel = a.n_sel[row];
-    const int64_t nsel_max = min64(a.idx_ld, win_start);
-    if (nsel < 0 || nsel > nsel_max) {
-      if (split == 0 && threadIdx.x == 0) flag_error(a.status, DEVFLAG_BAD_NSEL);
-      nsel = nsel < 0 ? 0 : nsel_max;
-    }
-    list_len = nsel + Wc;
-  }
-  const int64_t my_lo = static_cast<int64_t>(split) * a.split_len;
-  const int my_len = static_cast<int>(max64(0, min64(list_len, my_lo + a.split_len) - my_lo));
   const int64_t hq0 = static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * G;
-
-  if (my_len == 0) {  // empty split: weight zero in the merge
-    for (int i = threadIdx.x; i < G * D; i += kAttnThreads) {
-      const int head = i / D, dim = i % D;
-      a.part_o[((hq0 + head) * a.S + split) * D + dim] = 0.f;
-      if (dim == 0) a.part_lse[(hq0 + head) * a.S + split] = -INFINITY;
-    }
-    finish_split<D>(a, row, hq0, G);
-    return;
-  }
+  const int64_t my_lo = static_cast<int64_t>(split) * a.split_len;
+  // Issue every independent load of the prologue before using any of them: the sequence
+  // length, the selection count, this split's index entries (speculatively, validated
+  // below) and the query fragments.
+  int64_t T = a.seq_lens[b];
+  int64_t nsel = DENSE ? 0 : a.n_sel[row];
+  constexpr int kPre = 4;  // index entries per thread loaded up front (splits up to 512 tokens)
+  int32_t pre[kPre];
   if (!DENSE) {
     const int32_t* irow = a.idx + static_cast<int64_t>(row) * a.idx_ld;
-    for (int j = threadIdx.x; j < my_len; j += kAttnThreads) {
-      const int64_t pos = my_lo + j;
-      int64_t t;
-      if (pos < nsel) {
-        t = irow[pos];
-        if (t < 0 || t >= win_start) {
-          flag_error(a.status, DEVFLAG_BAD_INDEX);
-          t = -1;
-        }
-      } else {
-        t = win_start + (pos - nsel);
-      }
-      tok_s[j] = static_cast<int32_t>(t);
+#pragma unroll
+    for (int u = 0; u < kPre; ++u) {
+      const int64_t pos = my_lo + threadIdx.x + u * kAttnThreads;
+      pre[u] = (threadIdx.x + u * kAttnThreads < a.split_len && pos < a.idx_ld) ? __ldg(irow + pos) : -1;
     }
-    __syncthreads();
   }
-
   // Q^T as MMA B fragments: head nt*8 + g, dims kk*16 + 2c (+8)
   uint32_t qf[NTILE][KSTEPS][2];
   const __nv_bfloat16* Qg = static_cast<const __nv_bfloat16*>(a.Q) + hq0 * D;
@@ -181,6 +175,58 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
         qf[nt][kk][1] = 0u;
       }
     }
+  }
+  if (T < 0 || T > a.T_cap) {
+    if (split == 0 && threadIdx.x == 0) flag_error(a.status, DEVFLAG_BAD_SEQ_LEN);
+    T = T < 0 ? 0 : a.T_cap;
+  }
+  int64_t list_len, win_start;
+  if (DENSE) {
+    win_start = (a.window > 0) ? max64(0, T - a.window) : 0;
+    list_len = T - win_start;
+  } else {
+    const int64_t Wc = min64(max64(a.window, 0), T);
+    win_start = T - Wc;
+    const int64_t nsel_max = min64(a.idx_ld, win_start);
+    if (nsel < 0 || nsel > nsel_max) {
+      if (split == 0 && threadIdx.x == 0) flag_error(a.status, DEVFLAG_BAD_NSEL);
+      nsel = nsel < 0 ? 0 : nsel_max;
+    }
+    list_len = nsel + Wc;
+  }
+  const int my_len = static_cast<int>(max64(0, min64(list_len, my_lo + a.split_len) - my_lo));
+
+  if (my_len == 0) {  // empty split: weight zero in the merge
+    for (int i = threadIdx.x; i < G * D; i += kAttnThreads) {
+      const int head = i / D, dim = i % D;
+      a.part_o[((hq0 + head) * a.S + split) * D + dim] = 0.f;
+      if (dim == 0) a.part_lse[(hq0 + head) * a.S + split] = -INFINITY;
+    }
+    finish_split<D>(a, row, hq0, G, reinterpret_cast<float*>(smem_raw));
+    return;
+  }
+  if (!DENSE) {
+    const int32_t* irow = a.idx + static_cast<int64_t>(row) * a.idx_ld;
+    auto resolve = [&](int j, int64_t t) {  // selected entry (validated) or window position
+      const int64_t pos = my_lo + j;
+      if (pos < nsel) {
+        if (t < 0 || t >= win_start) {
+          flag_error(a.status, DEVFLAG_BAD_INDEX);
+          t = -1;
+        }
+      } else {
+        t = win_start + (pos - nsel);
+      }
+      tok_s[j] = static_cast<int32_t>(t);
+    };
+#pragma unroll
+    for (int u = 0; u < kPre; ++u) {
+      const int j = threadIdx.x + u * kAttnThreads;
+      if (j < my_len) resolve(j, pre[u]);
+    }
+    for (int j = threadIdx.x + kPre * kAttnThreads; j < my_len; j += kAttnThreads)
+      resolve(j, (my_lo + j < nsel) ? irow[my_lo + j] : 0);
+    __syncthreads();
   }
 
   const float scale_log2 = a.sm_scale * kLog2e;
@@ -365,7 +411,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
     a.part_o[((hq0 + head) * a.S + split) * D + dim] = o;
     if (dim == 0) a.part_lse[(hq0 + head) * a.S + split] = lse;
   }
-  finish_split<D>(a, row, hq0, G);
+  finish_split<D>(a, row, hq0, G, reinterpret_cast<float*>(smem_raw));
 }
 
 // ------------------------------------------------------------------ LSE merge

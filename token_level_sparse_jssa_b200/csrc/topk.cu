@@ -10,22 +10,22 @@
 //
 //   digit 1 (key bits 31..20): from the row's histogram, which the score scan builds
 //           as it streams the projected cache (or topk_hist_kernel for standalone
-//           calls); every CTA finds the digit itself.
+//           calls); each CTA stages it with its slice and finds the digit itself.
 //   scan 1 (the only pass over the whole slice): each warp lists, in index order, its
 //           keys above bin D1 ("definites", all selected) and inside bin D1
 //           ("candidates", about 1 % of the keys for the workloads here).
-//   digits 2 and 3 (bits 19..10, 9..0): each CTA histograms the candidates matching the
-//           prefix so far, adds the non-zero bins into rank 0's shared memory
-//           (distributed shared memory atomics), and after a cluster barrier every CTA
-//           reads the totals back and finds the digit.  A warp whose candidates overflow
-//           its list rescans its own range instead (same barriers, same result).
+//   digits 2 and 3 (bits 19..10, 9..0): the candidate keys of the whole row are
+//           gathered into rank 0's shared memory (distributed shared memory stores);
+//           after one cluster barrier every CTA copies them and finds both digits
+//           locally.  If the candidates do not fit, the cluster instead resolves each
+//           digit with a histogram summed in rank 0 (atomics) and read back by all.
 //   output: every key > K* plus, in index order, the first `need` keys == K*.  Per-warp
 //           and per-CTA counts exchanged across the cluster give each warp its output
 //           position; a warp marks its selected offsets in a bitmap and emits them in
 //           order (or, with overflowing lists, rescans its range with ballots).
 //
 // Each CTA's slice of scores is staged once into shared memory with one bulk copy
-// (TMA engine).  Four cluster barriers in total; cluster barriers are hardware
+// (TMA engine).  Three cluster barriers (five when the gather overflows); cluster barriers are hardware
 // barriers over co-scheduled CTAs, so no wait here can hang; the bulk-copy wait is
 // bounded in time.
 #include <cooperative_groups.h>
@@ -46,6 +46,7 @@ constexpr int kSliceTarget = 16384;   // keys per CTA the cluster size aims for
 constexpr int kMaxStaged = 32768;     // keys per CTA that still fit in shared memory
 constexpr int kCapW = 64;             // per-warp capacity of the definite and candidate lists
 constexpr int kMaskWords = 64;        // per-warp output bitmap: ranges of up to 2048 keys
+constexpr uint32_t kGather = 3072;    // candidate keys of a row gathered into rank 0
 
 // Exclusive prefix sum over the block; returns the sum over lower-numbered threads and
 // writes the block total.
@@ -115,16 +116,18 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   const int crank = static_cast<int>(cluster.block_rank());
   extern __shared__ __align__(128) unsigned char smem_raw[];
   float* fs = reinterpret_cast<float*>(smem_raw);                      // [per_cap] staged scores
-  uint32_t* hloc = reinterpret_cast<uint32_t*>(fs + per_cap);          // [kBins2] this CTA's histogram
-  uint32_t* totA = hloc + kBins2;                                       // [kBins2] digit-2 totals (rank 0)
-  uint32_t* totB = totA + kBins2;                                       // [kBins2] digit-3 totals (rank 0)
-  uint32_t* defs = totB + kBins2;                                       // [warps][kCapW] keys above bin D1
+  uint32_t* h1s = reinterpret_cast<uint32_t*>(fs + per_cap);           // [kBins1] the row's digit-1 histogram
+  uint32_t* gbuf = h1s + kBins1;                                        // [kGather] candidate keys of the row
+  uint32_t* hloc = gbuf + kGather;                                      // [kBins2] local histogram / bitmaps
+  uint32_t* defs = hloc + kBins2;                                       // [warps][kCapW] keys above bin D1
   uint32_t* cands = defs + kTopkWarps * kCapW;                          // [warps][kCapW] keys inside bin D1
-  uint32_t* masks = cands + kTopkWarps * kCapW;                         // [warps][kMaskWords] output bitmaps
+  uint32_t* totA = gbuf;                                                // fallback totals (rank 0) alias gbuf
+  uint32_t* totB = gbuf + kBins2;
+  uint32_t* masks = hloc;                                               // output bitmaps alias hloc
   __shared__ uint64_t bar;
-  __shared__ uint32_t dig, krem_s;
+  __shared__ uint32_t dig, krem_s, gcnt, gbase;
   __shared__ uint32_t cta_gt[kMaxCluster], cta_eq[kMaxCluster];
-  __shared__ uint32_t warp_gt[kTopkWarps], warp_eq[kTopkWarps];
+  __shared__ uint32_t warp_gt[kTopkWarps], warp_eq[kTopkWarps], warp_nc[kTopkWarps];
   __shared__ uint32_t scan_tmp[32];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -152,35 +155,35 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   const int len = max(0, min(n, lo + per) - lo);
   const int wc = ((len + kTopkWarps - 1) / kTopkWarps + 31) & ~31;
   const float* srow = a.scores + static_cast<int64_t>(row) * a.sc_ld + lo;
-  bool staged_ok = true;
-  if (STAGED && tid == 0) {
+  const uint32_t* hrow = a.hist + static_cast<int64_t>(row) * kBins1;
+  if (tid == 0) {
+    gcnt = 0;
     mbar_init(&bar, 1);
     fence_mbarrier_init();
   }
   __syncthreads();
-  if (STAGED) {
-    const bool bulk = (reinterpret_cast<uintptr_t>(srow) & 15u) == 0;
-    const int nbulk = bulk ? (len & ~3) : 0;
-    if (tid == 0 && nbulk > 0) {
-      mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nbulk) * 4u);
-      bulk_g2s(fs, srow, static_cast<uint32_t>(nbulk) * 4u, &bar, l2_policy_evict_first());
-    }
-    for (int i = nbulk + tid; i < len; i += kTopkThreads) fs[i] = __ldg(srow + i);
-    if (nbulk > 0) staged_ok = mbar_wait_bounded(&bar, 0, a.status);
+  const bool bulk = STAGED && (reinterpret_cast<uintptr_t>(srow) & 15u) == 0;
+  const int nbulk = bulk ? (len & ~3) : 0;
+  if (tid == 0) {  // the slice (when staged) and the row's digit-1 histogram, in one transaction
+    const uint64_t pol = l2_policy_evict_first();
+    mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nbulk) * 4u + kBins1 * 4u);
+    if (nbulk > 0) bulk_g2s(fs, srow, static_cast<uint32_t>(nbulk) * 4u, &bar, pol);
+    bulk_g2s(h1s, hrow, kBins1 * 4u, &bar, pol);
   }
+  if (STAGED)
+    for (int i = nbulk + tid; i < len; i += kTopkThreads) fs[i] = __ldg(srow + i);
   auto key_at = [&](int i) -> uint32_t { return float_to_ordered(STAGED ? fs[i] : __ldg(srow + i)); };
-
-  if (crank == 0)
-    for (int i = tid; i < kBins2; i += kTopkThreads) { totA[i] = 0; totB[i] = 0; }
-  // digit 1 from the row's global histogram (every CTA computes the same digit)
-  find_digit<kBins1>(a.hist + static_cast<int64_t>(row) * kBins1, static_cast<uint32_t>(k_eff), scan_tmp, &dig,
-                     &krem_s);
-  const uint32_t d1 = dig;
-  uint32_t krem = krem_s;
+  cluster.sync();  // S0: every CTA runs and rank 0's gather count is zero (overlaps the copies)
+  const bool staged_ok = mbar_wait_bounded(&bar, 0, a.status);
   const bool aborted = __syncthreads_or(!staged_ok);
 
-  // scan 1, the only pass over the whole slice: each warp lists (in index order) its keys
-  // above bin d1 ("definites", all selected) and inside bin d1 ("candidates")
+  // digit 1 from the row's histogram (every CTA computes the same digit)
+  find_digit<kBins1>(h1s, static_cast<uint32_t>(k_eff), scan_tmp, &dig, &krem_s);
+  const uint32_t d1 = dig;
+  const uint32_t k1 = krem_s;
+
+  // scan 1, the only pass over the whole slice: each warp lists, in index order, its
+  // keys above bin d1 ("definites", all selected) and inside bin d1 ("candidates")
   const int w_lo = warp * wc, w_hi = aborted ? w_lo : min(len, w_lo + wc);
   const uint32_t lt_mask = (1u << lane) - 1u;
   uint32_t* my_defs = defs + warp * kCapW;
@@ -205,38 +208,83 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     nca += __popc(mcan);
   }
   const bool cand_list = nca <= kCapW;   // warp-uniform: else this warp rescans its range
-  cluster.sync();  // rank 0's totals are zero and every CTA of the cluster is running
+  if (lane == 0) warp_nc[warp] = cand_list ? nca : (kGather + 1u);
+  __syncthreads();
 
-  uint32_t* totA0 = cluster.map_shared_rank(totA, 0);
-  uint32_t* totB0 = cluster.map_shared_rank(totB, 0);
-  uint32_t prefix = d1 << 20, mask = 0xFFF00000u;
+  // gather the keys of bin d1 from the whole row into rank 0 (distributed shared memory)
+  uint32_t* gcnt0 = cluster.map_shared_rank(&gcnt, 0);
+  uint32_t* gbuf0 = cluster.map_shared_rank(gbuf, 0);
+  if (tid == 0) {
+    uint32_t tot = 0;
+    for (int w = 0; w < kTopkWarps; ++w) tot += warp_nc[w];
+    tot = min(tot, kGather + 1u);
+    gbase = (tot > 0) ? atomicAdd(gcnt0, tot) : 0u;
+  }
+  __syncthreads();
+  {
+    uint32_t off = gbase;
+    for (int w = 0; w < warp; ++w) off += warp_nc[w];
+    if (cand_list && off + nca <= kGather)
+      for (int j = lane; j < static_cast<int>(nca); j += 32) gbuf0[off + j] = key_at(static_cast<int>(my_cands[j]));
+  }
+  cluster.sync();  // S1: the row's candidate keys (or an overflowed count) are in rank 0
+  const uint32_t gtotal = *gcnt0;
+  uint32_t prefix = d1 << 20, mask = 0xFFF00000u, krem = k1;
+  if (gtotal <= kGather) {
+    // exact selection among the gathered keys, locally in every CTA: digits 2 and 3
+    if (crank != 0)
+      for (int j = tid; j < static_cast<int>(gtotal); j += kTopkThreads) gbuf[j] = gbuf0[j];
 #pragma unroll 1
-  for (int pass = 0; pass < 2; ++pass) {
-    const int shift = (pass == 0) ? 10 : 0;
-    uint32_t* tot0 = (pass == 0) ? totA0 : totB0;
-    for (int i = tid; i < kBins2; i += kTopkThreads) hloc[i] = 0;
-    __syncthreads();
-    if (cand_list) {
-      for (int j = lane; j < static_cast<int>(nca); j += 32) {
-        const uint32_t key = key_at(static_cast<int>(my_cands[j]));
+    for (int pass = 0; pass < 2; ++pass) {
+      const int shift = (pass == 0) ? 10 : 0;
+      for (int i = tid; i < kBins2; i += kTopkThreads) hloc[i] = 0;
+      __syncthreads();
+      for (int j = tid; j < static_cast<int>(gtotal); j += kTopkThreads) {
+        const uint32_t key = gbuf[j];
         if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kBins2 - 1)], 1u);
       }
-    } else {
-      for (int i = w_lo + lane; i < w_hi; i += 32) {
-        const uint32_t key = key_at(i);
-        if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kBins2 - 1)], 1u);
-      }
+      __syncthreads();
+      find_digit<kBins2>(hloc, krem, scan_tmp, &dig, &krem_s);
+      prefix |= dig << shift;
+      mask |= static_cast<uint32_t>(kBins2 - 1) << shift;
+      krem = krem_s;
     }
-    __syncthreads();
-    for (int i = tid; i < kBins2; i += kTopkThreads) {
-      const uint32_t v = hloc[i];
-      if (v) atomicAdd(&tot0[i], v);
-    }
+  } else {
+    // too many candidates for the gather buffer: resolve digits 2 and 3 with cluster-wide
+    // histograms in rank 0 (every CTA takes this branch: gtotal is the same everywhere)
+    uint32_t* totA0 = cluster.map_shared_rank(totA, 0);
+    uint32_t* totB0 = cluster.map_shared_rank(totB, 0);
+    if (crank == 0)
+      for (int i = tid; i < kBins2; i += kTopkThreads) { totA[i] = 0; totB[i] = 0; }
     cluster.sync();
-    find_digit<kBins2>(tot0, krem, scan_tmp, &dig, &krem_s);
-    prefix |= dig << shift;
-    mask |= static_cast<uint32_t>(kBins2 - 1) << shift;
-    krem = krem_s;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+      const int shift = (pass == 0) ? 10 : 0;
+      uint32_t* tot0 = (pass == 0) ? totA0 : totB0;
+      for (int i = tid; i < kBins2; i += kTopkThreads) hloc[i] = 0;
+      __syncthreads();
+      if (cand_list) {
+        for (int j = lane; j < static_cast<int>(nca); j += 32) {
+          const uint32_t key = key_at(static_cast<int>(my_cands[j]));
+          if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kBins2 - 1)], 1u);
+        }
+      } else {
+        for (int i = w_lo + lane; i < w_hi; i += 32) {
+          const uint32_t key = key_at(i);
+          if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kBins2 - 1)], 1u);
+        }
+      }
+      __syncthreads();
+      for (int i = tid; i < kBins2; i += kTopkThreads) {
+        const uint32_t v = hloc[i];
+        if (v) atomicAdd(&tot0[i], v);
+      }
+      cluster.sync();
+      find_digit<kBins2>(tot0, krem, scan_tmp, &dig, &krem_s);
+      prefix |= dig << shift;
+      mask |= static_cast<uint32_t>(kBins2 - 1) << shift;
+      krem = krem_s;
+    }
   }
   const uint32_t kstar = prefix;  // the k-th largest key
   const uint32_t need = krem;     // keys equal to kstar to take, lowest index first
@@ -268,7 +316,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     *cluster.map_shared_rank(&cta_gt[crank], tid) = g;
     *cluster.map_shared_rank(&cta_eq[crank], tid) = e;
   }
-  cluster.sync();  // last access to another CTA's shared memory
+  cluster.sync();  // S2: last access to another CTA's shared memory
   if (aborted) {  // the staging copy never completed (flagged): report an empty selection
     for (int j = crank * kTopkThreads + tid; j < k_eff; j += C * kTopkThreads) out[j] = -1;
     return;
@@ -315,7 +363,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     __syncwarp();
     const uint32_t w0 = (lane < words) ? m[lane] : 0u;
     const uint32_t w1 = (lane + 32 < words) ? m[lane + 32] : 0u;
-    uint32_t c0 = __popc(w0), c1 = __popc(w1);
+    const uint32_t c0 = __popc(w0), c1 = __popc(w1);
     uint32_t x0 = c0, x1 = c1;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -325,14 +373,14 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     }
     const uint32_t tot0 = __shfl_sync(0xFFFFFFFFu, x0, 31);
     uint32_t p0 = pos + x0 - c0, p1 = pos + tot0 + x1 - c1;
-    const int gbase = lo + w_lo;
+    const int gb = lo + w_lo;
     for (uint32_t v = w0; v; v &= v - 1) {
-      if (p0 < static_cast<uint32_t>(k_eff)) out[p0] = gbase + lane * 32 + (__ffs(v) - 1);
+      if (p0 < static_cast<uint32_t>(k_eff)) out[p0] = gb + lane * 32 + (__ffs(v) - 1);
       else flag_error(a.status, DEVFLAG_BAD_INDEX);  // unreachable when the counts are consistent
       ++p0;
     }
     for (uint32_t v = w1; v; v &= v - 1) {
-      if (p1 < static_cast<uint32_t>(k_eff)) out[p1] = gbase + (lane + 32) * 32 + (__ffs(v) - 1);
+      if (p1 < static_cast<uint32_t>(k_eff)) out[p1] = gb + (lane + 32) * 32 + (__ffs(v) - 1);
       else flag_error(a.status, DEVFLAG_BAD_INDEX);
       ++p1;
     }
@@ -395,8 +443,9 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   const bool staged = per <= kMaxStaged;
   void (*kern)(TopkArgs, int) = staged ? topk_kernel<true> : topk_kernel<false>;
   const int per_cap = staged ? static_cast<int>(per) : 0;
+  static_assert(kTopkWarps * kMaskWords <= kBins2 && 2 * kBins2 <= kGather, "aliased shared-memory regions");
   const size_t smem = static_cast<size_t>(per_cap) * sizeof(float) +
-                      (3 * kBins2 + 2 * kTopkWarps * kCapW + kTopkWarps * kMaskWords) * sizeof(uint32_t);
+                      (kBins1 + kGather + kBins2 + 2 * kTopkWarps * kCapW) * sizeof(uint32_t);
   static int done_staged[64] = {0}, done_plain[64] = {0};
   cudaError_t e = set_smem_limit_once(kern, smem, staged ? done_staged : done_plain);
   if (e != cudaSuccess) return e;
