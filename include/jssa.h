@@ -35,8 +35,11 @@
  * calls.  All compute calls are asynchronous on `stream` (a cudaStream_t passed as
  * void*; NULL = the legacy default stream) and contain no host synchronisation, so
  * they can be captured into a CUDA graph.  Scratch memory is a caller-provided
- * workspace of at least jssa_workspace_size() bytes, 256-byte aligned; its
- * contents need not be initialised.
+ * workspace of at least jssa_workspace_size() bytes, 256-byte aligned, zeroed once
+ * with jssa_workspace_init() before its first use; every call leaves it ready for the
+ * next (some scratch, such as the selection histograms and the split counters, must
+ * be zero on entry and is cleared by the kernel that consumes it).  After a call
+ * that returned an error, initialise the workspace again.
  *
  * Errors.  Arguments are validated on the host before any launch; an invalid call
  * returns an error status and launches nothing.  A launch failure returns
@@ -190,9 +193,8 @@ JSSA_API jssa_status jssa_dense_decode(const jssa_layout* L, const void* Q, cons
                               float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
- * Zero the device status word at the start of a freshly allocated workspace (the
- * compute calls only ever set bits in it).  Needed once per workspace, before the
- * first jssa_read_device_status(); the compute results do not depend on it.
+ * Zero a freshly allocated workspace (asynchronously on `stream`): required once before
+ * its first use by any compute call, and again after a call that returned an error.
  */
 JSSA_API jssa_status jssa_workspace_init(void* workspace, size_t ws_bytes, void* stream);
 

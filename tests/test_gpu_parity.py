@@ -325,8 +325,14 @@ def test_decode_step_end_to_end(name, kw, seq, window):
     O = torch.full((w.B, w.Hq, w.dv), float("nan"), device="cuda")
     idx = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device="cuda")
     nsel = torch.empty((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+    p.Kp[torch.arange(w.B), :, p.seq_lens.long() - 1] = 0   # the step must project the newest key itself
     jssa.decode_step(p.L, p.Q, p.K, p.V, p.Kp, p.P, p.seq_lens, 1, w.k, window, w.sm_scale, O, None, idx, nsel, ws)
     torch.cuda.synchronize()
+    for b in range(w.B):
+        T = int(p.seq_lens[b])
+        for h in range(w.Hkv):
+            ref, _ = oracle.project_rows(u16(p.K[b, h, T - 1:T]), f32(p.P[h]))
+            np.testing.assert_array_equal(u16(p.Kp[b, h, T - 1:T]), ref)
     rows = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
     _check_step(p, w.k, window, O, idx, nsel, rows, name)
     _assert_status_clean(ws)

@@ -182,8 +182,12 @@ jssa_status run_prologue(const jssa_layout* L, const void* Q, const float* P, co
   return cu(launch_step_prologue(q, s));
 }
 
-jssa_status run_score(const jssa_layout* L, const void* Kp, const int32_t* seq_lens, int window, float* scores,
-                      int64_t sc_ld, const Workspace& w, cudaStream_t s) {
+// Score scan.  fuse_q: the kernel forms the projected group queries itself (GQA);
+// otherwise they come from the prologue kernel (MLA).  project_new: the kernel also
+// projects each sequence's newest key row into Kp.
+jssa_status run_score(const jssa_layout* L, const void* Q, const float* P, const void* K, void* Kp,
+                      const int32_t* seq_lens, int window, float* scores, int64_t sc_ld, bool fuse_q,
+                      bool project_new, const Workspace& w, cudaStream_t s) {
   ScoreArgs a{};
   a.Kp = Kp;
   memcpy(a.ps, L->kp_stride, sizeof a.ps);
@@ -198,6 +202,14 @@ jssa_status run_score(const jssa_layout* L, const void* Kp, const int32_t* seq_l
   a.T_cap = L->T_cap;
   a.window = window;
   a.status = w.status;
+  a.fuse_q = fuse_q ? 1 : 0;
+  a.project_new = project_new ? 1 : 0;
+  a.Q = Q;
+  a.P = P;
+  a.K = K;
+  memcpy(a.ks, L->k_stride, sizeof a.ks);
+  a.Hq = L->Hq;
+  a.d = L->d_k;
   return cu(launch_score(a, num_sms_current(), s));
 }
 
@@ -325,9 +337,14 @@ jssa_status jssa_score(const jssa_layout* L, const void* Q, const float* P, cons
   st = get_ws(L, 1, window, workspace, ws_bytes, &w);
   if (st != JSSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = run_prologue(L, Q, P, nullptr, nullptr, seq_lens, 0, w, s);
+  const bool fuse = L->mode == JSSA_MODE_GQA;
+  if (fuse) {
+    st = cu(cudaMemsetAsync(w.hist, 0, sizeof(uint32_t) * 4096 * L->B * L->Hkv, s));
+  } else {
+    st = run_prologue(L, Q, P, nullptr, nullptr, seq_lens, 0, w, s);
+  }
   if (st != JSSA_OK) return st;
-  return run_score(L, Kp, seq_lens, window, scores, L->T_cap, w, s);
+  return run_score(L, Q, P, nullptr, const_cast<void*>(Kp), seq_lens, window, scores, L->T_cap, fuse, false, w, s);
 }
 
 jssa_status jssa_topk(const jssa_layout* L, const float* scores, const int32_t* seq_lens, int32_t k, int32_t window,
@@ -374,14 +391,21 @@ jssa_status jssa_decode_step(const jssa_layout* L, const void* Q, const void* K,
   st = get_ws(L, k, window, workspace, ws_bytes, &w);
   if (st != JSSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (n_new > kMaxPrologueRows) {  // long appends go through the bulk projection kernel
+  // GQA folds the prologue (projected queries, newest key) into the score scan; MLA's
+  // 128-head query group gets its own prologue kernel.  More than one appended row per
+  // step goes through the bulk projection kernel first.
+  const bool fuse = L->mode == JSSA_MODE_GQA;
+  const bool bulk_new = fuse ? (n_new > 1) : (n_new > kMaxPrologueRows);
+  if (bulk_new) {
     ProjectArgs pa = project_args(L, K, P, Kp, nullptr, seq_lens, n_new, w.status);
     st = cu(launch_project_keys(pa, s));
     if (st != JSSA_OK) return st;
   }
-  st = run_prologue(L, Q, P, K, Kp, seq_lens, n_new > kMaxPrologueRows ? 0 : n_new, w, s);
-  if (st != JSSA_OK) return st;
-  st = run_score(L, Kp, seq_lens, window, w.scores, w.sc_ld, w, s);
+  if (!fuse) {
+    st = run_prologue(L, Q, P, K, Kp, seq_lens, bulk_new ? 0 : n_new, w, s);
+    if (st != JSSA_OK) return st;
+  }
+  st = run_score(L, Q, P, K, Kp, seq_lens, window, w.scores, w.sc_ld, fuse, fuse && n_new == 1, w, s);
   if (st != JSSA_OK) return st;
   int32_t* idx = idx_out ? idx_out : w.idx;
   int32_t* nsel = n_sel_out ? n_sel_out : w.n_sel;
@@ -406,7 +430,7 @@ jssa_status jssa_dense_decode(const jssa_layout* L, const void* Q, const void* K
 
 jssa_status jssa_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
   if (!workspace || !aligned(workspace, kAlign) || ws_bytes < sizeof(int)) return JSSA_ERR_WORKSPACE;
-  return cu(cudaMemsetAsync(workspace, 0, sizeof(int), static_cast<cudaStream_t>(stream)));
+  return cu(cudaMemsetAsync(workspace, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
 }
 
 jssa_status jssa_read_device_status(void* workspace, size_t ws_bytes, int32_t* flags, void* stream) {

@@ -143,6 +143,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
   const int G = a.Hq / a.Hkv;
   const int64_t hq0 = static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * G;
   const int64_t my_lo = static_cast<int64_t>(split) * a.split_len;
+  pdl_trigger();
+  pdl_wait();  // the selection comes from the top-k kernel
   // Issue every independent load of the prologue before using any of them: the sequence
   // length, the selection count, this split's index entries (speculatively, validated
   // below) and the query fragments.
@@ -484,9 +486,7 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
   static int done[64] = {0};
   cudaError_t e = set_smem_limit_once(attn_kernel<D, NTILE, DENSE>, smem, done);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.S, a.B * a.Hkv);
-  attn_kernel<D, NTILE, DENSE><<<grid, kAttnThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(attn_kernel<D, NTILE, DENSE>, dim3(a.S, a.B * a.Hkv), dim3(kAttnThreads), smem, s, 0, a);
 }
 
 template <int D, bool DENSE>

@@ -7,6 +7,7 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -142,6 +143,28 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
+// Round a double to bf16, nearest with ties to even, in a single rounding step.
+// Written from the IEEE binary-format definition: bf16 keeps the fp32 exponent
+// range and 7 stored fraction bits; below 2^-126 its spacing is 2^-133.
+__device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
+  const unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(x));
+  const uint16_t sign = static_cast<uint16_t>((u >> 48) & 0x8000u);
+  const unsigned long long a = u & 0x7FFFFFFFFFFFFFFFull;
+  if (a >= 0x7FF0000000000000ull) return (a > 0x7FF0000000000000ull) ? uint16_t(0x7FC0) : uint16_t(sign | 0x7F80);
+  const int e = static_cast<int>(a >> 52) - 1023;
+  if (e >= -126) {
+    unsigned long long keep = a >> 45;  // exponent and the top 7 fraction bits
+    const unsigned long long rem = a & ((1ull << 45) - 1);
+    const unsigned long long half = 1ull << 44;
+    if (rem > half || (rem == half && (keep & 1ull))) keep += 1;
+    const double r = __longlong_as_double(static_cast<long long>(keep << 45));
+    if (r >= 0x1p128) return uint16_t(sign | 0x7F80);
+    return uint16_t(sign | (__float_as_uint(static_cast<float>(r)) >> 16));
+  }
+  const double q = rint(__longlong_as_double(static_cast<long long>(a)) * 0x1p133);  // whole quanta of 2^-133
+  return uint16_t(sign | static_cast<uint16_t>(q));
+}
+
 // Order-preserving map of an fp32 value to uint32 (larger value -> larger key);
 // -0.0 and +0.0 map to the same key.
 __device__ __forceinline__ uint32_t float_to_ordered(float f) {
@@ -152,6 +175,40 @@ __device__ __forceinline__ uint32_t float_to_ordered(float f) {
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 __host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+// Programmatic dependent launch: a kernel launched with launch_pdl() may start while
+// the previous kernel of the stream finishes; it must pass pdl_wait() before touching
+// any memory that earlier stream work writes.  pdl_trigger() lets the next kernel of
+// the stream begin its own launch early.  Both are no-ops without the launch attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 0) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 
 // Raise a kernel's dynamic shared memory limit once per device (host side).  `done` is a
 // per-kernel table owned by the caller (a function-local static).

@@ -24,28 +24,6 @@
 
 namespace jssa {
 
-// Round a double to bf16, nearest with ties to even, in a single rounding step.
-// Written from the IEEE binary-format definition: bf16 keeps the fp32 exponent
-// range and 7 stored fraction bits; below 2^-126 its spacing is 2^-133.
-__device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
-  const unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(x));
-  const uint16_t sign = static_cast<uint16_t>((u >> 48) & 0x8000u);
-  const unsigned long long a = u & 0x7FFFFFFFFFFFFFFFull;
-  if (a >= 0x7FF0000000000000ull) return (a > 0x7FF0000000000000ull) ? uint16_t(0x7FC0) : uint16_t(sign | 0x7F80);
-  const int e = static_cast<int>(a >> 52) - 1023;
-  if (e >= -126) {
-    unsigned long long keep = a >> 45;  // exponent and the top 7 fraction bits
-    const unsigned long long rem = a & ((1ull << 45) - 1);
-    const unsigned long long half = 1ull << 44;
-    if (rem > half || (rem == half && (keep & 1ull))) keep += 1;
-    const double r = __longlong_as_double(static_cast<long long>(keep << 45));
-    if (r >= 0x1p128) return uint16_t(sign | 0x7F80);
-    return uint16_t(sign | (__float_as_uint(static_cast<float>(r)) >> 16));
-  }
-  const double q = rint(__longlong_as_double(static_cast<long long>(a)) * 0x1p133);  // whole quanta of 2^-133
-  return uint16_t(sign | static_cast<uint16_t>(q));
-}
-
 // Stage P_h [d][r] (fp32) into shared memory with 16-byte loads.
 __device__ __forceinline__ void stage_basis(float* Psm, const float* Ph, int n) {
   const float4* src = reinterpret_cast<const float4*>(Ph);

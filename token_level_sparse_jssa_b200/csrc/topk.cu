@@ -133,6 +133,13 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.y;
   const int b = row / a.Hkv;
+  if (tid == 0) {
+    gcnt = 0;
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+  }
+  pdl_trigger();
+  pdl_wait();  // scores and histograms come from the score scan
   int64_t T = a.seq_lens[b];
   if (T < 0 || T > a.T_cap) {
     if (crank == 0 && tid == 0) flag_error(a.status, DEVFLAG_BAD_SEQ_LEN);
@@ -144,8 +151,11 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   int32_t* out = a.idx + static_cast<int64_t>(row) * a.k;
   if (crank == 0 && tid == 0) a.n_sel[row] = k_eff;
   for (int j = k_eff + crank * kTopkThreads + tid; j < a.k; j += C * kTopkThreads) out[j] = -1;
+  uint32_t* hrow_w = a.hist + static_cast<int64_t>(row) * kBins1;
   if (k_eff == n) {  // everything is selected (includes n == 0)
     for (int j = crank * kTopkThreads + tid; j < n; j += C * kTopkThreads) out[j] = j;
+    if (crank == 0)  // leave the row's histogram zeroed for the next scan
+      for (int i = tid; i < kBins1; i += kTopkThreads) hrow_w[i] = 0u;
     return;
   }
 
@@ -156,11 +166,6 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   const int wc = ((len + kTopkWarps - 1) / kTopkWarps + 31) & ~31;
   const float* srow = a.scores + static_cast<int64_t>(row) * a.sc_ld + lo;
   const uint32_t* hrow = a.hist + static_cast<int64_t>(row) * kBins1;
-  if (tid == 0) {
-    gcnt = 0;
-    mbar_init(&bar, 1);
-    fence_mbarrier_init();
-  }
   __syncthreads();
   const bool bulk = STAGED && (reinterpret_cast<uintptr_t>(srow) & 15u) == 0;
   const int nbulk = bulk ? (len & ~3) : 0;
@@ -229,6 +234,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   }
   cluster.sync();  // S1: the row's candidate keys (or an overflowed count) are in rank 0
   const uint32_t gtotal = *gcnt0;
+  if (crank == 0)  // every CTA has staged the row's histogram: leave it zeroed for the next scan
+    for (int i = tid; i < kBins1; i += kTopkThreads) hrow_w[i] = 0u;
   uint32_t prefix = d1 << 20, mask = 0xFFF00000u, krem = k1;
   if (gtotal <= kGather) {
     // exact selection among the gathered keys, locally in every CTA: digits 2 and 3
@@ -449,21 +456,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   static int done_staged[64] = {0}, done_plain[64] = {0};
   cudaError_t e = set_smem_limit_once(kern, smem, staged ? done_staged : done_plain);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(C, a.B * a.Hkv, 1);
-  cfg.blockDim = dim3(kTopkThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, a, per_cap);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(C, a.B * a.Hkv, 1), dim3(kTopkThreads), smem, s, C, a, per_cap);
 }
 
 }  // namespace jssa
