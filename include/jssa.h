@@ -97,8 +97,8 @@ enum {
  * GQA: Hq = G * Hkv; query head hq belongs to KV head hq / G.  Supported: d_k = d_v in
  * {64, 128, 256}, G in {1, 2, 4, 8, 16}, r in {8, 16, 32, 64} (r <= d_k).
  * MLA: Hkv = 1, d_k = 576, d_v = 512, Hq = 128, r in {16, 32, 64}; V may alias K.
- * K/V/Kp base pointers and strides (except the unit inner stride) must be
- * multiples of 16 bytes.
+ * Q, P, K, V and Kp base pointers and the K/V/Kp strides (except the unit inner
+ * stride) must be multiples of 16 bytes.
  */
 typedef struct {
   int32_t mode;      /* JSSA_MODE_GQA or JSSA_MODE_MLA                    */

@@ -169,7 +169,6 @@ jssa_status run_prologue(const jssa_layout* L, const void* Q, const float* P, co
   q.Kp = Kp;
   memcpy(q.ps, L->kp_stride, sizeof q.ps);
   q.seq_lens = seq_lens;
-  q.hist = w.hist;
   q.counters = w.counters;
   q.n_new = n_new;
   q.B = L->B;
@@ -182,12 +181,8 @@ jssa_status run_prologue(const jssa_layout* L, const void* Q, const float* P, co
   return cu(launch_step_prologue(q, s));
 }
 
-// Score scan.  fuse_q: the kernel forms the projected group queries itself (GQA);
-// otherwise they come from the prologue kernel (MLA).  project_new: the kernel also
-// projects each sequence's newest key row into Kp.
-jssa_status run_score(const jssa_layout* L, const void* Q, const float* P, const void* K, void* Kp,
-                      const int32_t* seq_lens, int window, float* scores, int64_t sc_ld, bool fuse_q,
-                      bool project_new, const Workspace& w, cudaStream_t s) {
+jssa_status run_score(const jssa_layout* L, const void* Kp, const int32_t* seq_lens, int window, float* scores,
+                      int64_t sc_ld, const Workspace& w, cudaStream_t s) {
   ScoreArgs a{};
   a.Kp = Kp;
   memcpy(a.ps, L->kp_stride, sizeof a.ps);
@@ -202,14 +197,6 @@ jssa_status run_score(const jssa_layout* L, const void* Q, const float* P, const
   a.T_cap = L->T_cap;
   a.window = window;
   a.status = w.status;
-  a.fuse_q = fuse_q ? 1 : 0;
-  a.project_new = project_new ? 1 : 0;
-  a.Q = Q;
-  a.P = P;
-  a.K = K;
-  memcpy(a.ks, L->k_stride, sizeof a.ks);
-  a.Hq = L->Hq;
-  a.d = L->d_k;
   return cu(launch_score(a, num_sms_current(), s));
 }
 
@@ -322,7 +309,7 @@ jssa_status jssa_project_keys(const jssa_layout* L, const void* K, const float* 
   if (n_tokens < 0 || n_tokens > L->T_cap) return JSSA_ERR_INVALID_ARG;
   if (n_tokens == 0) return JSSA_OK;
   if (!K || !P || !Kp || (!t_begin && !seq_lens)) return JSSA_ERR_INVALID_ARG;
-  if (!aligned(K, 16) || !aligned(Kp, 16) || !aligned(P, 4)) return JSSA_ERR_INVALID_ARG;
+  if (!aligned(K, 16) || !aligned(Kp, 16) || !aligned(P, 16)) return JSSA_ERR_INVALID_ARG;
   ProjectArgs a = project_args(L, K, P, Kp, t_begin, seq_lens, n_tokens, nullptr);
   return cu(launch_project_keys(a, static_cast<cudaStream_t>(stream)));
 }
@@ -332,19 +319,16 @@ jssa_status jssa_score(const jssa_layout* L, const void* Q, const float* P, cons
   jssa_status st = check_layout(L);
   if (st != JSSA_OK) return st;
   if (!Q || !P || !Kp || !seq_lens || !scores || window < 0) return JSSA_ERR_INVALID_ARG;
-  if (!aligned(Q, 4) || !aligned(P, 4) || !aligned(Kp, 16) || !aligned(scores, 4)) return JSSA_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(P, 16) || !aligned(Kp, 16) || !aligned(scores, 4)) return JSSA_ERR_INVALID_ARG;
   Workspace w{};
   st = get_ws(L, 1, window, workspace, ws_bytes, &w);
   if (st != JSSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool fuse = L->mode == JSSA_MODE_GQA;
-  if (fuse) {
-    st = cu(cudaMemsetAsync(w.hist, 0, sizeof(uint32_t) * 4096 * L->B * L->Hkv, s));
-  } else {
-    st = run_prologue(L, Q, P, nullptr, nullptr, seq_lens, 0, w, s);
-  }
+  st = cu(cudaMemsetAsync(w.hist, 0, sizeof(uint32_t) * 4096 * L->B * L->Hkv, s));
   if (st != JSSA_OK) return st;
-  return run_score(L, Q, P, nullptr, const_cast<void*>(Kp), seq_lens, window, scores, L->T_cap, fuse, false, w, s);
+  st = run_prologue(L, Q, P, nullptr, nullptr, seq_lens, 0, w, s);
+  if (st != JSSA_OK) return st;
+  return run_score(L, Kp, seq_lens, window, scores, L->T_cap, w, s);
 }
 
 jssa_status jssa_topk(const jssa_layout* L, const float* scores, const int32_t* seq_lens, int32_t k, int32_t window,
@@ -384,28 +368,21 @@ jssa_status jssa_decode_step(const jssa_layout* L, const void* Q, const void* K,
   if (!Q || !K || !V || !Kp || !P || !seq_lens || !O || k < 1 || k > kMaxK || window < 0 || n_new < 0 ||
       n_new > L->T_cap)
     return JSSA_ERR_INVALID_ARG;
-  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(Kp, 16) || !aligned(P, 4) || !aligned(O, 4))
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(Kp, 16) || !aligned(P, 16) || !aligned(O, 4))
     return JSSA_ERR_INVALID_ARG;
   if ((idx_out && !aligned(idx_out, 4)) || (n_sel_out && !aligned(n_sel_out, 4))) return JSSA_ERR_INVALID_ARG;
   Workspace w{};
   st = get_ws(L, k, window, workspace, ws_bytes, &w);
   if (st != JSSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // GQA folds the prologue (projected queries, newest key) into the score scan; MLA's
-  // 128-head query group gets its own prologue kernel.  More than one appended row per
-  // step goes through the bulk projection kernel first.
-  const bool fuse = L->mode == JSSA_MODE_GQA;
-  const bool bulk_new = fuse ? (n_new > 1) : (n_new > kMaxPrologueRows);
-  if (bulk_new) {
+  if (n_new > kMaxPrologueRows) {  // long appends go through the bulk projection kernel
     ProjectArgs pa = project_args(L, K, P, Kp, nullptr, seq_lens, n_new, w.status);
     st = cu(launch_project_keys(pa, s));
     if (st != JSSA_OK) return st;
   }
-  if (!fuse) {
-    st = run_prologue(L, Q, P, K, Kp, seq_lens, bulk_new ? 0 : n_new, w, s);
-    if (st != JSSA_OK) return st;
-  }
-  st = run_score(L, Q, P, K, Kp, seq_lens, window, w.scores, w.sc_ld, fuse, fuse && n_new == 1, w, s);
+  st = run_prologue(L, Q, P, K, Kp, seq_lens, n_new > kMaxPrologueRows ? 0 : n_new, w, s);
+  if (st != JSSA_OK) return st;
+  st = run_score(L, Kp, seq_lens, window, w.scores, w.sc_ld, w, s);
   if (st != JSSA_OK) return st;
   int32_t* idx = idx_out ? idx_out : w.idx;
   int32_t* nsel = n_sel_out ? n_sel_out : w.n_sel;

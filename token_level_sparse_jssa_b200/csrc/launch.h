@@ -33,7 +33,6 @@ struct PrologueArgs {
   void* Kp;
   int64_t ps[3];
   const int32_t* seq_lens;
-  uint32_t* hist;   // nullable: [B*Hkv, 4096] zeroed here for the score scan
   int* counters;    // nullable: [B*Hkv] attention arrival counters zeroed here
   int n_new;
   int B, Hq, Hkv, d, r;
@@ -43,9 +42,9 @@ struct PrologueArgs {
 cudaError_t launch_step_prologue(const PrologueArgs& a, cudaStream_t s);
 
 struct ScoreArgs {
-  void* Kp;          // read; row T_b - 1 also written when project_new
+  const void* Kp;
   int64_t ps[3];
-  const float* qs;   // [B*Hkv, r] projected group queries (when !fuse_q)
+  const float* qs;   // [B*Hkv, r] projected group queries (from the step prologue)
   float* scores;     // [B*Hkv, sc_ld]
   int64_t sc_ld;
   uint32_t* hist;    // nullable: [B*Hkv, 4096] histogram of key bits [31:20], zero on entry
@@ -54,15 +53,6 @@ struct ScoreArgs {
   int64_t T_cap;
   int window;
   int* status;
-  // fused per-step prologue (GQA): form qs from Q and P in the kernel, and project the
-  // newest key row T_b - 1 of every (sequence, KV head) into Kp
-  int fuse_q;
-  int project_new;
-  const void* Q;     // [B, Hq, d]
-  const float* P;    // [Hkv, d, r]
-  const void* K;
-  int64_t ks[3];
-  int Hq, d;
 };
 cudaError_t launch_score(const ScoreArgs& a, int num_sms, cudaStream_t s);
 

@@ -18,7 +18,7 @@
 //                          qs = sum_g P_h^T q_g (fp32; the group sum first) and
 //                          projects the newest row(s) into Kp; every output column is
 //                          split over 256/r threads whose partial sums are added in a
-//                          fixed order.
+//                          fixed order.  It also re-arms the attention's split counters.
 #include "common.cuh"
 #include "launch.h"
 
@@ -104,33 +104,73 @@ cudaError_t launch_project_keys(const ProjectArgs& a, cudaStream_t s) {
 // ------------------------------------------------------------------ step prologue
 constexpr int kPrologueThreads = 256;
 constexpr int kMaxNewRowsInPrologue = 16;
+constexpr int kQStageBytes = 16384;  // query groups up to this size are staged with one bulk copy
 
+// One CTA per (sequence, KV head).  P_h, the group's queries and the newest key rows
+// arrive through bulk copies (TMA engine) issued together, so the whole prologue costs
+// about two memory round trips: one for P_h / Q (and the sequence length), one for
+// the key rows, whose position depends on the sequence length.
 __global__ void __launch_bounds__(kPrologueThreads) step_prologue_kernel(PrologueArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  extern __shared__ __align__(128) unsigned char smem_raw[];
   const int d = a.d, r = a.r;
-  float* Psm = reinterpret_cast<float*>(smem_raw);              // [d][r]
-  float* vec = Psm + d * r;                                      // [d]  group-summed query / key row
-  double* red = reinterpret_cast<double*>(vec + d + (d & 1));    // [parts][r] partial sums
   const int row = blockIdx.x;
   const int b = row / a.Hkv, h = row % a.Hkv;
   const int G = a.Hq / a.Hkv;
   const int tid = threadIdx.x;
-  stage_basis(Psm, a.P + static_cast<int64_t>(h) * d * r, d * r);
-  if (a.hist) {  // this row's first-digit histogram, filled by the score scan that follows
-    uint4* g = reinterpret_cast<uint4*>(a.hist + static_cast<int64_t>(row) * 4096);
-    for (int i = tid; i < 4096 / 4; i += blockDim.x) g[i] = make_uint4(0, 0, 0, 0);
-  }
-  if (a.counters && tid == 0) a.counters[row] = 0;
-  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.Q) + (static_cast<int64_t>(b) * a.Hq + h * G) * d;
-  for (int i = tid; i < d; i += blockDim.x) {
-    float s = 0.f;
-#pragma unroll 8
-    for (int g = 0; g < G; ++g) s += __bfloat162float(Q[static_cast<int64_t>(g) * d + i]);
-    vec[i] = s;
+  const bool q_bulk = G * d * 2 <= kQStageBytes;
+  const int n_new = a.n_new > 0 ? a.n_new : 0;
+  float* Psm = reinterpret_cast<float*>(smem_raw);                                  // [d][r]
+  __nv_bfloat16* Qsm = reinterpret_cast<__nv_bfloat16*>(Psm + d * r);              // [G][d] (q_bulk)
+  __nv_bfloat16* Ksm = Qsm + (q_bulk ? G * d : 0);                                  // [n_new][d]
+  float* vec = reinterpret_cast<float*>(Ksm + ((n_new * d + 7) & ~7));              // [d]
+  double* red = reinterpret_cast<double*>(vec + ((d + 1) & ~1));                    // [256]
+  __shared__ uint64_t bars[2];
+  __shared__ int64_t tb_s;
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbarrier_init();
   }
   __syncthreads();
-  // output column j = tid % r; this thread sums i = part, part + parts, ... (conflict-free
-  // shared loads: a warp reads consecutive columns of one row of P)
+  pdl_trigger();
+  pdl_wait();
+  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.Q) + (static_cast<int64_t>(b) * a.Hq + h * G) * d;
+  const __nv_bfloat16* Kb = static_cast<const __nv_bfloat16*>(a.K) + b * a.ks[0] + h * a.ks[1];
+  if (tid == 0) {
+    const uint32_t pbytes = static_cast<uint32_t>(d) * r * 4, qbytes = q_bulk ? static_cast<uint32_t>(G) * d * 2 : 0u;
+    mbar_arrive_expect_tx(&bars[0], pbytes + qbytes);
+    bulk_g2s(Psm, a.P + static_cast<int64_t>(h) * d * r, pbytes, &bars[0], l2_policy_evict_last());
+    if (q_bulk) bulk_g2s(Qsm, Q, qbytes, &bars[0], l2_policy_evict_first());
+    if (n_new > 0) {
+      int64_t T = a.seq_lens[b];
+      if (T < 0 || T > a.T_cap) {
+        flag_error(a.status, DEVFLAG_BAD_SEQ_LEN);
+        T = T < 0 ? 0 : a.T_cap;
+      }
+      const int64_t t0 = max64(0, T - n_new);
+      tb_s = t0;
+      const int rows = static_cast<int>(T - t0);
+      mbar_arrive_expect_tx(&bars[1], static_cast<uint32_t>(rows) * d * 2);
+      for (int q = 0; q < rows; ++q)  // one copy per row: rows may be strided
+        bulk_g2s(Ksm + q * d, Kb + (t0 + q) * a.ks[2], static_cast<uint32_t>(d) * 2, &bars[1], l2_policy_evict_first());
+    }
+  }
+  if (a.counters && tid == 0) a.counters[row] = 0;
+  // group-summed query (fp32, heads in ascending order)
+  bool ok = mbar_wait_bounded(&bars[0], 0, a.status);
+  for (int i = tid; i < d; i += blockDim.x) {
+    float sacc = 0.f;
+    if (q_bulk) {
+      for (int g = 0; g < G; ++g) sacc += __bfloat162float(Qsm[g * d + i]);
+    } else {
+#pragma unroll 8
+      for (int g = 0; g < G; ++g) sacc += __bfloat162float(Q[static_cast<int64_t>(g) * d + i]);
+    }
+    vec[i] = sacc;
+  }
+  __syncthreads();
+  // output column j = tid % r; this thread sums i = part, part + parts, ...; the partial
+  // sums are then added in a fixed order (a warp reads consecutive columns of P: no conflicts)
   const int parts = kPrologueThreads / r, j = tid % r, part = tid / r;
   {
     float acc = 0.f;
@@ -138,45 +178,48 @@ __global__ void __launch_bounds__(kPrologueThreads) step_prologue_kernel(Prologu
     red[part * r + j] = acc;
     __syncthreads();
     if (tid < r) {
-      float s = 0.f;
-      for (int q = 0; q < parts; ++q) s += static_cast<float>(red[q * r + tid]);
-      a.qs[static_cast<int64_t>(row) * r + tid] = s;
+      float t = 0.f;
+      for (int q = 0; q < parts; ++q) t += static_cast<float>(red[q * r + tid]);
+      a.qs[static_cast<int64_t>(row) * r + tid] = t;
     }
   }
-  if (a.n_new <= 0) return;
-  // project the newest n_new rows [T_b - n_new, T_b) of this (sequence, KV head)
-  int64_t T = a.seq_lens[b];
-  if (T < 0 || T > a.T_cap) {
-    if (tid == 0) flag_error(a.status, DEVFLAG_BAD_SEQ_LEN);
-    T = T < 0 ? 0 : a.T_cap;
-  }
-  const __nv_bfloat16* Kb = static_cast<const __nv_bfloat16*>(a.K) + b * a.ks[0] + h * a.ks[1];
+  if (n_new == 0) return;
+  // project the newest rows [T_b - n_new, T_b) into Kp (fp64 accumulation, one rounding)
+  __syncthreads();
+  ok = mbar_wait_bounded(&bars[1], 0, a.status) && ok;
+  const int64_t t0 = tb_s;
   uint16_t* Kpb = reinterpret_cast<uint16_t*>(a.Kp) + b * a.ps[0] + h * a.ps[1];
-  for (int64_t t = max64(0, T - a.n_new); t < T; ++t) {
-    __syncthreads();  // vec and red are free again
-    for (int i = tid; i < d; i += blockDim.x) vec[i] = __bfloat162float(Kb[t * a.ks[2] + i]);
-    __syncthreads();
+  for (int64_t t = t0; t < t0 + n_new; ++t) {
+    int64_t T = a.seq_lens[b];
+    T = T < 0 ? 0 : (T > a.T_cap ? a.T_cap : T);
+    if (t >= T) break;
+    const __nv_bfloat16* krow = Ksm + (t - t0) * d;
     double acc = 0.0;
-    for (int i = part; i < d; i += parts) acc = fma(static_cast<double>(vec[i]), static_cast<double>(Psm[i * r + j]), acc);
+    for (int i = part; i < d; i += parts)
+      acc = fma(static_cast<double>(__bfloat162float(krow[i])), static_cast<double>(Psm[i * r + j]), acc);
     red[part * r + j] = acc;
     __syncthreads();
-    if (tid < r) {
-      double s = 0.0;
-      for (int q = 0; q < parts; ++q) s += red[q * r + tid];
-      Kpb[t * a.ps[2] + tid] = f64_to_bf16_rne(s);
+    if (tid < r && ok) {
+      double t2 = 0.0;
+      for (int q = 0; q < parts; ++q) t2 += red[q * r + tid];
+      Kpb[t * a.ps[2] + tid] = f64_to_bf16_rne(t2);
     }
+    __syncthreads();
   }
 }
 
 cudaError_t launch_step_prologue(const PrologueArgs& a, cudaStream_t s) {
   if (a.n_new > kMaxNewRowsInPrologue) return cudaErrorInvalidValue;
-  const size_t smem = static_cast<size_t>(a.d) * a.r * sizeof(float) + static_cast<size_t>(a.d + 1) * sizeof(float) +
-                      static_cast<size_t>(kPrologueThreads) * sizeof(double);
+  const int G = a.Hq / a.Hkv;
+  const bool q_bulk = G * a.d * 2 <= kQStageBytes;
+  const int n_new = a.n_new > 0 ? a.n_new : 0;
+  const size_t smem = static_cast<size_t>(a.d) * a.r * 4 + (q_bulk ? static_cast<size_t>(G) * a.d * 2 : 0) +
+                      static_cast<size_t>((n_new * a.d + 7) & ~7) * 2 + static_cast<size_t>((a.d + 1) & ~1) * 4 +
+                      kPrologueThreads * sizeof(double);
   static int done[64] = {0};
   cudaError_t e = set_smem_limit_once(step_prologue_kernel, smem, done);
   if (e != cudaSuccess) return e;
-  step_prologue_kernel<<<a.B * a.Hkv, kPrologueThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(step_prologue_kernel, dim3(a.B * a.Hkv), dim3(kPrologueThreads), smem, s, 0, a);
 }
 
 }  // namespace jssa

@@ -21,15 +21,8 @@
 // vectors in a per-thread rotated order, so that every 8-thread phase of a 16-byte
 // shared load touches 8 different bank groups, and holds the matching rotated slice
 // of qs in registers.  Chunk bookkeeping advances incrementally (no divisions).
-//
-// For GQA the per-step prologue is folded in: at each row change the consumers form
-// the row's projected group query qs = sum_g P_h^T q_g themselves (fp32, group sum
-// first, each column split over 256/r threads and reduced in a fixed order) while the
-// producer keeps streaming, and the CTA that consumes a row's last chunk projects the
-// newest key row T_b - 1 into Kp (fp64 accumulation, one bf16 rounding), patches its
-// staged copy of that row before scoring it, and writes it back for later steps.
-// (With a window the newest row is not a candidate; the CTA numbered row % gridDim
-// projects it at start.)
+// The projected group queries of the rows a CTA covers (formed by the step prologue)
+// are loaded into shared memory in one batch at start, while the first chunks stream in.
 #include "common.cuh"
 #include "launch.h"
 
@@ -41,6 +34,7 @@ constexpr int kScoreStages = 3;
 constexpr int kChunkBytes = 16384;
 constexpr int kMaxBatch = 1024;
 constexpr int kHistBins = 4096;  // first radix digit of the selection: key bits [31:20]
+constexpr int kQRows = 8;        // projected queries preloaded per CTA
 
 // Position in the flattened chunk space: sequence b, KV head h, chunk ci of the row.
 struct ChunkIter {
@@ -62,63 +56,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Consumer-side (256 threads): qs_s[0..R) = sum_i P_h[i][j] * (sum_g q_g[i]) for `row`.
-template <int R>
-__device__ __forceinline__ void consumers_qs(const ScoreArgs& a, int row, float* vec, double* red, float* qs_s) {
-  const int tid = threadIdx.x;
-  const int b = row / a.Hkv, h = row % a.Hkv, G = a.Hq / a.Hkv, d = a.d;
-  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.Q) + (static_cast<int64_t>(b) * a.Hq + h * G) * d;
-  for (int i = tid; i < d; i += kScoreConsumers) {
-    float s = 0.f;
-#pragma unroll 4
-    for (int g = 0; g < G; ++g) s += __bfloat162float(Q[static_cast<int64_t>(g) * d + i]);
-    vec[i] = s;
-  }
-  consumers_sync();
-  constexpr int PARTS = kScoreConsumers / R;
-  const int j = tid % R, part = tid / R;
-  const float* Ph = a.P + static_cast<int64_t>(h) * d * R;
-  float acc = 0.f;
-#pragma unroll 8
-  for (int i = part; i < d; i += PARTS) acc = fmaf(__ldg(Ph + i * R + j), vec[i], acc);
-  red[part * R + j] = acc;
-  consumers_sync();
-  if (tid < R) {
-    float t = 0.f;
-    for (int q = 0; q < PARTS; ++q) t += static_cast<float>(red[q * R + tid]);
-    qs_s[tid] = t;
-  }
-  consumers_sync();
-}
-
-// Consumer-side (256 threads): project key row t of (b, h) into Kp in fp64 and round once;
-// the R bf16 values are written to Kp and returned in patch[0..R).
-template <int R>
-__device__ __forceinline__ void consumers_project(const ScoreArgs& a, int b, int h, int64_t t, float* vec,
-                                                  double* red, uint16_t* patch) {
-  const int tid = threadIdx.x, d = a.d;
-  const __nv_bfloat16* krow = static_cast<const __nv_bfloat16*>(a.K) + b * a.ks[0] + h * a.ks[1] + t * a.ks[2];
-  for (int i = tid; i < d; i += kScoreConsumers) vec[i] = __bfloat162float(krow[i]);
-  consumers_sync();
-  constexpr int PARTS = kScoreConsumers / R;
-  const int j = tid % R, part = tid / R;
-  const float* Ph = a.P + static_cast<int64_t>(h) * d * R;
-  double acc = 0.0;
-#pragma unroll 8
-  for (int i = part; i < d; i += PARTS)
-    acc = fma(static_cast<double>(vec[i]), static_cast<double>(__ldg(Ph + i * R + j)), acc);
-  red[part * R + j] = acc;
-  consumers_sync();
-  if (tid < R) {
-    double t2 = 0.0;
-    for (int q = 0; q < PARTS; ++q) t2 += red[q * R + tid];
-    const uint16_t v = f64_to_bf16_rne(t2);
-    patch[tid] = v;
-    reinterpret_cast<uint16_t*>(a.Kp)[b * a.ps[0] + h * a.ps[1] + t * a.ps[2] + tid] = v;
-  }
-  consumers_sync();
-}
-
 template <int R>
 __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
   constexpr int CH = kChunkBytes / (R * 2);           // tokens per chunk
@@ -133,13 +70,10 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
   uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + kScoreStages * kChunkBytes);
   uint64_t* empty = full + kScoreStages;
   uint32_t* hist = reinterpret_cast<uint32_t*>(empty + kScoreStages);               // [kHistBins]
-  double* red = reinterpret_cast<double*>(hist + kHistBins);                        // [256] partial sums
-  float* vec = reinterpret_cast<float*>(red + kScoreConsumers);                     // [d] query / key row
-  int64_t* cum = reinterpret_cast<int64_t*>(vec + ((a.d + 1) & ~1));              // [B + 1] chunk prefix
+  float* qtab = reinterpret_cast<float*>(hist + kHistBins);                         // [kQRows][R] projected queries
+  int64_t* cum = reinterpret_cast<int64_t*>(qtab + kQRows * R);                     // [B + 1] chunk prefix
   int64_t* per_head = cum + (a.B + 1);                                              // [B] chunks per row
   int64_t* nb = per_head + a.B;                                                     // [B] candidates
-  __shared__ float qs_s[64];
-  __shared__ uint16_t patch[64];
   __shared__ int aborted;
 
   const int tid = threadIdx.x;
@@ -176,17 +110,6 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
   const int64_t c_begin = total * blockIdx.x / gridDim.x;
   const int64_t c_end = total * (blockIdx.x + 1) / gridDim.x;
   const int64_t n_mine = c_end - c_begin;
-  if (a.project_new && !producer) {
-    // newest rows that are not candidates (a window, or an empty candidate range): the
-    // CTA numbered row % gridDim projects them; the others are patched in the scan
-    if (a.window > 0) {
-      for (int row = blockIdx.x; row < a.B * a.Hkv; row += gridDim.x) {
-        const int b = row / a.Hkv;
-        const int64_t T = min64(max64(a.seq_lens[b], 0), a.T_cap);
-        if (T >= 1) consumers_project<R>(a, b, row % a.Hkv, T - 1, vec, red, patch);
-      }
-    }
-  }
   if (n_mine <= 0) return;
 
   // iterator at c_begin (the only divisions of the kernel)
@@ -221,6 +144,13 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
       }
     }
   } else {
+    // projected queries of the first kQRows rows this CTA covers, in one batch
+    const int row0 = it0.b * a.Hkv + it0.h;
+    for (int i = tid; i < kQRows * R; i += kScoreConsumers) {
+      const int64_t rr = row0 + i / R;
+      if (rr < static_cast<int64_t>(a.B) * a.Hkv) qtab[i] = __ldg(a.qs + rr * R + i % R);
+    }
+    consumers_sync();
     // this thread's token within a pass, its slice of the token and its rotation
     const int sub = (TPT == 2) ? (tid & 1) : 0;
     const int tok_in_pass = tid / TPT;
@@ -245,11 +175,7 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
           consumers_sync();
         }
         cur_row = row;
-        const float* qsrc = a.qs + static_cast<int64_t>(row) * R;
-        if (a.fuse_q) {
-          consumers_qs<R>(a, row, vec, red, qs_s);
-          qsrc = qs_s;
-        }
+        const float* qsrc = (row - row0 < kQRows) ? qtab + (row - row0) * R : a.qs + static_cast<int64_t>(row) * R;
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
           const float4* qp = reinterpret_cast<const float4*>(qsrc + (sub * VPT + (j + rot) % VPT) * 8);
@@ -258,23 +184,13 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
           q[j][4] = q1.x; q[j][5] = q1.y; q[j][6] = q1.z; q[j][7] = q1.w;
         }
       }
-      // the row's last chunk holds its newest key (no window): project it now, before
-      // the staged (stale) copy of that row is scored
-      const bool newest_here = a.project_new && a.window <= 0 && c.ci == per_head[c.b] - 1;
-      if (newest_here) consumers_project<R>(a, c.b, c.h, nb[c.b] - 1, vec, red, patch);
       if (!dead && !mbar_wait_bounded(&full[s], static_cast<uint32_t>((it / kScoreStages) & 1), a.status)) {
         dead = true;
         atomicExch(&aborted, 1);
       }
       const int64_t t0 = c.ci * CH;
       const int cnt = static_cast<int>(min64(CH, nb[c.b] - t0));
-      unsigned char* buf = ring + s * kChunkBytes;
-      if (newest_here) {  // overwrite the staged row with the fresh projection (all consumers meet)
-        if (!dead && tid < R / 2)
-          reinterpret_cast<uint32_t*>(buf + (cnt - 1) * (R * 2))[tid] =
-              static_cast<uint32_t>(patch[2 * tid]) | (static_cast<uint32_t>(patch[2 * tid + 1]) << 16);
-        consumers_sync();
-      }
+      const unsigned char* buf = ring + s * kChunkBytes;
       if (!dead) {
         float* out = a.scores + static_cast<int64_t>(row) * a.sc_ld + t0;
 #pragma unroll
@@ -330,8 +246,7 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
 template <int R>
 static cudaError_t launch_score_r(const ScoreArgs& a, int num_sms, cudaStream_t s) {
   const size_t smem = kScoreStages * kChunkBytes + 2 * kScoreStages * sizeof(uint64_t) +
-                      kHistBins * sizeof(uint32_t) + kScoreConsumers * sizeof(double) +
-                      ((a.d + 1) & ~1) * sizeof(float) + (3 * a.B + 1) * sizeof(int64_t);
+                      kHistBins * sizeof(uint32_t) + kQRows * R * sizeof(float) + (3 * a.B + 1) * sizeof(int64_t);
   static int done[64] = {0};
   cudaError_t e = set_smem_limit_once(score_kernel<R>, smem, done);
   if (e != cudaSuccess) return e;
