@@ -17,13 +17,19 @@
 //   online softmax per head in fp32 (exp2 domain)
 //   O^T[d x 8 heads]     += V_sub^T . P^T               (P split into bf16 hi + lo parts,
 //                                                        so the weights keep ~16 bits)
-// The 4 warps' states are merged in shared memory and the CTA writes one normalised
-// partial (o, lse) per query head; the last CTA of each (sequence, KV head) row to
-// finish (a per-row arrival counter) combines the row's partials by log-sum-exp.
+// The 4 warps' states are merged in shared memory into one normalised partial (o, lse)
+// per query head.  Indexed attention runs the S <= 8 splits of a row as one thread-block
+// cluster and combines the partials by log-sum-exp through distributed shared memory;
+// the dense decode, with many more splits, writes partials to the workspace and the last
+// CTA of each row to finish (a per-row arrival counter) combines them.
+#include <cooperative_groups.h>
+
 #include <cmath>
 
 #include "common.cuh"
 #include "launch.h"
+
+namespace cg = cooperative_groups;
 
 namespace jssa {
 
@@ -42,7 +48,9 @@ struct AttnCfg {
   static constexpr int STAGE_BYTES = 2 * SUB_BYTES;
   static constexpr int RING_BYTES = kAttnWarps * STAGES * STAGE_BYTES;
   static constexpr int COMBINE_BYTES = kAttnWarps * 16 * D * 4 + 2 * kAttnWarps * 16 * 4;
-  static constexpr int MAIN_BYTES = RING_BYTES > COMBINE_BYTES ? RING_BYTES : COMBINE_BYTES;
+  static constexpr int PART_BYTES = 16 * D * 4 + 16 * 4;   // this CTA's partial (o, lse) for the cluster merge
+  static constexpr int MAIN_BYTES =
+      RING_BYTES > COMBINE_BYTES + PART_BYTES ? RING_BYTES : COMBINE_BYTES + PART_BYTES;
 };
 
 template <int D, bool DENSE>
@@ -127,6 +135,52 @@ __device__ __forceinline__ void finish_split(const AttnArgs& a, int row, int64_t
   if (threadIdx.x == 0) a.counters[row] = 0;
 }
 
+// Split merge inside a thread-block cluster (one CTA per split of the row, S <= 8):
+// every CTA keeps its normalised partial (o, lse) in its own shared memory; after a
+// cluster barrier CTA c combines output slice c of the row, reading the S partials
+// through distributed shared memory, and a second barrier keeps the partials alive
+// until every CTA has read them.
+template <int D>
+__device__ __forceinline__ void cluster_merge(const AttnArgs& a, int64_t hq0, int G, const float* pbuf,
+                                              const float* plse) {
+  __shared__ float wts[16 * 8];
+  cg::cluster_group cl = cg::this_cluster();
+  const int S = static_cast<int>(cl.num_blocks());
+  const int c = static_cast<int>(cl.block_rank());
+  cl.sync();
+  for (int i = threadIdx.x; i < G * S; i += blockDim.x) wts[i] = cl.map_shared_rank(plse, i % S)[i / S];
+  __syncthreads();
+  if (threadIdx.x < G) {
+    float* w = wts + threadIdx.x * S;
+    float M = -INFINITY;
+    for (int q = 0; q < S; ++q) M = fmaxf(M, w[q]);
+    float L = 0.f;
+    for (int q = 0; q < S; ++q) {
+      w[q] = (M == -INFINITY) ? 0.f : expf(w[q] - M);
+      L += w[q];
+    }
+    for (int q = 0; q < S; ++q) w[q] = (L > 0.f) ? w[q] / L : 0.f;
+    if (a.lse && c == 0) a.lse[hq0 + threadIdx.x] = (M == -INFINITY) ? -INFINITY : M + logf(L);
+  }
+  __syncthreads();
+  const int per = (G * D + S - 1) / S;
+  const int lo = c * per, hi = min(G * D, lo + per);
+  for (int i = lo + threadIdx.x; i < hi; i += blockDim.x) {
+    const int head = i / D;
+    float v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v[q] = (q < S) ? cl.map_shared_rank(pbuf, q)[i] : 0.f;
+    float o = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < S) o = fmaf(wts[head * S + q], v[q], o);
+    const int64_t qi = hq0 + head;
+    if (a.out_bf16) static_cast<__nv_bfloat16*>(a.O)[qi * D + (i % D)] = __float2bfloat16_rn(o);
+    else static_cast<float*>(a.O)[qi * D + (i % D)] = o;
+  }
+  cl.sync();
+}
+
 template <int D, int NTILE, bool DENSE>
 __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
   using Cfg = AttnCfg<D>;
@@ -143,8 +197,6 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
   const int G = a.Hq / a.Hkv;
   const int64_t hq0 = static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * G;
   const int64_t my_lo = static_cast<int64_t>(split) * a.split_len;
-  pdl_trigger();
-  pdl_wait();  // the selection comes from the top-k kernel
   // Issue every independent load of the prologue before using any of them: the sequence
   // length, the selection count, this split's index entries (speculatively, validated
   // below) and the query fragments.
@@ -198,7 +250,15 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
   }
   const int my_len = static_cast<int>(max64(0, min64(list_len, my_lo + a.split_len) - my_lo));
 
+  float* pbuf = reinterpret_cast<float*>(smem_raw + Cfg::COMBINE_BYTES);   // [16][D] (cluster merge)
+  float* plse = pbuf + 16 * D;                                              // [16]
   if (my_len == 0) {  // empty split: weight zero in the merge
+    if (!DENSE) {
+      for (int i = threadIdx.x; i < G * D; i += kAttnThreads) pbuf[i] = 0.f;
+      if (threadIdx.x < G) plse[threadIdx.x] = -INFINITY;
+      cluster_merge<D>(a, hq0, G, pbuf, plse);
+      return;
+    }
     for (int i = threadIdx.x; i < G * D; i += kAttnThreads) {
       const int head = i / D, dim = i % D;
       a.part_o[((hq0 + head) * a.S + split) * D + dim] = 0.f;
@@ -410,8 +470,18 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
       o /= L;
       lse = (M + log2f(L)) * kLn2;
     }
-    a.part_o[((hq0 + head) * a.S + split) * D + dim] = o;
-    if (dim == 0) a.part_lse[(hq0 + head) * a.S + split] = lse;
+    if (!DENSE) {
+      pbuf[i] = o;
+      if (dim == 0) plse[head] = lse;
+    } else {
+      a.part_o[((hq0 + head) * a.S + split) * D + dim] = o;
+      if (dim == 0) a.part_lse[(hq0 + head) * a.S + split] = lse;
+    }
+  }
+  if (!DENSE) {
+    __syncthreads();
+    cluster_merge<D>(a, hq0, G, pbuf, plse);
+    return;
   }
   finish_split<D>(a, row, hq0, G, reinterpret_cast<float*>(smem_raw));
 }
@@ -467,13 +537,15 @@ void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int n
     const int64_t Sr = ceil_div(list_max, len);
     if (Sr != S) continue;
     if (indexed && mode != 1 && len > kMaxTokList) continue;  // the token list lives in shared memory
+    if (indexed && mode != 1 && S > 8) break;                 // one cluster per row
     const int64_t ctas = static_cast<int64_t>(rows) * Sr;
     const int64_t waves = ceil_div(ctas, slots);
     const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
     if (eff > best_eff + 0.02) { best_eff = eff; best_S = S; best_len = len; }
   }
-  if (best_S == 0) {  // only reachable for lists longer than 256 splits of the maximum length
-    best_len = ceil_div(ceil_div(list_max, 256), 16) * 16;
+  if (best_S == 0) {  // only reachable for very long lists
+    const int cap = (indexed && mode != 1) ? 8 : 256;
+    best_len = ceil_div(ceil_div(list_max, cap), 16) * 16;
     best_S = static_cast<int>(ceil_div(list_max, best_len));
   }
   *S_out = best_S;
@@ -486,7 +558,9 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
   static int done[64] = {0};
   cudaError_t e = set_smem_limit_once(attn_kernel<D, NTILE, DENSE>, smem, done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attn_kernel<D, NTILE, DENSE>, dim3(a.S, a.B * a.Hkv), dim3(kAttnThreads), smem, s, 0, a);
+  // indexed: the S (<= 8) splits of a row form one cluster and merge through shared memory
+  return launch_ex(attn_kernel<D, NTILE, DENSE>, dim3(a.S, a.B * a.Hkv), dim3(kAttnThreads), smem, s,
+                   DENSE ? 0 : a.S, a);
 }
 
 template <int D, bool DENSE>
@@ -497,7 +571,7 @@ static cudaError_t launch_attn_d(const AttnArgs& a, cudaStream_t s) {
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s) {
   const bool dense = (a.idx == nullptr);
-  if (!dense && a.split_len > kMaxTokList) return cudaErrorInvalidValue;
+  if (!dense && (a.split_len > kMaxTokList || a.S > 8)) return cudaErrorNotSupported;
   switch (a.dk) {
     case 64: return dense ? launch_attn_d<64, true>(a, s) : launch_attn_d<64, false>(a, s);
     case 128: return dense ? launch_attn_d<128, true>(a, s) : launch_attn_d<128, false>(a, s);

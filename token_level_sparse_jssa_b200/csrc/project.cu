@@ -35,7 +35,7 @@ constexpr int kProjRows = 32;     // rows of K per CTA
 constexpr int kProjThreads = 256;
 
 __global__ void __launch_bounds__(kProjThreads) project_keys_kernel(ProjectArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  extern __shared__ __align__(128) unsigned char smem_raw[];
   const int d = a.d, r = a.r;
   float* Psm = reinterpret_cast<float*>(smem_raw);                                 // [d][r]
   __nv_bfloat16* krows = reinterpret_cast<__nv_bfloat16*>(Psm + d * r);          // [kProjRows][d]
@@ -132,8 +132,6 @@ __global__ void __launch_bounds__(kPrologueThreads) step_prologue_kernel(Prologu
     fence_mbarrier_init();
   }
   __syncthreads();
-  pdl_trigger();
-  pdl_wait();
   const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.Q) + (static_cast<int64_t>(b) * a.Hq + h * G) * d;
   const __nv_bfloat16* Kb = static_cast<const __nv_bfloat16*>(a.K) + b * a.ks[0] + h * a.ks[1];
   if (tid == 0) {
@@ -219,7 +217,7 @@ cudaError_t launch_step_prologue(const PrologueArgs& a, cudaStream_t s) {
   static int done[64] = {0};
   cudaError_t e = set_smem_limit_once(step_prologue_kernel, smem, done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(step_prologue_kernel, dim3(a.B * a.Hkv), dim3(kPrologueThreads), smem, s, 0, a);
+  return launch_ex(step_prologue_kernel, dim3(a.B * a.Hkv), dim3(kPrologueThreads), smem, s, 0, a);
 }
 
 }  // namespace jssa

@@ -79,8 +79,6 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
   const int tid = threadIdx.x;
   const bool producer = tid >= kScoreConsumers;
   for (int i = tid; i < kHistBins; i += blockDim.x) hist[i] = 0;
-  pdl_trigger();
-  pdl_wait();  // inputs below may come from the previous kernel of the stream
   for (int b = tid; b < a.B; b += blockDim.x) {
     int64_t T = a.seq_lens[b];
     if (T < 0 || T > a.T_cap) {
@@ -251,7 +249,7 @@ static cudaError_t launch_score_r(const ScoreArgs& a, int num_sms, cudaStream_t 
   cudaError_t e = set_smem_limit_once(score_kernel<R>, smem, done);
   if (e != cudaSuccess) return e;
   const int grid = num_sms * 3;
-  return launch_pdl(score_kernel<R>, dim3(grid), dim3(kScoreThreads), smem, s, 0, a);
+  return launch_ex(score_kernel<R>, dim3(grid), dim3(kScoreThreads), smem, s, 0, a);
 }
 
 cudaError_t launch_score(const ScoreArgs& a, int num_sms, cudaStream_t s) {

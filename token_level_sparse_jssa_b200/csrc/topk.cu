@@ -138,8 +138,6 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     mbar_init(&bar, 1);
     fence_mbarrier_init();
   }
-  pdl_trigger();
-  pdl_wait();  // scores and histograms come from the score scan
   int64_t T = a.seq_lens[b];
   if (T < 0 || T > a.T_cap) {
     if (crank == 0 && tid == 0) flag_error(a.status, DEVFLAG_BAD_SEQ_LEN);
@@ -194,23 +192,34 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   uint32_t* my_defs = defs + warp * kCapW;
   uint32_t* my_cands = cands + warp * kCapW;
   uint32_t nd = 0, nca = 0;
-  for (int base = w_lo; base < w_hi; base += 32) {
-    const int i = base + lane;
-    const bool valid = i < w_hi;
-    const uint32_t dk = valid ? (key_at(i) >> 20) : 0u;
-    const bool isdef = valid && dk > d1, iscand = valid && dk == d1;
-    const uint32_t mdef = __ballot_sync(0xFFFFFFFFu, isdef);
-    const uint32_t mcan = __ballot_sync(0xFFFFFFFFu, iscand);
-    if (isdef) {
-      const uint32_t p = nd + __popc(mdef & lt_mask);
-      if (p < kCapW) my_defs[p] = static_cast<uint32_t>(i);
+  constexpr int U = 4;  // 32-key groups per step: independent loads and ballots, in index order
+  for (int base = w_lo; base < w_hi; base += 32 * U) {
+    uint32_t dk[U], mdef[U], mcan[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * 32 + lane;
+      dk[u] = (i < w_hi) ? (key_at(i) >> 20) : 0u;
     }
-    if (iscand) {
-      const uint32_t p = nca + __popc(mcan & lt_mask);
-      if (p < kCapW) my_cands[p] = static_cast<uint32_t>(i);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const bool valid = base + u * 32 + lane < w_hi;
+      mdef[u] = __ballot_sync(0xFFFFFFFFu, valid && dk[u] > d1);
+      mcan[u] = __ballot_sync(0xFFFFFFFFu, valid && dk[u] == d1);
     }
-    nd += __popc(mdef);
-    nca += __popc(mcan);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t i = static_cast<uint32_t>(base + u * 32 + lane);
+      if ((mdef[u] >> lane) & 1u) {
+        const uint32_t p = nd + __popc(mdef[u] & lt_mask);
+        if (p < kCapW) my_defs[p] = i;
+      }
+      if ((mcan[u] >> lane) & 1u) {
+        const uint32_t p = nca + __popc(mcan[u] & lt_mask);
+        if (p < kCapW) my_cands[p] = i;
+      }
+      nd += __popc(mdef[u]);
+      nca += __popc(mcan[u]);
+    }
   }
   const bool cand_list = nca <= kCapW;   // warp-uniform: else this warp rescans its range
   if (lane == 0) warp_nc[warp] = cand_list ? nca : (kGather + 1u);
@@ -456,7 +465,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   static int done_staged[64] = {0}, done_plain[64] = {0};
   cudaError_t e = set_smem_limit_once(kern, smem, staged ? done_staged : done_plain);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(C, a.B * a.Hkv, 1), dim3(kTopkThreads), smem, s, C, a, per_cap);
+  return launch_ex(kern, dim3(C, a.B * a.Hkv, 1), dim3(kTopkThreads), smem, s, C, a, per_cap);
 }
 
 }  // namespace jssa
