@@ -71,7 +71,8 @@ typedef enum {
   JSSA_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small       */
   JSSA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed             */
   JSSA_ERR_DEVICE_CHECK = 5, /* the kernels flagged out-of-range device data     */
-  JSSA_ERR_TIMEOUT = 6       /* a bounded wait inside a kernel gave up           */
+  JSSA_ERR_TIMEOUT = 6,      /* a bounded wait inside a kernel gave up           */
+  JSSA_ERR_SCRATCH_LIMIT = 7 /* beyond the built-in scratch of jssa_topk_noalloc */
 } jssa_status;
 
 enum { JSSA_MODE_GQA = 0, JSSA_MODE_MLA = 1 };
@@ -157,6 +158,25 @@ JSSA_API jssa_status jssa_score(const jssa_layout* L, const void* Q, const float
 JSSA_API jssa_status jssa_topk(const jssa_layout* L, const float* scores, const int32_t* seq_lens,
                       int32_t k, int32_t window, int32_t* idx, int32_t* n_sel,
                       void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Allocation-free top-k: the same selection as jssa_topk, with no workspace argument.
+ * The paper has no counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory for a workspace: code running inside a host framework that owns
+ * all device memory and hands plug-ins no allocator, or code that must not allocate
+ * while a stream is being captured.  Its scratch (the per-row first-digit histograms) is
+ * a 4 MB array inside the library, present on every GPU that loads the library until the
+ * process exits; it holds at most 256 (sequence, KV head) rows: larger batches return
+ * JSSA_ERR_SCRATCH_LIMIT and launch nothing.  The call allocates nothing: it clears the
+ * part of the scratch it uses (the previous call's contents remain otherwise) and runs
+ * the selection kernels.  The first call on a device looks up the scratch's device
+ * address (once per device); make that first call before any stream capture.  All
+ * calls share one scratch, so calls that may overlap on the GPU (other streams, other
+ * host threads) race and must be serialised by the caller.  No device status word is
+ * kept.
+ */
+JSSA_API jssa_status jssa_topk_noalloc(const jssa_layout* L, const float* scores, const int32_t* seq_lens,
+                                       int32_t k, int32_t window, int32_t* idx, int32_t* n_sel, void* stream);
 
 /*
  * Gather-free indexed attention (§3.3) with split-T partials and a log-sum-exp merge.

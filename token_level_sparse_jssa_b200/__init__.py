@@ -11,4 +11,4 @@ fails loudly if it has not been built.
 from ._binding import (  # noqa: F401
     EXPORTS, LIB_PATH, MODE_GQA, MODE_MLA, OUT_BF16, OUT_F32, JssaError, Layout, alloc_workspace, decode_step,
     dense_decode, indexed_attn, load, make_layout, project_keys, read_device_status, score, status_string, topk,
-    version, workspace_init, workspace_size)
+    topk_noalloc, version, workspace_init, workspace_size)

@@ -19,12 +19,13 @@ MODE_GQA, MODE_MLA = 0, 1
 OUT_F32, OUT_BF16 = 0, 1
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape or mode", 3: "workspace missing, misaligned or too small",
-          4: "CUDA error", 5: "device-side check failed", 6: "bounded wait timed out"}
+          4: "CUDA error", 5: "device-side check failed", 6: "bounded wait timed out",
+          7: "beyond the built-in scratch of the allocation-free entry point"}
 DEV_BAD_SEQ_LEN, DEV_BAD_INDEX, DEV_BAD_NSEL, DEV_TIMEOUT = 1, 2, 4, 8
 
 EXPORTS = ("jssa_status_string", "jssa_version", "jssa_workspace_size", "jssa_project_keys", "jssa_score",
-           "jssa_topk", "jssa_indexed_attn", "jssa_decode_step", "jssa_dense_decode", "jssa_workspace_init",
-           "jssa_read_device_status")
+           "jssa_topk", "jssa_topk_noalloc", "jssa_indexed_attn", "jssa_decode_step", "jssa_dense_decode",
+           "jssa_workspace_init", "jssa_read_device_status")
 
 
 class JssaError(RuntimeError):
@@ -61,6 +62,7 @@ def load(path: str = LIB_PATH):
         "jssa_project_keys": (C.c_int, [LP, vp, vp, vp, vp, vp, i64, vp]),
         "jssa_score": (C.c_int, [LP, vp, vp, vp, vp, i32, vp, vp, sz, vp]),
         "jssa_topk": (C.c_int, [LP, vp, vp, i32, i32, vp, vp, vp, sz, vp]),
+        "jssa_topk_noalloc": (C.c_int, [LP, vp, vp, i32, i32, vp, vp, vp]),
         "jssa_indexed_attn": (C.c_int, [LP, vp, vp, vp, vp, i32, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
         "jssa_decode_step": (C.c_int, [LP, vp, vp, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, vp, vp, sz, vp]),
         "jssa_dense_decode": (C.c_int, [LP, vp, vp, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
@@ -163,6 +165,13 @@ def topk(L, scores, seq_lens, k: int, window: int, idx, n_sel, ws=None, stream=N
     w, n = _ws(ws)
     _check("jssa_topk", load().jssa_topk(C.byref(L), _c(scores), _c(seq_lens), k, window, _c(idx), _c(n_sel),
                                          w, n, _stream(stream)))
+
+
+def topk_noalloc(L, scores, seq_lens, k: int, window: int, idx, n_sel, stream=None):
+    """Top-k without a workspace: the library's built-in scratch (up to 256 rows) is used;
+    for callers that cannot allocate device memory.  Overlapping calls race."""
+    _check("jssa_topk_noalloc", load().jssa_topk_noalloc(C.byref(L), _c(scores), _c(seq_lens), k, window, _c(idx),
+                                                         _c(n_sel), _stream(stream)))
 
 
 def indexed_attn(L, Q, K, V, idx, k: int, n_sel, seq_lens, window: int, sm_scale: float, O, lse, ws, stream=None):

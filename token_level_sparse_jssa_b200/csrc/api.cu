@@ -285,6 +285,7 @@ const char* jssa_status_string(jssa_status s) {
     case JSSA_ERR_CUDA: return "CUDA error";
     case JSSA_ERR_DEVICE_CHECK: return "device-side check failed";
     case JSSA_ERR_TIMEOUT: return "bounded wait timed out";
+    case JSSA_ERR_SCRATCH_LIMIT: return "request exceeds the built-in scratch of the allocation-free entry point";
   }
   return "unknown status";
 }
@@ -341,6 +342,39 @@ jssa_status jssa_topk(const jssa_layout* L, const float* scores, const int32_t* 
   st = get_ws(L, k, window, workspace, ws_bytes, &w);
   if (st != JSSA_OK) return st;
   return run_topk(L, scores, L->T_cap, seq_lens, k, window, idx, n_sel, w, true, static_cast<cudaStream_t>(stream));
+}
+
+jssa_status jssa_topk_noalloc(const jssa_layout* L, const float* scores, const int32_t* seq_lens, int32_t k,
+                              int32_t window, int32_t* idx, int32_t* n_sel, void* stream) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  if (!scores || !seq_lens || !idx || !n_sel || k < 1 || k > kMaxK || window < 0) return JSSA_ERR_INVALID_ARG;
+  if (!aligned(scores, 4) || !aligned(idx, 4) || !aligned(n_sel, 4)) return JSSA_ERR_INVALID_ARG;
+  const int rows = L->B * L->Hkv;
+  if (rows > topk_noalloc_max_rows()) return JSSA_ERR_SCRATCH_LIMIT;
+  uint32_t* hist = nullptr;
+  st = cu(topk_noalloc_scratch(&hist));
+  if (st != JSSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the shared scratch keeps the previous call's contents: clear the histograms first
+  st = cu(cudaMemsetAsync(hist, 0, sizeof(uint32_t) * 4096 * rows, s));
+  if (st != JSSA_OK) return st;
+  TopkArgs a{};
+  a.scores = scores;
+  a.sc_ld = L->T_cap;
+  a.hist = hist;
+  a.seq_lens = seq_lens;
+  a.B = L->B;
+  a.Hkv = L->Hkv;
+  a.T_cap = L->T_cap;
+  a.k = k;
+  a.window = window;
+  a.idx = idx;
+  a.n_sel = n_sel;
+  a.status = nullptr;
+  st = cu(launch_topk_histogram(a, num_sms_current(), s));
+  if (st != JSSA_OK) return st;
+  return cu(launch_topk(a, s));
 }
 
 jssa_status jssa_indexed_attn(const jssa_layout* L, const void* Q, const void* K, const void* V, const int32_t* idx,

@@ -71,6 +71,10 @@ struct TopkArgs {
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 // Standalone path: build the per-row first-digit histogram (hist must be zeroed).
 cudaError_t launch_topk_histogram(const TopkArgs& a, int num_sms, cudaStream_t s);
+// Allocation-free selection: device address of the built-in histogram scratch on the
+// current device (looked up once per device), and the number of rows it holds.
+cudaError_t topk_noalloc_scratch(uint32_t** hist);
+int topk_noalloc_max_rows();
 
 struct AttnArgs {
   const void* Q;    // [B, Hq, dk]

@@ -30,6 +30,8 @@
 // bounded in time.
 #include <cooperative_groups.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -443,6 +445,36 @@ __global__ void __launch_bounds__(256) topk_hist_kernel(TopkArgs a) {
   uint32_t* g = a.hist + static_cast<int64_t>(row) * kBins1;
   for (int i = threadIdx.x; i < kBins1; i += blockDim.x)
     if (h[i]) atomicAdd(g + i, h[i]);
+}
+
+// ------------------------------------------------------------------ allocation-free variant
+// Scratch of jssa_topk_noalloc: the first-digit histograms (4096 counters, 16 KB) of up to
+// kNoAllocMaxRows (sequence, KV head) rows, in a file-scope device array: 4 MB that every
+// GPU which loads the library keeps until the process exits.  All calls share it.
+constexpr int kNoAllocMaxRows = 256;
+static __device__ __align__(256) uint32_t g_noalloc_hist[kNoAllocMaxRows * kBins1];
+
+int topk_noalloc_max_rows() { return kNoAllocMaxRows; }
+
+// Device address of g_noalloc_hist on the current device.  Host code cannot use the
+// array's name as a pointer (it denotes a host-side stand-in), so the address is looked
+// up with cudaGetSymbolAddress once per device, with that device current, and cached.
+cudaError_t topk_noalloc_scratch(uint32_t** out) {
+  static std::mutex mu;
+  static uint32_t* ptrs[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_hist);
+    if (e != cudaSuccess) return e;
+    ptrs[dev] = static_cast<uint32_t*>(p);
+  }
+  *out = ptrs[dev];
+  return cudaSuccess;
 }
 
 cudaError_t launch_topk_histogram(const TopkArgs& a, int, cudaStream_t s) {
