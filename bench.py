@@ -35,7 +35,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode steps/s and µs/step at 128K (1×B200); % of HBM roofline; × vs own dense kernel"
 UNIT = "steps/s"
-KERNELS_PER_STEP = 4  # prologue (qs + newest key + resets), score (+ digit-1 histogram), topk, attention (+ merge)
+# prologue (qs + newest key + resets), score (+ digit-1 histogram), topk, attention (+ merge in the GQA
+# kernel; the MLA path launches its merge separately)
+KERNELS_PER_STEP = {"gqa": 4, "mla": 5}
 
 
 def parse():
@@ -217,8 +219,9 @@ def stage_times(st, Q, reps=50):
         "topk_us": lambda: jssa.topk(st.L, sc, st.seq_lens, w.k, w.window, st.idx, st.nsel, st.ws),
         "attention_us": lambda: jssa.indexed_attn(st.L, Q, st.K, st.V, st.idx, w.k, st.nsel, st.seq_lens,
                                                   w.window, w.sm_scale, st.O, None, st.ws),
-        "dense_us": lambda: st.dense(Q),
     }
+    if st.w.mode != "mla":  # the MLA path is indexed only
+        calls["dense_us"] = lambda: st.dense(Q)
     out = {}
     for name, fn in calls.items():
         fn()
@@ -333,13 +336,15 @@ def main():
     value = world * args.steps / (ms / 1000.0)
     del g_warm, g_timed
 
-    # dense full-KV comparator at the same shape
-    nd = max(5, min(200, args.steps // 10))
-    g_dw = graph_of(st.dense, [Qs[i] for i in range(3)])
-    g_dw.replay()
-    g_d = graph_of(st.dense, [Qs[i % nq] for i in range(nd)])
-    dense_ms = timed_graph(g_d, barrier) / nd
-    del g_dw, g_d
+    # dense full-KV comparator at the same shape (GQA; the MLA path has no dense kernel)
+    dense_ms = None
+    if w.mode != "mla":
+        nd = max(5, min(200, args.steps // 10))
+        g_dw = graph_of(st.dense, [Qs[i] for i in range(3)])
+        g_dw.replay()
+        g_d = graph_of(st.dense, [Qs[i % nq] for i in range(nd)])
+        dense_ms = timed_graph(g_d, barrier) / nd
+        del g_dw, g_d
 
     stages = stage_times(st, Qs[0])
     hbm, peak_kind = peaks()
@@ -394,9 +399,10 @@ def main():
             "us_per_step": ms_step * 1000.0, "tokens_per_s": value * w.B,
             "bytes_per_step": bm["step"], "effective_GBps": bm["step"] / (ms_step * 1e-3) / 1e9,
             "step_hbm_frac": bm["step"] / (ms_step * 1e-3) / 1e9 / hbm,
-            "dense_us_per_step": dense_ms * 1000.0, "speedup_vs_dense": dense_ms / ms_step,
+            "dense_us_per_step": dense_ms * 1000.0 if dense_ms else None,
+            "speedup_vs_dense": dense_ms / ms_step if dense_ms else None,
             "byte_ratio": bm["dense"] / bm["step"],
-            "dense_hbm_frac": bm["dense"] / (dense_ms * 1e-3) / 1e9 / hbm,
+            "dense_hbm_frac": bm["dense"] / (dense_ms * 1e-3) / 1e9 / hbm if dense_ms else None,
             "stage_us": stages,
             "roofline": {"kernel": "score_kernel (timed together with its step prologue)", "bound": "hbm", "achieved": achieved, "peak": hbm,
                          "unit": "GB/s", "frac": achieved / hbm, "peak_kind": peak_kind,
@@ -405,7 +411,7 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": ne / (e2e_ms / 1000.0) * world, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "gpu_launches": KERNELS_PER_STEP[w.mode] * args.steps,
             "clocks": clk.summary(),
             "device_status": flags,
         }

@@ -115,6 +115,13 @@ def test_bad_layouts_are_rejected_on_the_host(lib, kw, code):
         assert got == code
 
 
+def test_mla_dense_decode_is_unsupported(lib):
+    # the MLA path is indexed only: the dense entry point refuses the layout before launching
+    L = _layout(mode=1, B=1, Hq=128, Hkv=1, d=576, dv=512, r=64)
+    assert lib.jssa_dense_decode(C.byref(L), FAKE, FAKE, FAKE, FAKE, 0, 1.0, FAKE, None, C.c_void_p(FAKE), 1 << 30,
+                                 None) == 2
+
+
 def test_bad_arguments_are_rejected_before_launch(lib):
     L = _layout()
     ws = C.c_void_p(FAKE)

@@ -200,6 +200,10 @@ def test_topk_with_few_distinct_values(T, k, levels):
     ("h128k", dict(B=1, T=3000, Hq=32, Hkv=2), [3000], 257, 0, 0),           # G = 16
     ("hybrid", dict(B=2, T=6000), [6000, 1500], 1024, 1024, 0),              # d = 256 + window
     ("hybrid", dict(B=1, T=2000), [2000], 7, 3, 1),                          # bf16 output
+    ("mla", dict(B=2, T=3000), [3000, 1234], 700, 0, 0),                     # tensor-core MLA kernel
+    ("mla", dict(B=1, T=4100), [4100], 2048, 0, 0),                          # 16 full 128-token tiles
+    ("mla", dict(B=3, T=2000), [2000, 333, 1999], 150, 64, 0),               # ragged tiles + window
+    ("mla", dict(B=1, T=1000), [1000], 37, 5, 1),                            # bf16 output
 ])
 def test_indexed_attention_matches_oracle(name, kw, seq, k, window, out):
     w = W[name].with_(**kw)
@@ -272,6 +276,38 @@ def test_sparse_with_k_equal_T_equals_dense():
     assert float((O_s - O_d).abs().max()) < 1e-5
 
 
+def test_mla_single_token_returns_the_latent_value_row():
+    # one selected token: P = 1 exactly, so O is the first 512 latent dims of that row, and
+    # lse is the scaled logit q_h . C_t over all 576 dims
+    w = W["mla"].with_(B=2, T=700)
+    p = Problem(w)
+    picks = [5, 699]
+    idx = torch.full((w.B, 1, 4), -1, dtype=torch.int32, device="cuda")
+    for b, t in enumerate(picks):
+        idx[b, 0, 0] = t
+    nsel = torch.ones((w.B, 1), dtype=torch.int32, device="cuda")
+    ws = p.workspace(4)
+    O = torch.empty((w.B, w.Hq, w.dv), device="cuda")
+    lse = torch.empty((w.B, w.Hq), device="cuda")
+    jssa.indexed_attn(p.L, p.Q, p.K, p.V, idx, 4, nsel, p.seq_lens, 0, w.sm_scale, O, lse, ws)
+    torch.cuda.synchronize()
+    for b, t in enumerate(picks):
+        row = p.K[b, 0, t].double().cpu()
+        assert torch.equal(O[b], p.K[b, 0, t, :w.dv].float().expand(w.Hq, -1))
+        ref = (p.Q[b].double().cpu() @ row) * w.sm_scale
+        np.testing.assert_allclose(lse[b].double().cpu().numpy(), ref.numpy(), atol=1e-4, rtol=1e-5)
+    _assert_status_clean(ws)
+
+
+def test_mla_has_no_dense_path():
+    w = W["mla"].with_(B=1, T=300)
+    p = Problem(w)
+    ws = p.workspace(4)
+    O = torch.empty((w.B, w.Hq, w.dv), device="cuda")
+    with pytest.raises(jssa.JssaError):
+        jssa.dense_decode(p.L, p.Q, p.K, p.V, p.seq_lens, 0, w.sm_scale, O, ws=ws)
+
+
 def test_single_token_selection_returns_the_value_row():
     w = W["tiny"].with_(T=600)
     p = Problem(w)
@@ -316,6 +352,7 @@ def _check_step(p, k, window, O, idx, nsel, rows, what):
     ("llama8b", dict(B=2, T=6000, k=512), [6000, 4321], 0),
     ("h128k", dict(B=2, T=20000, k=1024), [20000, 11111], 0),
     ("hybrid", dict(B=2, T=9000, k=512), [9000, 3000], 1024),
+    ("mla", dict(B=2, T=5000, k=512), [5000, 3210], 0),
 ])
 def test_decode_step_end_to_end(name, kw, seq, window):
     w = W[name].with_(**kw)

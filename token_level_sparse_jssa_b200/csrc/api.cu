@@ -86,9 +86,11 @@ jssa_status carve(const jssa_layout* L, int64_t k, int64_t window, void* base, W
   int S_cap = 1, S = 1, len = 0;
   attn_split_policy(L->mode, true, rows, min64(k + window, L->T_cap), num_sms, &S, &len);
   S_cap = S > S_cap ? S : S_cap;
-  attn_split_policy(L->mode, false, rows, L->T_cap, num_sms, &S, &len);
-  S_cap = S > S_cap ? S : S_cap;
-  if (window > 0) {
+  if (L->mode != JSSA_MODE_MLA) {  // MLA has no dense path
+    attn_split_policy(L->mode, false, rows, L->T_cap, num_sms, &S, &len);
+    S_cap = S > S_cap ? S : S_cap;
+  }
+  if (window > 0 && L->mode != JSSA_MODE_MLA) {
     attn_split_policy(L->mode, false, rows, min64(window, L->T_cap), num_sms, &S, &len);
     S_cap = S > S_cap ? S : S_cap;
   }
@@ -430,6 +432,7 @@ jssa_status jssa_dense_decode(const jssa_layout* L, const void* Q, const void* K
                               void* workspace, size_t ws_bytes, void* stream) {
   jssa_status st = check_layout(L);
   if (st != JSSA_OK) return st;
+  if (L->mode == JSSA_MODE_MLA) return JSSA_ERR_UNSUPPORTED;
   if (!Q || !K || !V || !seq_lens || !O || window < 0) return JSSA_ERR_INVALID_ARG;
   if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 4)) return JSSA_ERR_INVALID_ARG;
   Workspace w{};

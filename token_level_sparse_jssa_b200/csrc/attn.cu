@@ -523,10 +523,26 @@ __global__ void __launch_bounds__(256) merge_kernel(AttnArgs a) {
 // ------------------------------------------------------------------ host side
 void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int num_sms, int* S_out, int* split_out) {
   // Choose the split length (a multiple of the 16-token subtile, at least 64 tokens) that
-  // keeps the last wave of CTAs fullest; fewer splits win ties.  MLA splits are longer
-  // (each CTA amortises the 128-head query block over more tokens).
-  const int min_split = (mode == 1) ? 128 : 64;
-  const int slots = num_sms * ((mode == 1) ? 1 : 2);
+  // keeps the last wave of CTAs fullest; fewer splits win ties.
+  if (mode == 1) {
+    // MLA (tensor-core kernel): one tile of at most 128 tokens per CTA and one CTA per SM.
+    // Every CTA also streams the 147 KB query block and writes a 256 KB partial, about as
+    // much as a full tile's token work, so the cost is waves x (1 + len / 128).
+    if (list_max <= 0) { *S_out = 1; *split_out = mla_max_split(); return; }
+    int best_len = mla_max_split();
+    double best_cost = 1e300;
+    for (int len = mla_max_split(); len >= 16; len -= 16) {
+      const int64_t S = ceil_div(list_max, len);
+      const int64_t waves = ceil_div(static_cast<int64_t>(rows) * S, num_sms);
+      const double cost = static_cast<double>(waves) * (1.0 + len / 128.0);
+      if (cost < best_cost - 1e-9) { best_cost = cost; best_len = len; }
+    }
+    *split_out = best_len;
+    *S_out = static_cast<int>(ceil_div(list_max, best_len));
+    return;
+  }
+  const int min_split = 64;
+  const int slots = num_sms * 2;
   if (list_max <= 0) { *S_out = 1; *split_out = min_split; return; }
   int best_S = 0;
   int64_t best_len = 0;
@@ -536,15 +552,15 @@ void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int n
     if (len < min_split) len = min_split;
     const int64_t Sr = ceil_div(list_max, len);
     if (Sr != S) continue;
-    if (indexed && mode != 1 && len > kMaxTokList) continue;  // the token list lives in shared memory
-    if (indexed && mode != 1 && S > 8) break;                 // one cluster per row
+    if (indexed && len > kMaxTokList) continue;  // the token list lives in shared memory
+    if (indexed && S > 8) break;                 // one cluster per row
     const int64_t ctas = static_cast<int64_t>(rows) * Sr;
     const int64_t waves = ceil_div(ctas, slots);
     const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
     if (eff > best_eff + 0.02) { best_eff = eff; best_S = S; best_len = len; }
   }
   if (best_S == 0) {  // only reachable for very long lists
-    const int cap = (indexed && mode != 1) ? 8 : 256;
+    const int cap = indexed ? 8 : 256;
     best_len = ceil_div(ceil_div(list_max, cap), 16) * 16;
     best_S = static_cast<int>(ceil_div(list_max, best_len));
   }
