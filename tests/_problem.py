@@ -97,3 +97,37 @@ def score_error_bound(Qg: np.ndarray, P: np.ndarray, Kp: np.ndarray) -> np.ndarr
     r = kp.shape[1]
     qs_abs = np.abs(qs_exact) + err_qs
     return gam(r) * (np.abs(kp) @ qs_abs) + np.abs(kp) @ err_qs
+
+
+def check_step_rows(p: Problem, k: int, window: int, O, idx, nsel, rows, what="", kp_checked=False):
+    """Check sampled (b, h) rows of a decode step against the oracle run on the same inputs:
+    the selection within the tie window, and the attention output against the oracle's
+    (on the GPU's own index set when an allowed swap occurred).  Returns the number of rows
+    whose selection was identical."""
+    w = p.w
+    G = w.G
+    n_same = 0
+    for (b, h) in rows:
+        T = int(p.seq_lens[b])
+        hst = p.host(b, h)
+        Kp_or, _ = oracle.project_rows(hst["K"][:T], hst["P"])
+        if kp_checked:  # the scoring cache the step read is the oracle's projection, bit for bit
+            np.testing.assert_array_equal(hst["Kp"][:T], Kp_or)
+        res = oracle.decode_head(hst["Q"], hst["K"][:T], hst["V"][:T], Kp_or, hst["P"], T, k, window, w.sm_scale)
+        g_idx = idx[b, h].cpu().numpy()
+        _, same = check_selection(g_idx, int(nsel[b, h]), res["scores"], k)
+        O_gpu = O[b, h * G:(h + 1) * G].float().cpu().numpy().astype(np.float64)
+        if same:
+            O_ref = res["O"]
+            n_same += 1
+        else:  # an allowed swap inside the tie window: the oracle runs on the GPU's own set
+            n = int(nsel[b, h])
+            toks = np.concatenate([g_idx[:n], np.arange(T - min(window, T), T)])
+            O_ref, _ = oracle.attention(hst["Q"], hst["K"], hst["V"], toks, w.sm_scale)
+        check_attention(O_gpu, O_ref, f"{what} b={b} h={h}")
+    return n_same
+
+
+def assert_status_clean(ws):
+    code, flags = jssa.read_device_status(ws)
+    assert code == 0 and flags == 0, (code, flags)

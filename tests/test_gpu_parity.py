@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import oracle
-from tests._problem import Problem, check_attention, check_selection, score_error_bound
+from tests._problem import Problem, check_attention, check_selection, check_step_rows, score_error_bound
 from tests._util import u16, f32, rel_l2
 import token_level_sparse_jssa_b200 as jssa
 from token_level_sparse_jssa_b200 import synth
@@ -324,29 +324,6 @@ def test_single_token_selection_returns_the_value_row():
 
 
 # ----------------------------------------------------------------------------- fused step
-def _check_step(p, k, window, O, idx, nsel, rows, what):
-    w = p.w
-    G = w.G
-    n_same = 0
-    for (b, h) in rows:
-        T = int(p.seq_lens[b])
-        hst = p.host(b, h)
-        Kp_or, _ = oracle.project_rows(hst["K"][:T], hst["P"])
-        res = oracle.decode_head(hst["Q"], hst["K"][:T], hst["V"][:T], Kp_or, hst["P"], T, k, window, w.sm_scale)
-        g_idx = idx[b, h].cpu().numpy()
-        _, same = check_selection(g_idx, int(nsel[b, h]), res["scores"], k)
-        O_gpu = O[b, h * G:(h + 1) * G].float().cpu().numpy().astype(np.float64)
-        if same:
-            O_ref = res["O"]
-            n_same += 1
-        else:  # an allowed swap inside the tie window: the oracle runs on the GPU's own set
-            n = int(nsel[b, h])
-            toks = np.concatenate([g_idx[:n], np.arange(T - min(window, T), T)])
-            O_ref, _ = oracle.attention(hst["Q"], hst["K"], hst["V"], toks, w.sm_scale)
-        check_attention(O_gpu, O_ref, f"{what} b={b} h={h}")
-    return n_same
-
-
 @pytest.mark.parametrize("name,kw,seq,window", [
     ("tiny", {}, None, 0),
     ("llama8b", dict(B=2, T=6000, k=512), [6000, 4321], 0),
@@ -371,7 +348,7 @@ def test_decode_step_end_to_end(name, kw, seq, window):
             ref, _ = oracle.project_rows(u16(p.K[b, h, T - 1:T]), f32(p.P[h]))
             np.testing.assert_array_equal(u16(p.Kp[b, h, T - 1:T]), ref)
     rows = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
-    _check_step(p, w.k, window, O, idx, nsel, rows, name)
+    check_step_rows(p, w.k, window, O, idx, nsel, rows, name)
     _assert_status_clean(ws)
 
 
@@ -397,7 +374,7 @@ def test_decode_step_append_loop_updates_the_scoring_cache():
             for h in range(w.Hkv):
                 ref, _ = oracle.project_rows(u16(p.K[b, h, T - 1:T]), f32(p.P[h]))
                 np.testing.assert_array_equal(u16(p.Kp[b, h, T - 1:T]), ref)
-        _check_step(p, w.k, 0, O, idx, nsel, [(0, 0), (1, 7), (1, 3)], f"append step {step}")
+        check_step_rows(p, w.k, 0, O, idx, nsel, [(0, 0), (1, 7), (1, 3)], f"append step {step}")
 
 
 def test_decode_step_in_a_cuda_graph_matches_eager():
@@ -475,4 +452,4 @@ def test_empty_sequences_and_short_rows():
     assert torch.all(O[0] == 0) and torch.all(torch.isneginf(lse[0]))
     assert torch.all(nsel[0] == 0) and torch.all(idx[0] == -1)
     assert torch.all(nsel[1] == 5) and torch.equal(idx[1, :, :5].cpu(), torch.arange(5).expand(w.Hkv, 5).int())
-    _check_step(p, w.k, 0, O, idx, nsel, [(1, 0), (1, 1), (2, 0), (2, 1)], "short")
+    check_step_rows(p, w.k, 0, O, idx, nsel, [(1, 0), (1, 1), (2, 0), (2, 1)], "short")
