@@ -35,9 +35,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode steps/s and µs/step at 128K (1×B200); % of HBM roofline; × vs own dense kernel"
 UNIT = "steps/s"
-# prologue (qs + newest key + resets), score (+ digit-1 histogram), topk, attention (+ merge in the GQA
+# selection (query and newest-key projection, score scan, top-k) and attention (+ merge in the GQA
 # kernel; the MLA path launches its merge separately)
-KERNELS_PER_STEP = {"gqa": 4, "mla": 5}
+KERNELS_PER_STEP = {"gqa": 2, "mla": 3}   # caches up to 131072 tokens; longer ones add 2 (score, topk)
 
 
 def parse():
@@ -63,7 +63,10 @@ def byte_model(w, T, k, window, out_bytes=2):
     sel = rows * (keff + min(window, T)) * kv_row
     qo = w.B * w.Hq * (w.dk * 2 + w.dv * out_bytes)
     dense = rows * T * kv_row + qo
-    return dict(kp=kp, selected=sel, qo=qo, step=kp + sel + qo, dense=dense, scores=rows * n * 4)
+    # the selection kernel: Kp scan, queries, bases, the newest key row in and its Kp row
+    # out, indices and counts out (the scores and histograms stay on chip)
+    select = kp + w.B * w.Hq * w.dk * 2 + w.Hkv * w.dk * w.r * 4 + rows * (w.dk * 2 + w.r * 2) + rows * (k * 4 + 4)
+    return dict(kp=kp, selected=sel, qo=qo, step=kp + sel + qo, dense=dense, scores=rows * n * 4, select=select)
 
 
 def peaks():
@@ -209,14 +212,13 @@ def timed_graph(g, barrier):
 
 def stage_times(st, Q, reps=50):
     """Device time of the public entry points that make up the step, each replayed from a
-    CUDA graph of `reps` calls (CUDA events on the replay stream).  score = prologue +
-    score scan; topk = standalone selection (builds its own first-digit histogram);
-    attention = indexed attention with its fused merge."""
+    CUDA graph of `reps` calls (CUDA events on the replay stream).  select = the selection
+    half of the step (projections, score scan, top-k: one kernel when the cache fits a
+    cluster); attention = indexed attention with its merge; dense = the full-KV comparator."""
     jssa, w = st.jssa, st.w
-    sc = torch.empty(w.B, w.Hkv, st.T_cap, device="cuda")
     calls = {
-        "score_us": lambda: jssa.score(st.L, Q, st.P, st.Kp, st.seq_lens, w.window, sc, st.ws),
-        "topk_us": lambda: jssa.topk(st.L, sc, st.seq_lens, w.k, w.window, st.idx, st.nsel, st.ws),
+        "select_us": lambda: jssa.select(st.L, Q, st.K, st.Kp, st.P, st.seq_lens, 1, w.k, w.window, st.idx,
+                                         st.nsel, st.ws),
         "attention_us": lambda: jssa.indexed_attn(st.L, Q, st.K, st.V, st.idx, w.k, st.nsel, st.seq_lens,
                                                   w.window, w.sm_scale, st.O, None, st.ws),
     }
@@ -348,9 +350,9 @@ def main():
 
     stages = stage_times(st, Qs[0])
     hbm, peak_kind = peaks()
-    score_bytes = bm["kp"] + bm["scores"]
-    score_s = stages["score_us"] * 1e-6   # includes the (tiny) prologue launched with it
-    shash = source_hash("score.cu", "common.cuh")
+    sel_bytes = bm["select"]
+    sel_s = stages["select_us"] * 1e-6
+    shash = source_hash("select.cu", "common.cuh")
 
     # end to end through the public API with host buffers: per step, H2D of the query and of
     # the newest token's K/V rows from pinned memory, the step, and D2H of the output
@@ -391,7 +393,7 @@ def main():
         if not args.no_cpu_baseline and world == 1:
             rate, desc = cpu_oracle_rate(w, args.cpu_seconds, data=(st.K, st.V, Qs[0], st.P))
             cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
-        achieved = score_bytes / score_s / 1e9
+        achieved = sel_bytes / sel_s / 1e9
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -404,10 +406,11 @@ def main():
             "byte_ratio": bm["dense"] / bm["step"],
             "dense_hbm_frac": bm["dense"] / (dense_ms * 1e-3) / 1e9 / hbm if dense_ms else None,
             "stage_us": stages,
-            "roofline": {"kernel": "score_kernel (timed together with its step prologue)", "bound": "hbm", "achieved": achieved, "peak": hbm,
+            "roofline": {"kernel": "select_kernel (query and newest-key projection, score scan, top-k)",
+                         "bound": "hbm", "achieved": achieved, "peak": hbm,
                          "unit": "GB/s", "frac": achieved / hbm, "peak_kind": peak_kind,
-                         "traffic": traffic_for("score_kernel", w.name, shash),
-                         "algorithmic_bytes_per_launch": score_bytes},
+                         "traffic": traffic_for("select_kernel", w.name, shash),
+                         "algorithmic_bytes_per_launch": sel_bytes},
             "cpu_baseline": cpu,
             "e2e": {"value": ne / (e2e_ms / 1000.0) * world, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},

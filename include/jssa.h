@@ -191,6 +191,21 @@ JSSA_API jssa_status jssa_indexed_attn(const jssa_layout* L, const void* Q, cons
                               void* O, float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * The selection half of a decode step (Figure 1 up to the "top-B positions"; §3.2 keys
+ * projected on write): project the last n_new rows of each sequence into Kp, form the
+ * projected group query, score every candidate [0, T_b - W) and select the top-k per
+ * (sequence, KV head), with the ties, ordering and padding rules of jssa_topk.
+ *   idx    device int32 [B, Hkv, k]      n_sel  device int32 [B, Hkv]
+ * When T_cap <= 131072 all of this runs in one kernel with one 8-CTA cluster per
+ * (sequence, KV head), the scores never leaving shared memory; longer caches take the
+ * jssa_score + jssa_topk kernels.  Up to 16 appended rows are projected inside the
+ * selection; more are projected by the bulk projection kernel first.
+ */
+JSSA_API jssa_status jssa_select(const jssa_layout* L, const void* Q, const void* K, void* Kp, const float* P,
+                                 const int32_t* seq_lens, int32_t n_new, int32_t k, int32_t window, int32_t* idx,
+                                 int32_t* n_sel, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * One fused decode step (Figure 1): project the last n_new rows of each sequence
  * into Kp (n_new may be 0 when Kp is already current), score, select the top-k per
  * (sequence, KV head), attend over the selection (plus the window) and merge.

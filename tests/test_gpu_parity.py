@@ -330,6 +330,7 @@ def test_single_token_selection_returns_the_value_row():
     ("h128k", dict(B=2, T=20000, k=1024), [20000, 11111], 0),
     ("hybrid", dict(B=2, T=9000, k=512), [9000, 3000], 1024),
     ("mla", dict(B=2, T=5000, k=512), [5000, 3210], 0),
+    ("h128k", dict(B=1, Hq=8, Hkv=2, T=140000, k=1024), [140000], 0),   # rows beyond one cluster: unfused path
 ])
 def test_decode_step_end_to_end(name, kw, seq, window):
     w = W[name].with_(**kw)
@@ -349,6 +350,51 @@ def test_decode_step_end_to_end(name, kw, seq, window):
             np.testing.assert_array_equal(u16(p.Kp[b, h, T - 1:T]), ref)
     rows = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
     check_step_rows(p, w.k, window, O, idx, nsel, rows, name)
+    _assert_status_clean(ws)
+
+
+@pytest.mark.parametrize("name,kw,seq,window", [
+    ("tiny", {}, None, 0),
+    ("h128k", dict(B=3, T=20000, k=2048), [20000, 1500, 19999], 0),     # one row below k: select all
+    ("hybrid", dict(B=2, T=9000, k=512), [9000, 1800], 1024),
+    ("mla", dict(B=2, T=7000, k=700), [7000, 6001], 0),
+    ("h128k", dict(B=1, Hq=8, Hkv=2, T=131073, k=512), [131073], 0),   # one token beyond the fused kernel
+])
+def test_select_matches_the_oracle_selection(name, kw, seq, window):
+    w = W[name].with_(**kw)
+    p = Problem(w, seq_lens=seq)
+    p.fill_kp()
+    ws = p.workspace(w.k, window)
+    idx = torch.full((w.B, w.Hkv, w.k), -7, dtype=torch.int32, device="cuda")
+    nsel = torch.full((w.B, w.Hkv), -7, dtype=torch.int32, device="cuda")
+    jssa.select(p.L, p.Q, p.K, p.Kp, p.P, p.seq_lens, 0, w.k, window, idx, nsel, ws)
+    torch.cuda.synchronize()
+    for b in range(w.B):
+        T = int(p.seq_lens[b])
+        for h in range(w.Hkv):
+            hst = p.host(b, h)
+            res = oracle.decode_head(hst["Q"], hst["K"][:T], hst["V"][:T], hst["Kp"][:T], hst["P"], T, w.k, window,
+                                     w.sm_scale)
+            check_selection(idx[b, h].cpu().numpy(), int(nsel[b, h]), res["scores"], w.k)
+    _assert_status_clean(ws)
+
+
+@pytest.mark.parametrize("n_new", [3, 16, 40])
+def test_decode_step_projects_many_appended_rows(n_new):
+    # up to 16 appended rows are projected inside the selection kernel, more by the bulk kernel first
+    w = W["tiny"].with_(B=2, T=3000, k=200)
+    p = Problem(w, seq_lens=[3000, 2000])
+    p.fill_kp()
+    for b, T in enumerate([3000, 2000]):
+        p.Kp[b, :, T - n_new:T] = 0
+    ws = p.workspace(w.k)
+    O = torch.full((w.B, w.Hq, w.dv), float("nan"), device="cuda")
+    idx = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device="cuda")
+    nsel = torch.empty((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+    jssa.decode_step(p.L, p.Q, p.K, p.V, p.Kp, p.P, p.seq_lens, n_new, w.k, 0, w.sm_scale, O, None, idx, nsel, ws)
+    torch.cuda.synchronize()
+    rows = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    check_step_rows(p, w.k, 0, O, idx, nsel, rows, f"n_new={n_new}", kp_checked=True)
     _assert_status_clean(ws)
 
 

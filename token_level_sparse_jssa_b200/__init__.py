@@ -10,5 +10,5 @@ fails loudly if it has not been built.
 """
 from ._binding import (  # noqa: F401
     EXPORTS, LIB_PATH, MODE_GQA, MODE_MLA, OUT_BF16, OUT_F32, JssaError, Layout, alloc_workspace, decode_step,
-    dense_decode, indexed_attn, load, make_layout, project_keys, read_device_status, score, status_string, topk,
+    dense_decode, indexed_attn, load, make_layout, project_keys, read_device_status, score, select, status_string, topk,
     topk_noalloc, version, workspace_init, workspace_size)

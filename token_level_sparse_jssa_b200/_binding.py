@@ -24,7 +24,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape or mode", 3: "wo
 DEV_BAD_SEQ_LEN, DEV_BAD_INDEX, DEV_BAD_NSEL, DEV_TIMEOUT = 1, 2, 4, 8
 
 EXPORTS = ("jssa_status_string", "jssa_version", "jssa_workspace_size", "jssa_project_keys", "jssa_score",
-           "jssa_topk", "jssa_topk_noalloc", "jssa_indexed_attn", "jssa_decode_step", "jssa_dense_decode",
+           "jssa_topk", "jssa_topk_noalloc", "jssa_select", "jssa_indexed_attn", "jssa_decode_step",
+           "jssa_dense_decode",
            "jssa_workspace_init", "jssa_read_device_status")
 
 
@@ -63,6 +64,7 @@ def load(path: str = LIB_PATH):
         "jssa_score": (C.c_int, [LP, vp, vp, vp, vp, i32, vp, vp, sz, vp]),
         "jssa_topk": (C.c_int, [LP, vp, vp, i32, i32, vp, vp, vp, sz, vp]),
         "jssa_topk_noalloc": (C.c_int, [LP, vp, vp, i32, i32, vp, vp, vp]),
+        "jssa_select": (C.c_int, [LP, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
         "jssa_indexed_attn": (C.c_int, [LP, vp, vp, vp, vp, i32, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
         "jssa_decode_step": (C.c_int, [LP, vp, vp, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, vp, vp, sz, vp]),
         "jssa_dense_decode": (C.c_int, [LP, vp, vp, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
@@ -179,6 +181,12 @@ def indexed_attn(L, Q, K, V, idx, k: int, n_sel, seq_lens, window: int, sm_scale
     _check("jssa_indexed_attn", load().jssa_indexed_attn(C.byref(L), _c(Q), _p(K), _p(V), _c(idx), k, _c(n_sel),
                                                          _c(seq_lens), window, sm_scale, _c(O), _c(lse), w, n,
                                                          _stream(stream)))
+
+
+def select(L, Q, K, Kp, P, seq_lens, n_new: int, k: int, window: int, idx, n_sel, ws, stream=None):
+    w, n = _ws(ws)
+    _check("jssa_select", load().jssa_select(C.byref(L), _c(Q), _p(K), _p(Kp), _c(P), _c(seq_lens), n_new, k,
+                                             window, _c(idx), _c(n_sel), w, n, _stream(stream)))
 
 
 def decode_step(L, Q, K, V, Kp, P, seq_lens, n_new: int, k: int, window: int, sm_scale: float, O, lse=None,

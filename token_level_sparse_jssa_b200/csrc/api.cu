@@ -271,6 +271,49 @@ jssa_status run_attention(const jssa_layout* L, const void* Q, const void* K, co
   return cu(launch_attention(a, s));  // merges in its last CTA per row
 }
 
+// The selection half of the step: newest-key projection, query projection, scan, top-k.
+jssa_status run_select(const jssa_layout* L, const void* Q, const void* K, void* Kp, const float* P,
+                       const int32_t* seq_lens, int n_new, int k, int window, int32_t* idx, int32_t* nsel,
+                       const Workspace& w, cudaStream_t s) {
+  jssa_status st = JSSA_OK;
+  if (n_new > kMaxPrologueRows) {  // long appends go through the bulk projection kernel
+    ProjectArgs pa = project_args(L, K, P, Kp, nullptr, seq_lens, n_new, w.status);
+    st = cu(launch_project_keys(pa, s));
+    if (st != JSSA_OK) return st;
+  }
+  const int n_in = n_new > kMaxPrologueRows ? 0 : n_new;
+  if (L->T_cap <= select_max_candidates()) {
+    // rows that fit a cluster's shared memory: projections, scan and top-k in one kernel
+    SelectArgs sa{};
+    sa.Q = Q;
+    sa.P = P;
+    sa.K = K;
+    memcpy(sa.ks, L->k_stride, sizeof sa.ks);
+    sa.Kp = Kp;
+    memcpy(sa.ps, L->kp_stride, sizeof sa.ps);
+    sa.seq_lens = seq_lens;
+    sa.n_new = n_in;
+    sa.B = L->B;
+    sa.Hq = L->Hq;
+    sa.Hkv = L->Hkv;
+    sa.d = L->d_k;
+    sa.r = L->r;
+    sa.T_cap = L->T_cap;
+    sa.window = window;
+    sa.k = k;
+    sa.idx = idx;
+    sa.n_sel = nsel;
+    sa.counters = w.counters;
+    sa.status = w.status;
+    return cu(launch_select(sa, num_sms_current(), s));
+  }
+  st = run_prologue(L, Q, P, K, Kp, seq_lens, n_in, w, s);
+  if (st != JSSA_OK) return st;
+  st = run_score(L, Kp, seq_lens, window, w.scores, w.sc_ld, w, s);
+  if (st != JSSA_OK) return st;
+  return run_topk(L, w.scores, w.sc_ld, seq_lens, k, window, idx, nsel, w, false, s);
+}
+
 }  // namespace
 }  // namespace jssa
 
@@ -395,6 +438,23 @@ jssa_status jssa_indexed_attn(const jssa_layout* L, const void* Q, const void* K
                        static_cast<cudaStream_t>(stream));
 }
 
+jssa_status jssa_select(const jssa_layout* L, const void* Q, const void* K, void* Kp, const float* P,
+                        const int32_t* seq_lens, int32_t n_new, int32_t k, int32_t window, int32_t* idx,
+                        int32_t* n_sel, void* workspace, size_t ws_bytes, void* stream) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  if (!Q || !K || !Kp || !P || !seq_lens || !idx || !n_sel || k < 1 || k > kMaxK || window < 0 || n_new < 0 ||
+      n_new > L->T_cap)
+    return JSSA_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(Kp, 16) || !aligned(P, 16) || !aligned(idx, 4) ||
+      !aligned(n_sel, 4))
+    return JSSA_ERR_INVALID_ARG;
+  Workspace w{};
+  st = get_ws(L, k, window, workspace, ws_bytes, &w);
+  if (st != JSSA_OK) return st;
+  return run_select(L, Q, K, Kp, P, seq_lens, n_new, k, window, idx, n_sel, w, static_cast<cudaStream_t>(stream));
+}
+
 jssa_status jssa_decode_step(const jssa_layout* L, const void* Q, const void* K, const void* V, void* Kp,
                              const float* P, const int32_t* seq_lens, int32_t n_new, int32_t k, int32_t window,
                              float sm_scale, void* O, float* lse, int32_t* idx_out, int32_t* n_sel_out, void* workspace,
@@ -411,18 +471,9 @@ jssa_status jssa_decode_step(const jssa_layout* L, const void* Q, const void* K,
   st = get_ws(L, k, window, workspace, ws_bytes, &w);
   if (st != JSSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (n_new > kMaxPrologueRows) {  // long appends go through the bulk projection kernel
-    ProjectArgs pa = project_args(L, K, P, Kp, nullptr, seq_lens, n_new, w.status);
-    st = cu(launch_project_keys(pa, s));
-    if (st != JSSA_OK) return st;
-  }
-  st = run_prologue(L, Q, P, K, Kp, seq_lens, n_new > kMaxPrologueRows ? 0 : n_new, w, s);
-  if (st != JSSA_OK) return st;
-  st = run_score(L, Kp, seq_lens, window, w.scores, w.sc_ld, w, s);
-  if (st != JSSA_OK) return st;
   int32_t* idx = idx_out ? idx_out : w.idx;
   int32_t* nsel = n_sel_out ? n_sel_out : w.n_sel;
-  st = run_topk(L, w.scores, w.sc_ld, seq_lens, k, window, idx, nsel, w, false, s);
+  st = run_select(L, Q, K, Kp, P, seq_lens, n_new, k, window, idx, nsel, w, s);
   if (st != JSSA_OK) return st;
   return run_attention(L, Q, K, V, idx, k, nsel, seq_lens, window, sm_scale, O, lse, w, true, s);
 }

@@ -100,6 +100,30 @@ struct AttnArgs {
   int out_bf16;
   int* status;
 };
+// Fused selection (query projection, newest-key projection, score scan, top-k) with one
+// 8-CTA cluster per (sequence, KV head); rows of up to select_max_candidates() tokens.
+struct SelectArgs {
+  const void* Q;     // [B, Hq, d]
+  const float* P;    // [Hkv, d, r]
+  const void* K;     // newest rows projected from here
+  int64_t ks[3];
+  void* Kp;
+  int64_t ps[3];
+  const int32_t* seq_lens;
+  int n_new;         // <= select_max_new_rows()
+  int B, Hq, Hkv, d, r;
+  int64_t T_cap;
+  int window, k;
+  int per, stages;   // set by the launcher
+  int32_t* idx;      // [B*Hkv, k]
+  int32_t* n_sel;    // [B*Hkv]
+  int* counters;     // nullable: attention arrival counters zeroed here
+  int* status;
+};
+cudaError_t launch_select(const SelectArgs& a, int num_sms, cudaStream_t s);
+int64_t select_max_candidates();
+int select_max_new_rows();
+
 // Split policy shared by the workspace sizing and the launch.
 void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int num_sms, int* S, int* split_len);
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);   // GQA path
