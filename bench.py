@@ -274,12 +274,34 @@ def cpu_oracle_rate(w, seconds: float, data=None):
     return 1.0 / step_s, desc
 
 
+# --------------------------------------------------------------------------- ranks
+def rank_env():
+    """(rank, world, local_rank) from the launcher's environment (1 process when absent)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, dist=None, device="cuda") -> float:
+    """The maximum of a per-rank scalar over all ranks (identity without a process group)."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, steps: int, ms: float) -> float:
+    """Steps per second of the whole job: every rank ran `steps` steps of its own batch and
+    the slowest rank took `ms` milliseconds."""
+    return world * steps / (ms / 1000.0)
+
+
 # --------------------------------------------------------------------------- arms
 def run_reference(args, w, cfg):
-    rank = int(os.environ.get("RANK", "0"))
+    rank, _, _ = rank_env()
     if rank != 0:
         return 0
-    rate, desc = cpu_oracle_rate(w, max(5.0, args.cpu_seconds))
+    rate, desc = cpu_oracle_rate(w, max(0.2, args.cpu_seconds))
     line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / rate, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
@@ -293,9 +315,7 @@ def main():
     args = parse()
     from token_level_sparse_jssa_b200 import synth
     w = synth.WORKLOADS[args.workload]
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = rank_env()
     bm = byte_model(w, w.T, w.k, w.window)
     cfg = {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} d_k={w.dk} d_v={w.dv} r={w.r} T={w.T} k={w.k}"
                        + (f" W={w.window}" if w.window else "") + f" ({w.mode.upper()})",
@@ -330,12 +350,9 @@ def main():
     g_timed = graph_of(st.step, [Qs[args.warmup + i] for i in range(args.steps)])
     with ClockSampler(local) as clk:
         ms = timed_graph(g_timed, barrier)
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist)
     ms_step = ms / args.steps
-    value = world * args.steps / (ms / 1000.0)
+    value = whole_job_rate(world, args.steps, ms)
     del g_warm, g_timed
 
     # dense full-KV comparator at the same shape (GQA; the MLA path has no dense kernel)
@@ -345,7 +362,7 @@ def main():
         g_dw = graph_of(st.dense, [Qs[i] for i in range(3)])
         g_dw.replay()
         g_d = graph_of(st.dense, [Qs[i % nq] for i in range(nd)])
-        dense_ms = timed_graph(g_d, barrier) / nd
+        dense_ms = max_over_ranks(timed_graph(g_d, barrier) / nd, dist)
         del g_dw, g_d
 
     stages = stage_times(st, Qs[0])
@@ -380,10 +397,7 @@ def main():
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist)
     h2d = Qd.numel() * 2 + newk.numel() * 2 + (newv.numel() * 2 if newv is not None else 0)
     d2h = Oh.numel() * Oh.element_size()
 
@@ -412,7 +426,7 @@ def main():
                          "traffic": traffic_for("select_kernel", w.name, shash),
                          "algorithmic_bytes_per_launch": sel_bytes},
             "cpu_baseline": cpu,
-            "e2e": {"value": ne / (e2e_ms / 1000.0) * world, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "e2e": {"value": whole_job_rate(world, ne, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": KERNELS_PER_STEP[w.mode] * args.steps,
             "clocks": clk.summary(),
