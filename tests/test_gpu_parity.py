@@ -331,6 +331,10 @@ def test_single_token_selection_returns_the_value_row():
     ("hybrid", dict(B=2, T=9000, k=512), [9000, 3000], 1024),
     ("mla", dict(B=2, T=5000, k=512), [5000, 3210], 0),
     ("h128k", dict(B=1, Hq=8, Hkv=2, T=140000, k=1024), [140000], 0),   # rows beyond one cluster: unfused path
+    ("h128k", dict(B=2, T=3000, Hq=16, Hkv=16, k=300), [3000, 2500], 0),   # G = 1
+    ("h128k", dict(B=1, T=3000, Hq=32, Hkv=2, k=257), [3000], 0),           # G = 16
+    ("tiny", dict(T=1000, dk=64, dv=64, r=8, k=100), None, 0),               # d = 64
+    ("h128k", dict(B=2, T=5000, k=512), [5000, 300], 700),                   # window; a row below k
 ])
 def test_decode_step_end_to_end(name, kw, seq, window):
     w = W[name].with_(**kw)
@@ -396,6 +400,22 @@ def test_decode_step_projects_many_appended_rows(n_new):
     rows = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
     check_step_rows(p, w.k, 0, O, idx, nsel, rows, f"n_new={n_new}", kp_checked=True)
     _assert_status_clean(ws)
+
+
+def test_decode_step_bf16_output_is_the_rounded_fp32_result():
+    w = W["h128k"].with_(B=2, T=6000, k=700)
+    p32 = Problem(w, seq_lens=[6000, 4444])
+    p16 = Problem(w, seq_lens=[6000, 4444], out_dtype=jssa.OUT_BF16)
+    for p in (p32, p16):
+        p.fill_kp()
+    O32 = torch.empty((w.B, w.Hq, w.dv), device="cuda")
+    O16 = torch.empty((w.B, w.Hq, w.dv), device="cuda", dtype=torch.bfloat16)
+    jssa.decode_step(p32.L, p32.Q, p32.K, p32.V, p32.Kp, p32.P, p32.seq_lens, 0, w.k, 0, w.sm_scale, O32,
+                     ws=p32.workspace(w.k))
+    jssa.decode_step(p16.L, p16.Q, p16.K, p16.V, p16.Kp, p16.P, p16.seq_lens, 0, w.k, 0, w.sm_scale, O16,
+                     ws=p16.workspace(w.k))
+    torch.cuda.synchronize()
+    assert torch.equal(O16, O32.to(torch.bfloat16))
 
 
 def test_decode_step_append_loop_updates_the_scoring_cache():

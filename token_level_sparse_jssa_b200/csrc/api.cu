@@ -271,10 +271,21 @@ jssa_status run_attention(const jssa_layout* L, const void* Q, const void* K, co
   return cu(launch_attention(a, s));  // merges in its last CTA per row
 }
 
-// The selection half of the step: newest-key projection, query projection, scan, top-k.
+// Attention to run inside the selection kernel (nullptr: none).
+struct FusedAttn {
+  const void* V;
+  float sm_scale;
+  void* O;
+  float* lse;
+};
+
+// The selection half of the step: newest-key projection, query projection, scan, top-k;
+// with `fa`, also the attention of the selected rows when the selection kernel can run it
+// (*fused is then set).
 jssa_status run_select(const jssa_layout* L, const void* Q, const void* K, void* Kp, const float* P,
                        const int32_t* seq_lens, int n_new, int k, int window, int32_t* idx, int32_t* nsel,
-                       const Workspace& w, cudaStream_t s) {
+                       const Workspace& w, cudaStream_t s, const FusedAttn* fa = nullptr, bool* fused = nullptr) {
+  if (fused) *fused = false;
   jssa_status st = JSSA_OK;
   if (n_new > kMaxPrologueRows) {  // long appends go through the bulk projection kernel
     ProjectArgs pa = project_args(L, K, P, Kp, nullptr, seq_lens, n_new, w.status);
@@ -305,6 +316,22 @@ jssa_status run_select(const jssa_layout* L, const void* Q, const void* K, void*
     sa.n_sel = nsel;
     sa.counters = w.counters;
     sa.status = w.status;
+    if (fa && L->mode == JSSA_MODE_GQA) {
+      sa.V = fa->V;
+      memcpy(sa.vs, L->v_stride, sizeof sa.vs);
+      sa.sm_scale = fa->sm_scale;
+      sa.O = fa->O;
+      sa.lse = fa->lse;
+      sa.out_bf16 = (L->out_dtype == JSSA_OUT_BF16);
+      const cudaError_t e = launch_select(sa, num_sms_current(), s);
+      if (e == cudaSuccess) {
+        if (fused) *fused = true;
+        return JSSA_OK;
+      }
+      if (e != cudaErrorNotSupported) return cu(e);
+      (void)cudaGetLastError();
+      sa.V = nullptr;  // this shape keeps the attention in its own kernel
+    }
     return cu(launch_select(sa, num_sms_current(), s));
   }
   st = run_prologue(L, Q, P, K, Kp, seq_lens, n_in, w, s);
@@ -473,8 +500,10 @@ jssa_status jssa_decode_step(const jssa_layout* L, const void* Q, const void* K,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* idx = idx_out ? idx_out : w.idx;
   int32_t* nsel = n_sel_out ? n_sel_out : w.n_sel;
-  st = run_select(L, Q, K, Kp, P, seq_lens, n_new, k, window, idx, nsel, w, s);
-  if (st != JSSA_OK) return st;
+  const FusedAttn fa{V, sm_scale, O, lse};
+  bool fused = false;
+  st = run_select(L, Q, K, Kp, P, seq_lens, n_new, k, window, idx, nsel, w, s, &fa, &fused);
+  if (st != JSSA_OK || fused) return st;
   return run_attention(L, Q, K, V, idx, k, nsel, seq_lens, window, sm_scale, O, lse, w, true, s);
 }
 

@@ -22,163 +22,13 @@
 // cluster and combines the partials by log-sum-exp through distributed shared memory;
 // the dense decode, with many more splits, writes partials to the workspace and the last
 // CTA of each row to finish (a per-row arrival counter) combines them.
-#include <cooperative_groups.h>
-
-#include <cmath>
-
-#include "common.cuh"
-#include "launch.h"
-
-namespace cg = cooperative_groups;
+#include "attn_core.cuh"
 
 namespace jssa {
-
-constexpr int kAttnWarps = 4;
-constexpr int kAttnThreads = kAttnWarps * 32;
-constexpr int kSub = 16;                 // tokens per warp subtile
-constexpr int kMaxTokList = 4096;        // indexed mode: split length bound (token list in smem)
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-
-template <int D>
-struct AttnCfg {
-  static constexpr int STAGES = (D <= 64) ? 4 : (D <= 128 ? 3 : 2);
-  static constexpr int CPR = D / 8;                    // 16-byte chunks per row
-  static constexpr int SUB_BYTES = kSub * D * 2;       // one K or V subtile
-  static constexpr int STAGE_BYTES = 2 * SUB_BYTES;
-  static constexpr int RING_BYTES = kAttnWarps * STAGES * STAGE_BYTES;
-  static constexpr int COMBINE_BYTES = kAttnWarps * 16 * D * 4 + 2 * kAttnWarps * 16 * 4;
-  static constexpr int PART_BYTES = 16 * D * 4 + 16 * 4;   // this CTA's partial (o, lse) for the cluster merge
-  static constexpr int MAIN_BYTES =
-      RING_BYTES > COMBINE_BYTES + PART_BYTES ? RING_BYTES : COMBINE_BYTES + PART_BYTES;
-};
 
 template <int D, bool DENSE>
 static size_t attn_smem_bytes() {
   return AttnCfg<D>::MAIN_BYTES + (DENSE ? 0 : kMaxTokList * sizeof(int32_t));
-}
-
-// Combine the S split partials of query heads [hq0, hq0 + G) into O (and lse):
-// O = sum_s w_s o_s with w_s = exp(lse_s - M) / sum_s' exp(lse_s' - M), M = max lse;
-// lse = M + log(sum exp(lse_s - M)).  Run by the last CTA of a row to finish, on
-// partials every CTA made visible with a device-scope fence before counting itself
-// in.  The split weights go through shared memory (wsm: G * S floats); every thread
-// then issues all the loads of two outputs (up to 16 splits each) before using them,
-// so the merge costs about one memory round trip per two outputs.
-constexpr int kMergeUnroll = 16;
-template <int D>
-__device__ __forceinline__ void merge_row(const AttnArgs& a, int64_t hq0, int G, float* wsm) {
-  const int S = a.S;
-  for (int i = threadIdx.x; i < G * S; i += blockDim.x) wsm[i] = __ldcg(a.part_lse + (hq0 + i / S) * S + i % S);
-  __syncthreads();
-  if (threadIdx.x < G) {
-    float* w = wsm + threadIdx.x * S;
-    float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, w[s]);
-    float L = 0.f;
-    if (M != -INFINITY)
-      for (int s = 0; s < S; ++s) { w[s] = expf(w[s] - M); L += w[s]; }
-    const float inv = (M != -INFINITY) ? 1.f / L : 0.f;
-    for (int s = 0; s < S; ++s) w[s] = (M != -INFINITY) ? w[s] * inv : 0.f;
-    if (a.lse) a.lse[hq0 + threadIdx.x] = (M == -INFINITY) ? -INFINITY : M + logf(L);
-  }
-  __syncthreads();
-  for (int i0 = threadIdx.x; i0 < G * D; i0 += 2 * blockDim.x) {
-    const int i1 = i0 + blockDim.x;
-    const bool has1 = i1 < G * D;
-    const int h0 = i0 / D, d0 = i0 % D, h1 = has1 ? i1 / D : h0, d1 = has1 ? i1 % D : d0;
-    const float* o0 = a.part_o + (hq0 + h0) * S * D + d0;
-    const float* o1 = a.part_o + (hq0 + h1) * S * D + d1;
-    float acc0 = 0.f, acc1 = 0.f;
-    for (int s0 = 0; s0 < S; s0 += kMergeUnroll) {
-      float v0[kMergeUnroll], v1[kMergeUnroll];
-#pragma unroll
-      for (int u = 0; u < kMergeUnroll; ++u) {
-        const bool ok = s0 + u < S;
-        v0[u] = ok ? __ldcg(o0 + static_cast<int64_t>(s0 + u) * D) : 0.f;
-        v1[u] = (ok && has1) ? __ldcg(o1 + static_cast<int64_t>(s0 + u) * D) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < kMergeUnroll; ++u) {
-        if (s0 + u < S) {
-          acc0 = fmaf(wsm[h0 * S + s0 + u], v0[u], acc0);
-          acc1 = fmaf(wsm[h1 * S + s0 + u], v1[u], acc1);
-        }
-      }
-    }
-    const int64_t q0 = hq0 + h0, q1 = hq0 + h1;
-    if (a.out_bf16) {
-      static_cast<__nv_bfloat16*>(a.O)[q0 * D + d0] = __float2bfloat16_rn(acc0);
-      if (has1) static_cast<__nv_bfloat16*>(a.O)[q1 * D + d1] = __float2bfloat16_rn(acc1);
-    } else {
-      static_cast<float*>(a.O)[q0 * D + d0] = acc0;
-      if (has1) static_cast<float*>(a.O)[q1 * D + d1] = acc1;
-    }
-  }
-}
-
-// Count this CTA's finished partial in; the CTA that completes the row merges it and
-// re-arms the counter for the next call.
-template <int D>
-__device__ __forceinline__ void finish_split(const AttnArgs& a, int row, int64_t hq0, int G, float* wsm) {
-  __shared__ int is_last;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int prev = atomicAdd(a.counters + row, 1);
-    is_last = (prev == a.S - 1);
-  }
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  merge_row<D>(a, hq0, G, wsm);
-  if (threadIdx.x == 0) a.counters[row] = 0;
-}
-
-// Split merge inside a thread-block cluster (one CTA per split of the row, S <= 8):
-// every CTA keeps its normalised partial (o, lse) in its own shared memory; after a
-// cluster barrier CTA c combines output slice c of the row, reading the S partials
-// through distributed shared memory, and a second barrier keeps the partials alive
-// until every CTA has read them.
-template <int D>
-__device__ __forceinline__ void cluster_merge(const AttnArgs& a, int64_t hq0, int G, const float* pbuf,
-                                              const float* plse) {
-  __shared__ float wts[16 * 8];
-  cg::cluster_group cl = cg::this_cluster();
-  const int S = static_cast<int>(cl.num_blocks());
-  const int c = static_cast<int>(cl.block_rank());
-  cl.sync();
-  for (int i = threadIdx.x; i < G * S; i += blockDim.x) wts[i] = cl.map_shared_rank(plse, i % S)[i / S];
-  __syncthreads();
-  if (threadIdx.x < G) {
-    float* w = wts + threadIdx.x * S;
-    float M = -INFINITY;
-    for (int q = 0; q < S; ++q) M = fmaxf(M, w[q]);
-    float L = 0.f;
-    for (int q = 0; q < S; ++q) {
-      w[q] = (M == -INFINITY) ? 0.f : expf(w[q] - M);
-      L += w[q];
-    }
-    for (int q = 0; q < S; ++q) w[q] = (L > 0.f) ? w[q] / L : 0.f;
-    if (a.lse && c == 0) a.lse[hq0 + threadIdx.x] = (M == -INFINITY) ? -INFINITY : M + logf(L);
-  }
-  __syncthreads();
-  const int per = (G * D + S - 1) / S;
-  const int lo = c * per, hi = min(G * D, lo + per);
-  for (int i = lo + threadIdx.x; i < hi; i += blockDim.x) {
-    const int head = i / D;
-    float v[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) v[q] = (q < S) ? cl.map_shared_rank(pbuf, q)[i] : 0.f;
-    float o = 0.f;
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      if (q < S) o = fmaf(wts[head * S + q], v[q], o);
-    const int64_t qi = hq0 + head;
-    if (a.out_bf16) static_cast<__nv_bfloat16*>(a.O)[qi * D + (i % D)] = __float2bfloat16_rn(o);
-    else static_cast<float*>(a.O)[qi * D + (i % D)] = o;
-  }
-  cl.sync();
 }
 
 template <int D, int NTILE, bool DENSE>
@@ -212,24 +62,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
       pre[u] = (threadIdx.x + u * kAttnThreads < a.split_len && pos < a.idx_ld) ? __ldg(irow + pos) : -1;
     }
   }
-  // Q^T as MMA B fragments: head nt*8 + g, dims kk*16 + 2c (+8)
   uint32_t qf[NTILE][KSTEPS][2];
-  const __nv_bfloat16* Qg = static_cast<const __nv_bfloat16*>(a.Q) + hq0 * D;
-#pragma unroll
-  for (int nt = 0; nt < NTILE; ++nt) {
-    const int head = nt * 8 + g;
-#pragma unroll
-    for (int kk = 0; kk < KSTEPS; ++kk) {
-      if (head < G) {
-        const uint32_t* qp = reinterpret_cast<const uint32_t*>(Qg + static_cast<int64_t>(head) * D + kk * 16 + 2 * c);
-        qf[nt][kk][0] = __ldg(qp);
-        qf[nt][kk][1] = __ldg(qp + 4);
-      } else {
-        qf[nt][kk][0] = 0u;
-        qf[nt][kk][1] = 0u;
-      }
-    }
-  }
+  load_q_frags<D, NTILE>(a.Q, hq0, G, qf);
   if (T < 0 || T > a.T_cap) {
     if (split == 0 && threadIdx.x == 0) flag_error(a.status, DEVFLAG_BAD_SEQ_LEN);
     T = T < 0 ? 0 : a.T_cap;
@@ -291,233 +125,71 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
     __syncthreads();
   }
 
-  const float scale_log2 = a.sm_scale * kLog2e;
-  float m_run[NTILE][2], l_run[NTILE][2];
-  float acc[KSTEPS][NTILE][4];
-#pragma unroll
-  for (int nt = 0; nt < NTILE; ++nt) {
-    m_run[nt][0] = m_run[nt][1] = -INFINITY;
-    l_run[nt][0] = l_run[nt][1] = 0.f;
-#pragma unroll
-    for (int mt = 0; mt < KSTEPS; ++mt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-  }
-
-  const __nv_bfloat16* Kb = static_cast<const __nv_bfloat16*>(a.K) + b * a.ks[0] + h * a.ks[1];
-  const __nv_bfloat16* Vb = static_cast<const __nv_bfloat16*>(a.V) + b * a.vs[0] + h * a.vs[1];
-  const int nsub = (my_len + kSub - 1) / kSub;
-  const int my_count = (nsub > warp) ? (nsub - warp + kAttnWarps - 1) / kAttnWarps : 0;
-
-  auto token_at = [&](int j) -> int64_t {
-    if (j >= my_len) return -1;
-    return DENSE ? (win_start + my_lo + j) : static_cast<int64_t>(tok_s[j]);
-  };
-  auto issue = [&](int i) {  // i-th subtile of this warp into stage i % STAGES
-    const int sub = warp + i * kAttnWarps;
-    unsigned char* kbuf = ring + (i % STAGES) * Cfg::STAGE_BYTES;
-    unsigned char* vbuf = kbuf + Cfg::SUB_BYTES;
-#pragma unroll
-    for (int q = 0; q < (kSub * CPR) / 32; ++q) {
-      const int cid = lane + q * 32;
-      const int tin = cid / CPR, ch = cid % CPR;
-      const int64_t t = token_at(sub * kSub + tin);
-      const uint32_t nbytes = (t >= 0) ? 16u : 0u;
-      const int64_t tt = (t >= 0) ? t : 0;
-      const int soff = (tin * CPR + (ch ^ (tin & 7))) * 16;
-      cp_async16(kbuf + soff, Kb + tt * a.ks[2] + ch * 8, nbytes);
-      cp_async16(vbuf + soff, Vb + tt * a.vs[2] + ch * 8, nbytes);
-    }
-  };
-
-#pragma unroll
-  for (int s = 0; s < STAGES - 1; ++s) {
-    if (s < my_count) issue(s);
-    cp_async_commit();
-  }
-  for (int i = 0; i < my_count; ++i) {
-    if (i + STAGES - 1 < my_count) issue(i + STAGES - 1);
-    cp_async_commit();
-    cp_async_wait<STAGES - 1>();
-    __syncwarp();
-    const int sub = warp + i * kAttnWarps;
-    const unsigned char* kbuf = ring + (i % STAGES) * Cfg::STAGE_BYTES;
-    const unsigned char* vbuf = kbuf + Cfg::SUB_BYTES;
-
-    // ---- S^T = K_sub . Q^T
-    float sacc[NTILE][4];
-#pragma unroll
-    for (int nt = 0; nt < NTILE; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-    {
-      const int tin = (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-      for (int kk = 0; kk < KSTEPS; ++kk) {
-        const int ch = 2 * kk + (lane >> 4);
-        uint32_t af[4];
-        ldmatrix_x4(af, kbuf + (tin * CPR + (ch ^ (tin & 7))) * 16);
-#pragma unroll
-        for (int nt = 0; nt < NTILE; ++nt) mma_bf16_16816(sacc[nt], af, qf[nt][kk][0], qf[nt][kk][1]);
-      }
-    }
-    // ---- online softmax over the 16 tokens of this subtile
-    const bool v0 = token_at(sub * kSub + g) >= 0;
-    const bool v1 = token_at(sub * kSub + g + 8) >= 0;
-    uint32_t bhi[NTILE][2], blo[NTILE][2];
-#pragma unroll
-    for (int nt = 0; nt < NTILE; ++nt) {
-      float x[4];
-      x[0] = v0 ? sacc[nt][0] * scale_log2 : -INFINITY;
-      x[1] = v0 ? sacc[nt][1] * scale_log2 : -INFINITY;
-      x[2] = v1 ? sacc[nt][2] * scale_log2 : -INFINITY;
-      x[3] = v1 ? sacc[nt][3] * scale_log2 : -INFINITY;
-      float p[4];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        float mx = fmaxf(x[e], x[2 + e]);
-        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
-        const float m_new = fmaxf(m_run[nt][e], mx);
-        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = exp2f(m_run[nt][e] - m_use);
-        p[e] = exp2f(x[e] - m_use);
-        p[2 + e] = exp2f(x[2 + e] - m_use);
-        l_run[nt][e] = l_run[nt][e] * alpha + p[e] + p[2 + e];
-        m_run[nt][e] = m_new;
-#pragma unroll
-        for (int mt = 0; mt < KSTEPS; ++mt) {
-          acc[mt][nt][e] *= alpha;
-          acc[mt][nt][2 + e] *= alpha;
-        }
-      }
-      // P^T as B fragments (tokens x heads) via an in-register 8x8 transpose
-      const uint32_t h0 = pack_bf16x2(p[0], p[1]);
-      const uint32_t h1 = pack_bf16x2(p[2], p[3]);
-      const uint32_t l0 = pack_bf16x2(p[0] - bf16_bits_to_float(h0 & 0xFFFFu), p[1] - bf16_bits_to_float(h0 >> 16));
-      const uint32_t l1 = pack_bf16x2(p[2] - bf16_bits_to_float(h1 & 0xFFFFu), p[3] - bf16_bits_to_float(h1 >> 16));
-      bhi[nt][0] = movmatrix_trans(h0);
-      bhi[nt][1] = movmatrix_trans(h1);
-      blo[nt][0] = movmatrix_trans(l0);
-      blo[nt][1] = movmatrix_trans(l1);
-    }
-    // ---- O^T += V_sub^T . P^T
-    {
-      const int tin = (lane & 7) + (lane >> 4) * 8;
-#pragma unroll
-      for (int mt = 0; mt < KSTEPS; ++mt) {
-        const int ch = 2 * mt + ((lane >> 3) & 1);
-        uint32_t vf[4];
-        ldmatrix_x4_trans(vf, vbuf + (tin * CPR + (ch ^ (tin & 7))) * 16);
-#pragma unroll
-        for (int nt = 0; nt < NTILE; ++nt) {
-          mma_bf16_16816(acc[mt][nt], vf, bhi[nt][0], bhi[nt][1]);
-          mma_bf16_16816(acc[mt][nt], vf, blo[nt][0], blo[nt][1]);
-        }
-      }
-    }
-    __syncwarp();
-  }
-  cp_async_wait<0>();
-
-  // ---- merge the 4 warps' states in shared memory
-#pragma unroll
-  for (int nt = 0; nt < NTILE; ++nt)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      float l = l_run[nt][e];
-      l += __shfl_xor_sync(0xFFFFFFFFu, l, 4);
-      l += __shfl_xor_sync(0xFFFFFFFFu, l, 8);
-      l += __shfl_xor_sync(0xFFFFFFFFu, l, 16);
-      l_run[nt][e] = l;
-    }
-  __syncthreads();  // ring no longer needed
-  float* o_w = reinterpret_cast<float*>(smem_raw);           // [warps][16 heads][D]
-  float* m_w = o_w + kAttnWarps * 16 * D;                     // [warps][16]
-  float* l_w = m_w + kAttnWarps * 16;                         // [warps][16]
-#pragma unroll
-  for (int nt = 0; nt < NTILE; ++nt) {
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int head = nt * 8 + 2 * c + e;
-      if (g == 0) {
-        m_w[warp * 16 + head] = m_run[nt][e];
-        l_w[warp * 16 + head] = l_run[nt][e];
-      }
-#pragma unroll
-      for (int mt = 0; mt < KSTEPS; ++mt) {
-        o_w[(warp * 16 + head) * D + mt * 16 + g] = acc[mt][nt][e];
-        o_w[(warp * 16 + head) * D + mt * 16 + g + 8] = acc[mt][nt][2 + e];
-      }
-    }
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < G * D; i += kAttnThreads) {
-    const int head = i / D, dim = i % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, m_w[w * 16 + head]);
-    float o = 0.f, lse = -INFINITY;
-    if (M != -INFINITY) {
-      float L = 0.f;
-#pragma unroll
-      for (int w = 0; w < kAttnWarps; ++w) {
-        const float sc = exp2f(m_w[w * 16 + head] - M);
-        L += l_w[w * 16 + head] * sc;
-        o += o_w[(w * 16 + head) * D + dim] * sc;
-      }
-      o /= L;
-      lse = (M + log2f(L)) * kLn2;
-    }
-    if (!DENSE) {
-      pbuf[i] = o;
-      if (dim == 0) plse[head] = lse;
-    } else {
-      a.part_o[((hq0 + head) * a.S + split) * D + dim] = o;
-      if (dim == 0) a.part_lse[(hq0 + head) * a.S + split] = lse;
-    }
-  }
-  if (!DENSE) {
-    __syncthreads();
-    cluster_merge<D>(a, hq0, G, pbuf, plse);
-    return;
-  }
-  finish_split<D>(a, row, hq0, G, reinterpret_cast<float*>(smem_raw));
+  attn_core<D, NTILE, DENSE>(a, row, split, b, h, G, hq0, qf, DENSE ? nullptr : tok_s, win_start, my_lo, my_len,
+                             smem_raw);
 }
 
 // ------------------------------------------------------------------ LSE merge
-// O = sum_s w_s o_s / sum_s w_s with w_s = exp(lse_s - max lse); lse = max + log(sum w).
+// O = sum_s w_s o_s with w_s = exp(lse_s - M) / sum_s' exp(lse_s' - M), M = max lse; lse =
+// M + log(sum exp(lse_s - M)).  One CTA per (sequence, query head), one thread per 4 output
+// dims (16-byte loads); warp 0 forms the split weights, then every thread issues the loads
+// of 8 splits at a time before using them.
+constexpr int kMergeBatch = 8;
 __global__ void __launch_bounds__(256) merge_kernel(AttnArgs a) {
   extern __shared__ float wsh[];  // [S]
-  __shared__ float sh_M, sh_L;
+  __shared__ float sh_L;
   const int64_t q = blockIdx.x;   // b * Hq + hq
   const int S = a.S, D = a.dv;
   const float* lse_s = a.part_lse + q * S;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < 32) {
     float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, lse_s[s]);
+    for (int s = threadIdx.x; s < S; s += 32) M = fmaxf(M, lse_s[s]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, off));
     float L = 0.f;
-    for (int s = 0; s < S; ++s) {
+    for (int s = threadIdx.x; s < S; s += 32) {
       const float w = (M == -INFINITY) ? 0.f : expf(lse_s[s] - M);
       wsh[s] = w;
       L += w;
     }
-    sh_M = M;
-    sh_L = L;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, off);
+    if (threadIdx.x == 0) {
+      sh_L = L;
+      if (a.lse) a.lse[q] = (M == -INFINITY) ? -INFINITY : M + logf(L);
+    }
   }
   __syncthreads();
-  const float M = sh_M, L = sh_L;
-  for (int dim = threadIdx.x; dim < D; dim += blockDim.x) {
-    float o = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < S; ++s) o += wsh[s] * a.part_o[(q * S + s) * D + dim];
-      o /= L;
+  const float inv = (sh_L > 0.f) ? 1.f / sh_L : 0.f;
+  const int d4 = threadIdx.x;
+  if (4 * d4 >= D) return;
+  const float4* po = reinterpret_cast<const float4*>(a.part_o + q * S * D) + d4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < S; s0 += kMergeBatch) {
+    float4 v[kMergeBatch];
+#pragma unroll
+    for (int u = 0; u < kMergeBatch; ++u)
+      v[u] = (s0 + u < S) ? __ldcs(po + static_cast<int64_t>(s0 + u) * (D / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < kMergeBatch; ++u) {
+      const float w = (s0 + u < S) ? wsh[s0 + u] : 0.f;
+      acc.x = fmaf(w, v[u].x, acc.x);
+      acc.y = fmaf(w, v[u].y, acc.y);
+      acc.z = fmaf(w, v[u].z, acc.z);
+      acc.w = fmaf(w, v[u].w, acc.w);
     }
-    if (a.out_bf16) static_cast<__nv_bfloat16*>(a.O)[q * D + dim] = __float2bfloat16_rn(o);
-    else static_cast<float*>(a.O)[q * D + dim] = o;
   }
-  if (a.lse && threadIdx.x == 0) a.lse[q] = (M == -INFINITY) ? -INFINITY : M + logf(L);
+  acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+  if (a.out_bf16) {
+    __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.O) + q * D) + 2 * d4;
+    o[0] = __floats2bfloat162_rn(acc.x, acc.y);
+    o[1] = __floats2bfloat162_rn(acc.z, acc.w);
+  } else if ((reinterpret_cast<uintptr_t>(a.O) & 15u) == 0) {
+    reinterpret_cast<float4*>(static_cast<float*>(a.O) + q * D)[d4] = acc;
+  } else {  // the API only guarantees 4-byte alignment of O
+    float* o = static_cast<float*>(a.O) + q * D + 4 * d4;
+    o[0] = acc.x; o[1] = acc.y; o[2] = acc.z; o[3] = acc.w;
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -597,7 +269,8 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_merge(const AttnArgs& a, cudaStream_t s) {
-  merge_kernel<<<a.B * a.Hq, 256, a.S * sizeof(float), s>>>(a);
+  if (a.dv % 4 != 0 || a.dv / 4 > 256) return cudaErrorInvalidValue;
+  merge_kernel<<<a.B * a.Hq, ((a.dv / 4 + 31) / 32) * 32, a.S * sizeof(float), s>>>(a);
   return cudaGetLastError();
 }
 

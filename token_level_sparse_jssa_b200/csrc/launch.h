@@ -119,6 +119,14 @@ struct SelectArgs {
   int32_t* n_sel;    // [B*Hkv]
   int* counters;     // nullable: attention arrival counters zeroed here
   int* status;
+  int keys_words;    // set by the launcher
+  // attention of the selected rows inside the same kernel (GQA, d <= 128): V == nullptr skips it
+  const void* V;
+  int64_t vs[3];
+  float sm_scale;
+  void* O;           // [B, Hq, d]
+  float* lse;        // nullable
+  int out_bf16;
 };
 cudaError_t launch_select(const SelectArgs& a, int num_sms, cudaStream_t s);
 int64_t select_max_candidates();

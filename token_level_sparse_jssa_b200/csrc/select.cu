@@ -23,10 +23,9 @@
 #include <mutex>
 #include <tuple>
 
+#include "attn_core.cuh"
 #include "common.cuh"
 #include "launch.h"
-
-namespace cg = cooperative_groups;
 
 namespace jssa {
 namespace {
@@ -117,7 +116,7 @@ __device__ __forceinline__ void sel_find_digit(const uint32_t* hist, uint32_t kr
   __syncthreads();
 }
 
-template <int R>
+template <int R, int D, int NTILE>
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
   constexpr int CH = kSelStage / (R * 2);          // tokens per stage
   constexpr int V = R / 8;                         // 16-byte vectors per token
@@ -130,16 +129,17 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
   const int C = static_cast<int>(cluster.num_blocks());  // 8 or 16
-  const int own_bins = kSelBins1 / C;
+  const int own_bins = (((kSelBins1 + C - 1) / C) + 1) & ~1;  // even: a packed bin pair has one owner
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const int S = a.stages;
-  const int keys_words = max(a.per, kSelKeysMin / 4);
+  const int keys_words = a.keys_words;
   unsigned char* ring = smem_raw;                                                        // [S][16 KB]
   uint32_t* keys = reinterpret_cast<uint32_t*>(ring + S * kSelStage);                   // [keys_words]
   uint32_t* histp = keys + keys_words;                                                   // [2048] packed 16-bit bins
   uint32_t* own = histp + kSelBins1 / 2;                                                 // [4096 / C] owned row bins
   float* qpart = reinterpret_cast<float*>(own + kSelBins1 / 8);                         // [R] this CTA's share of qs
   double* npart = reinterpret_cast<double*>(qpart + kSelMaxR);                          // [n_new][R] newest-row shares
+  uint16_t* kpn = reinterpret_cast<uint16_t*>(npart + a.n_new * R);                     // [n_new][R] newest Kp rows
   // after the scan the ring holds the row histogram copy and the selection scratch
   uint32_t* ghist = reinterpret_cast<uint32_t*>(ring);                                   // [4096]
   uint32_t* hloc = ghist + kSelBins1;                                                    // [1024]
@@ -156,7 +156,6 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
 
   __shared__ __align__(8) uint64_t full[8], empty[8];
   __shared__ float qs[kSelMaxR];
-  __shared__ uint16_t kpn[kSelMaxNew * kSelMaxR];
   __shared__ uint32_t dig, krem_s, gcnt, gbase;
   __shared__ uint32_t cta_gt[kSelMaxCluster], cta_eq[kSelMaxCluster];
   __shared__ uint32_t warp_gt[kSelWarps], warp_eq[kSelWarps], warp_nc[kSelWarps];
@@ -369,290 +368,356 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
   }
   __syncthreads();
 
+  // the attended list of the row (selection, then the window) and this CTA's share of it
+  // when the attention runs here: positions [crank * L, crank * L + L) of the list
+  const int list_len = k_eff + static_cast<int>(Wc);
+  const int L = (list_len + C - 1) / C;
+  int32_t* tok_list = reinterpret_cast<int32_t*>(own);  // own[] is free once the selection is known
   if (select_all) {  // every candidate is selected (also n == 0)
     for (int j = crank * kSelThreads + tid; j < n; j += C * kSelThreads) out[j] = j;
     cluster.sync();  // no CTA exits while another may still read its shares
-    return;
-  }
-  const bool aborted = aborted_s != 0;
-  if (aborted && tid == kSelConsumers) {  // let every copy still in flight land before the CTA moves on
-    for (int s = 0; s < S; ++s)
-      for (int par = 0; par < 2; ++par) mbar_wait_bounded(&full[s], par, nullptr, 50000000ull);
-  }
-  __syncthreads();
-
-  // ---- the row's first-digit histogram, assembled in the owners' shared memory
-  for (int i = tid; i < kSelBins1 / 2; i += kSelThreads) {
-    const uint32_t v = histp[i];
-    if (v == 0u) continue;
-    const int bin0 = 2 * i;
-    uint32_t* dst = cluster.map_shared_rank(own, bin0 / own_bins) + (bin0 % own_bins);
-    if (v & 0xFFFFu) atomicAdd(dst, v & 0xFFFFu);
-    if (v >> 16) atomicAdd(dst + 1, v >> 16);
-  }
-  cluster.sync();  // the row histogram is complete
-  {
-    constexpr int kPerT = (kSelBins1 + kSelThreads - 1) / kSelThreads;
-    uint32_t v[kPerT];
-#pragma unroll
-    for (int u = 0; u < kPerT; ++u) {  // all remote loads in flight before the first store
-      const int i = tid + u * kSelThreads;
-      v[u] = (i < kSelBins1) ? *(cluster.map_shared_rank(own, i / own_bins) + i % own_bins) : 0u;
-    }
-#pragma unroll
-    for (int u = 0; u < kPerT; ++u) {
-      const int i = tid + u * kSelThreads;
-      if (i < kSelBins1) ghist[i] = v[u];
-    }
-  }
-  __syncthreads();
-  sel_find_digit<kSelBins1>(ghist, static_cast<uint32_t>(k_eff), scan_tmp, &dig, &krem_s);
-  const uint32_t d1 = dig;
-  const uint32_t k1 = krem_s;
-
-  // ---- one pass over the slice: each warp marks its keys above bin d1 ("definites", all
-  // selected) in a bitmap of its range and lists, in index order, its keys inside bin d1
-  // ("candidates").  A lane reads four consecutive keys per step (128 keys per warp step).
-  const int wc = ((len + kSelWarps - 1) / kSelWarps + 31) & ~31;
-  const int w_lo = warp * wc, w_hi = min(len, w_lo + wc);
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  uint32_t* my_mask = masks + warp * kSelMaskWords;
-  uint32_t* my_cands = cands + warp * kSelCapW;
-  uint32_t nd = 0, nca = 0;
-  const bool use_mask = wc <= 32 * kSelMaskWords;  // block-uniform
-  for (int base = w_lo; base < w_hi; base += 128) {
-    const int i0 = base + 4 * lane;
-    const uint4 kv = (i0 < w_hi) ? *reinterpret_cast<const uint4*>(keys + i0) : make_uint4(0u, 0u, 0u, 0u);
-    const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
-    uint32_t dn = 0u, cn = 0u;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const bool valid = i0 + e < w_hi;
-      const uint32_t bin = kk[e] >> 20;
-      dn |= static_cast<uint32_t>(valid && bin > d1) << e;
-      cn |= static_cast<uint32_t>(valid && bin == d1) << e;
-    }
-    nd += __popc(dn);
-    if (use_mask) {  // word (base - w_lo) / 32 + lane / 8 gathers the nibbles of 8 lanes
-      uint32_t wv = dn << (4 * (lane & 7));
-      wv |= __shfl_xor_sync(0xFFFFFFFFu, wv, 1);
-      wv |= __shfl_xor_sync(0xFFFFFFFFu, wv, 2);
-      wv |= __shfl_xor_sync(0xFFFFFFFFu, wv, 4);
-      const int wi = (base - w_lo) / 32 + (lane >> 3);
-      if ((lane & 7) == 0 && wi < kSelMaskWords) my_mask[wi] = wv;
-    }
-    if (__any_sync(0xFFFFFFFFu, cn != 0u)) {
-      const uint32_t m0 = __ballot_sync(0xFFFFFFFFu, cn & 1u), m1 = __ballot_sync(0xFFFFFFFFu, cn & 2u);
-      const uint32_t m2 = __ballot_sync(0xFFFFFFFFu, cn & 4u), m3 = __ballot_sync(0xFFFFFFFFu, cn & 8u);
-      uint32_t p = nca + __popc(m0 & lt_mask) + __popc(m1 & lt_mask) + __popc(m2 & lt_mask) + __popc(m3 & lt_mask);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if ((cn >> e) & 1u) {
-          if (p < kSelCapW) my_cands[p] = static_cast<uint32_t>(i0 + e);
-          ++p;
-        }
-      }
-      nca += __popc(m0) + __popc(m1) + __popc(m2) + __popc(m3);
-    }
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) nd += __shfl_xor_sync(0xFFFFFFFFu, nd, off);
-  const bool cand_list = nca <= kSelCapW;  // warp-uniform: else this warp rescans its range
-  if (lane == 0) warp_nc[warp] = cand_list ? nca : (kSelGather + 1u);
-  __syncthreads();
-
-  // ---- gather the row's in-bin keys into rank 0 (its packed histogram is no longer read)
-  uint32_t* gcnt0 = cluster.map_shared_rank(&gcnt, 0);
-  uint32_t* gbuf0 = cluster.map_shared_rank(gbuf, 0);
-  if (tid == 0) {
-    uint32_t tot = 0;
-    for (int w = 0; w < kSelWarps; ++w) tot += warp_nc[w];
-    tot = min(tot, kSelGather + 1u);
-    gbase = (tot > 0) ? atomicAdd(gcnt0, tot) : 0u;
-  }
-  __syncthreads();
-  {
-    uint32_t off = gbase;
-    for (int w = 0; w < warp; ++w) off += warp_nc[w];
-    if (cand_list && off + nca <= kSelGather)
-      for (int j = lane; j < static_cast<int>(nca); j += 32) gbuf0[off + j] = keys[my_cands[j]];
-  }
-  cluster.sync();  // the row's in-bin keys (or an overflowed count) are in rank 0
-  const uint32_t gtotal = *gcnt0;
-  uint32_t prefix = d1 << 20, mask = 0xFFF00000u, krem = k1;
-  if (gtotal <= kSelGather) {
-    // exact selection among the gathered keys, locally in every CTA: digits 2 and 3
-    if (crank != 0)
-      for (int j = tid; j < static_cast<int>(gtotal); j += kSelThreads) gbuf[j] = gbuf0[j];
-#pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {
-      const int shift = (pass == 0) ? 10 : 0;
-      for (int i = tid; i < kSelBins2; i += kSelThreads) hloc[i] = 0;
-      __syncthreads();
-      for (int j = tid; j < static_cast<int>(gtotal); j += kSelThreads) {
-        const uint32_t key = gbuf[j];
-        if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kSelBins2 - 1)], 1u);
-      }
-      __syncthreads();
-      sel_find_digit<kSelBins2>(hloc, krem, scan_tmp, &dig, &krem_s);
-      prefix |= dig << shift;
-      mask |= static_cast<uint32_t>(kSelBins2 - 1) << shift;
-      krem = krem_s;
-    }
+    if constexpr (D == 0) return;
   } else {
-    // too many in-bin keys for the gather buffer: digits 2 and 3 from cluster-wide
-    // histograms in rank 0 (every CTA takes this branch: gtotal is the same everywhere)
-    uint32_t* totA0 = cluster.map_shared_rank(totA, 0);
-    uint32_t* totB0 = cluster.map_shared_rank(totB, 0);
-    if (crank == 0)
-      for (int i = tid; i < kSelBins2; i += kSelThreads) { totA[i] = 0; totB[i] = 0; }
-    cluster.sync();
-#pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {
-      const int shift = (pass == 0) ? 10 : 0;
-      uint32_t* tot0 = (pass == 0) ? totA0 : totB0;
-      for (int i = tid; i < kSelBins2; i += kSelThreads) hloc[i] = 0;
-      __syncthreads();
-      if (cand_list) {
-        for (int j = lane; j < static_cast<int>(nca); j += 32) {
-          const uint32_t key = keys[my_cands[j]];
-          if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kSelBins2 - 1)], 1u);
-        }
-      } else {
-        for (int i = w_lo + lane; i < w_hi; i += 32) {
-          const uint32_t key = keys[i];
-          if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kSelBins2 - 1)], 1u);
-        }
-      }
-      __syncthreads();
-      for (int i = tid; i < kSelBins2; i += kSelThreads) {
-        const uint32_t v = hloc[i];
-        if (v) atomicAdd(&tot0[i], v);
-      }
-      cluster.sync();
-      sel_find_digit<kSelBins2>(tot0, krem, scan_tmp, &dig, &krem_s);
-      prefix |= dig << shift;
-      mask |= static_cast<uint32_t>(kSelBins2 - 1) << shift;
-      krem = krem_s;
+    const bool aborted = aborted_s != 0;
+    if (aborted && tid == kSelConsumers) {  // let every copy still in flight land before the CTA moves on
+      for (int s = 0; s < S; ++s)
+        for (int par = 0; par < 2; ++par) mbar_wait_bounded(&full[s], par, nullptr, 50000000ull);
     }
-  }
-  const uint32_t kstar = prefix;  // the k-th largest key
-  const uint32_t need = krem;     // keys equal to kstar to take, lowest index first
+    __syncthreads();
 
-  // ---- per-warp counts of keys > kstar and == kstar, published to every CTA
-  {
-    uint32_t ngt = nd, neq = 0;
-    if (cand_list) {
-      for (int j0 = 0; j0 < static_cast<int>(nca); j0 += 32) {
-        const int j = j0 + lane;
-        const uint32_t key = (j < static_cast<int>(nca)) ? keys[my_cands[j]] : 0u;
-        ngt += __popc(__ballot_sync(0xFFFFFFFFu, j < static_cast<int>(nca) && key > kstar));
-        neq += __popc(__ballot_sync(0xFFFFFFFFu, j < static_cast<int>(nca) && key == kstar));
+    // ---- the row's first-digit histogram, assembled in the owners' shared memory
+    for (int i = tid; i < kSelBins1 / 2; i += kSelThreads) {
+      const uint32_t v = histp[i];
+      if (v == 0u) continue;
+      const int bin0 = 2 * i;
+      uint32_t* dst = cluster.map_shared_rank(own, bin0 / own_bins) + (bin0 % own_bins);
+      if (v & 0xFFFFu) atomicAdd(dst, v & 0xFFFFu);
+      if (v >> 16) atomicAdd(dst + 1, v >> 16);
+    }
+    cluster.sync();  // the row histogram is complete
+    {
+      constexpr int kPerT = (kSelBins1 + kSelThreads - 1) / kSelThreads;
+      uint32_t v[kPerT];
+#pragma unroll
+      for (int u = 0; u < kPerT; ++u) {  // all remote loads in flight before the first store
+        const int i = tid + u * kSelThreads;
+        v[u] = (i < kSelBins1) ? *(cluster.map_shared_rank(own, i / own_bins) + i % own_bins) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kPerT; ++u) {
+        const int i = tid + u * kSelThreads;
+        if (i < kSelBins1) ghist[i] = v[u];
+      }
+    }
+    __syncthreads();
+    sel_find_digit<kSelBins1>(ghist, static_cast<uint32_t>(k_eff), scan_tmp, &dig, &krem_s);
+    const uint32_t d1 = dig;
+    const uint32_t k1 = krem_s;
+
+    // ---- one pass over the slice: each warp marks its keys above bin d1 ("definites", all
+    // selected) in a bitmap of its range and lists, in index order, its keys inside bin d1
+    // ("candidates").  A lane reads four consecutive keys per step (128 keys per warp step).
+    const int wc = ((len + kSelWarps - 1) / kSelWarps + 31) & ~31;
+    const int w_lo = warp * wc, w_hi = min(len, w_lo + wc);
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    uint32_t* my_mask = masks + warp * kSelMaskWords;
+    uint32_t* my_cands = cands + warp * kSelCapW;
+    uint32_t nd = 0, nca = 0;
+    const bool use_mask = wc <= 32 * kSelMaskWords;  // block-uniform
+    {
+      for (int base = w_lo; base < w_hi; base += 128) {
+        const int i0 = base + 4 * lane;
+        const uint4 kv = (i0 < w_hi) ? *reinterpret_cast<const uint4*>(keys + i0) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
+        uint32_t dn = 0u, cn = 0u;
+    #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const bool valid = i0 + e < w_hi;
+          const uint32_t bin = kk[e] >> 20;
+          dn |= static_cast<uint32_t>(valid && bin > d1) << e;
+          cn |= static_cast<uint32_t>(valid && bin == d1) << e;
+        }
+        nd += __popc(dn);
+        if (use_mask) {  // word (base - w_lo) / 32 + lane / 8 gathers the nibbles of 8 lanes
+          uint32_t wv = dn << (4 * (lane & 7));
+          wv |= __shfl_xor_sync(0xFFFFFFFFu, wv, 1);
+          wv |= __shfl_xor_sync(0xFFFFFFFFu, wv, 2);
+          wv |= __shfl_xor_sync(0xFFFFFFFFu, wv, 4);
+          const int wi = (base - w_lo) / 32 + (lane >> 3);
+          if ((lane & 7) == 0 && wi < kSelMaskWords) my_mask[wi] = wv;
+        }
+        if (__any_sync(0xFFFFFFFFu, cn != 0u)) {
+          const uint32_t m0 = __ballot_sync(0xFFFFFFFFu, cn & 1u), m1 = __ballot_sync(0xFFFFFFFFu, cn & 2u);
+          const uint32_t m2 = __ballot_sync(0xFFFFFFFFu, cn & 4u), m3 = __ballot_sync(0xFFFFFFFFu, cn & 8u);
+          uint32_t p = nca + __popc(m0 & lt_mask) + __popc(m1 & lt_mask) + __popc(m2 & lt_mask) + __popc(m3 & lt_mask);
+    #pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if ((cn >> e) & 1u) {
+              if (p < kSelCapW) my_cands[p] = static_cast<uint32_t>(i0 + e);
+              ++p;
+            }
+          }
+          nca += __popc(m0) + __popc(m1) + __popc(m2) + __popc(m3);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) nd += __shfl_xor_sync(0xFFFFFFFFu, nd, off);
+    }
+    const bool cand_list = nca <= kSelCapW;  // warp-uniform: else this warp rescans its range
+    if (lane == 0) warp_nc[warp] = cand_list ? nca : (kSelGather + 1u);
+    __syncthreads();
+
+    // ---- gather the row's in-bin keys into rank 0 (its packed histogram is no longer read)
+    uint32_t* gcnt0 = cluster.map_shared_rank(&gcnt, 0);
+    uint32_t* gbuf0 = cluster.map_shared_rank(gbuf, 0);
+    if (tid == 0) {
+      uint32_t tot = 0;
+      for (int w = 0; w < kSelWarps; ++w) tot += warp_nc[w];
+      tot = min(tot, kSelGather + 1u);
+      gbase = (tot > 0) ? atomicAdd(gcnt0, tot) : 0u;
+    }
+    __syncthreads();
+    {
+      uint32_t off = gbase;
+      for (int w = 0; w < warp; ++w) off += warp_nc[w];
+      if (cand_list && off + nca <= kSelGather)
+        for (int j = lane; j < static_cast<int>(nca); j += 32) gbuf0[off + j] = keys[my_cands[j]];
+    }
+    cluster.sync();  // the row's in-bin keys (or an overflowed count) are in rank 0
+    const uint32_t gtotal = *gcnt0;
+    uint32_t prefix = d1 << 20, mask = 0xFFF00000u, krem = k1;
+    if (gtotal <= kSelGather) {
+      // exact selection among the gathered keys, locally in every CTA: digits 2 and 3
+      if (crank != 0)
+        for (int j = tid; j < static_cast<int>(gtotal); j += kSelThreads) gbuf[j] = gbuf0[j];
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        const int shift = (pass == 0) ? 10 : 0;
+        for (int i = tid; i < kSelBins2; i += kSelThreads) hloc[i] = 0;
+        __syncthreads();
+        for (int j = tid; j < static_cast<int>(gtotal); j += kSelThreads) {
+          const uint32_t key = gbuf[j];
+          if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kSelBins2 - 1)], 1u);
+        }
+        __syncthreads();
+        sel_find_digit<kSelBins2>(hloc, krem, scan_tmp, &dig, &krem_s);
+        prefix |= dig << shift;
+        mask |= static_cast<uint32_t>(kSelBins2 - 1) << shift;
+        krem = krem_s;
       }
     } else {
-      for (int base = w_lo; base < w_hi; base += 32) {
-        const int i = base + lane;
-        const uint32_t key = (i < w_hi) ? keys[i] : 0u;
-        ngt += __popc(__ballot_sync(0xFFFFFFFFu, i < w_hi && key > kstar && (key >> 20) == d1));
-        neq += __popc(__ballot_sync(0xFFFFFFFFu, i < w_hi && key == kstar));
+      // too many in-bin keys for the gather buffer: digits 2 and 3 from cluster-wide
+      // histograms in rank 0 (every CTA takes this branch: gtotal is the same everywhere)
+      uint32_t* totA0 = cluster.map_shared_rank(totA, 0);
+      uint32_t* totB0 = cluster.map_shared_rank(totB, 0);
+      if (crank == 0)
+        for (int i = tid; i < kSelBins2; i += kSelThreads) { totA[i] = 0; totB[i] = 0; }
+      cluster.sync();
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        const int shift = (pass == 0) ? 10 : 0;
+        uint32_t* tot0 = (pass == 0) ? totA0 : totB0;
+        for (int i = tid; i < kSelBins2; i += kSelThreads) hloc[i] = 0;
+        __syncthreads();
+        if (cand_list) {
+          for (int j = lane; j < static_cast<int>(nca); j += 32) {
+            const uint32_t key = keys[my_cands[j]];
+            if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kSelBins2 - 1)], 1u);
+          }
+        } else {
+          for (int i = w_lo + lane; i < w_hi; i += 32) {
+            const uint32_t key = keys[i];
+            if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (kSelBins2 - 1)], 1u);
+          }
+        }
+        __syncthreads();
+        for (int i = tid; i < kSelBins2; i += kSelThreads) {
+          const uint32_t v = hloc[i];
+          if (v) atomicAdd(&tot0[i], v);
+        }
+        cluster.sync();
+        sel_find_digit<kSelBins2>(tot0, krem, scan_tmp, &dig, &krem_s);
+        prefix |= dig << shift;
+        mask |= static_cast<uint32_t>(kSelBins2 - 1) << shift;
+        krem = krem_s;
       }
     }
-    if (lane == 0) { warp_gt[warp] = ngt; warp_eq[warp] = neq; }
-  }
-  __syncthreads();
-  if (tid < C) {
-    uint32_t g = 0, e = 0;
-    for (int w = 0; w < kSelWarps; ++w) { g += warp_gt[w]; e += warp_eq[w]; }
-    *cluster.map_shared_rank(&cta_gt[crank], tid) = g;
-    *cluster.map_shared_rank(&cta_eq[crank], tid) = e;
-  }
-  cluster.sync();  // last access to another CTA's shared memory
-  if (aborted) {   // a wait gave up (flagged): report an empty selection
-    for (int j = crank * kSelThreads + tid; j < k_eff; j += C * kSelThreads) out[j] = -1;
-    return;
-  }
+    const uint32_t kstar = prefix;  // the k-th largest key
+    const uint32_t need = krem;     // keys equal to kstar to take, lowest index first
 
-  // ---- output positions: CTAs in rank order, warps in index order
-  uint32_t base_out = 0, eq_before = 0;
-  for (int c = 0; c < crank; ++c) {
-    const uint32_t qv = (need > eq_before) ? min(cta_eq[c], need - eq_before) : 0u;
-    base_out += cta_gt[c] + qv;
-    eq_before += cta_eq[c];
-  }
-  const uint32_t quota = (need > eq_before) ? min(cta_eq[crank], need - eq_before) : 0u;
-  uint32_t pos = base_out, eq_rank = 0;
-  for (int w = 0; w < warp; ++w) {
-    const uint32_t qv = (quota > eq_rank) ? min(warp_eq[w], quota - eq_rank) : 0u;
-    pos += warp_gt[w] + qv;
-    eq_rank += warp_eq[w];
-  }
-  const uint32_t wquota = (quota > eq_rank) ? min(warp_eq[warp], quota - eq_rank) : 0u;
-  const int words = (w_hi > w_lo) ? (w_hi - w_lo + 31) / 32 : 0;  // bitmap words written by the scan
-  if (cand_list && use_mask) {
-    // add the selected candidates to the bitmap of definites, then emit the range in order
-    uint32_t* m = my_mask;
-    uint32_t eq_run = 0;
-    for (int j0 = 0; j0 < static_cast<int>(nca); j0 += 32) {
-      const int j = j0 + lane;
-      const uint32_t i = (j < static_cast<int>(nca)) ? my_cands[j] : 0u;
-      const uint32_t key = (j < static_cast<int>(nca)) ? keys[i] : 0u;
-      const bool gt = j < static_cast<int>(nca) && key > kstar;
-      const bool eq = j < static_cast<int>(nca) && key == kstar;
-      const uint32_t eq_m = __ballot_sync(0xFFFFFFFFu, eq);
-      if (gt || (eq && (eq_run + __popc(eq_m & lt_mask)) < wquota)) {
-        const uint32_t o = i - static_cast<uint32_t>(w_lo);
-        atomicOr(&m[o >> 5], 1u << (o & 31));
+    // ---- per-warp counts of keys > kstar and == kstar, published to every CTA
+    {
+      uint32_t ngt = nd, neq = 0;
+      if (cand_list) {
+        for (int j0 = 0; j0 < static_cast<int>(nca); j0 += 32) {
+          const int j = j0 + lane;
+          const uint32_t key = (j < static_cast<int>(nca)) ? keys[my_cands[j]] : 0u;
+          ngt += __popc(__ballot_sync(0xFFFFFFFFu, j < static_cast<int>(nca) && key > kstar));
+          neq += __popc(__ballot_sync(0xFFFFFFFFu, j < static_cast<int>(nca) && key == kstar));
+        }
+      } else {
+        for (int base = w_lo; base < w_hi; base += 32) {
+          const int i = base + lane;
+          const uint32_t key = (i < w_hi) ? keys[i] : 0u;
+          ngt += __popc(__ballot_sync(0xFFFFFFFFu, i < w_hi && key > kstar && (key >> 20) == d1));
+          neq += __popc(__ballot_sync(0xFFFFFFFFu, i < w_hi && key == kstar));
+        }
       }
-      eq_run += __popc(eq_m);
+      if (lane == 0) { warp_gt[warp] = ngt; warp_eq[warp] = neq; }
     }
-    __syncwarp();
-    const uint32_t w0 = (lane < words) ? m[lane] : 0u;
-    const uint32_t w1 = (lane + 32 < words) ? m[lane + 32] : 0u;
-    const uint32_t c0 = __popc(w0), c1 = __popc(w1);
-    uint32_t x0 = c0, x1 = c1;
+    __syncthreads();
+    if (tid < C) {
+      uint32_t g = 0, e = 0;
+      for (int w = 0; w < kSelWarps; ++w) { g += warp_gt[w]; e += warp_eq[w]; }
+      *cluster.map_shared_rank(&cta_gt[crank], tid) = g;
+      *cluster.map_shared_rank(&cta_eq[crank], tid) = e;
+    }
+    cluster.sync();  // the counts are everywhere; other CTAs' memory is no longer read
+    if (aborted) {   // a wait gave up (flagged): report an empty selection
+      for (int j = crank * kSelThreads + tid; j < k_eff; j += C * kSelThreads) out[j] = -1;
+      if constexpr (D > 0) for (int j = tid; j < L; j += kSelThreads) tok_list[j] = -1;
+    } else {
+
+      // ---- output positions: CTAs in rank order, warps in index order
+      uint32_t base_out = 0, eq_before = 0;
+      for (int c = 0; c < crank; ++c) {
+        const uint32_t qv = (need > eq_before) ? min(cta_eq[c], need - eq_before) : 0u;
+        base_out += cta_gt[c] + qv;
+        eq_before += cta_eq[c];
+      }
+      const uint32_t quota = (need > eq_before) ? min(cta_eq[crank], need - eq_before) : 0u;
+      uint32_t pos = base_out, eq_rank = 0;
+      for (int w = 0; w < warp; ++w) {
+        const uint32_t qv = (quota > eq_rank) ? min(warp_eq[w], quota - eq_rank) : 0u;
+        pos += warp_gt[w] + qv;
+        eq_rank += warp_eq[w];
+      }
+      const uint32_t wquota = (quota > eq_rank) ? min(warp_eq[warp], quota - eq_rank) : 0u;
+      const int words = (w_hi > w_lo) ? (w_hi - w_lo + 31) / 32 : 0;  // bitmap words written by the scan
+      if (cand_list && use_mask) {
+        // add the selected candidates to the bitmap of definites, then emit the range in order
+        uint32_t* m = my_mask;
+        for (int j0 = 0; j0 < static_cast<int>(nca); j0 += 32) {
+          const int j = j0 + lane;
+          const uint32_t i = (j < static_cast<int>(nca)) ? my_cands[j] : 0u;
+          const uint32_t key = (j < static_cast<int>(nca)) ? keys[i] : 0u;
+          const bool gt = j < static_cast<int>(nca) && key > kstar;
+          bool take = gt;
+          if (j < static_cast<int>(nca) && key == kstar) {
+            // rank among this warp's keys equal to kstar by position (the list may be unordered)
+            uint32_t rank = 0;
+            for (int jj = 0; jj < static_cast<int>(nca); ++jj) {
+              const uint32_t o2 = my_cands[jj];
+              rank += (o2 < i && keys[o2] == kstar) ? 1u : 0u;
+            }
+            take = rank < wquota;
+          }
+          if (take) {
+            const uint32_t o = i - static_cast<uint32_t>(w_lo);
+            atomicOr(&m[o >> 5], 1u << (o & 31));
+          }
+        }
+        __syncwarp();
+        const uint32_t w0 = (lane < words) ? m[lane] : 0u;
+        const uint32_t w1 = (lane + 32 < words) ? m[lane + 32] : 0u;
+        const uint32_t c0 = __popc(w0), c1 = __popc(w1);
+        uint32_t x0 = c0, x1 = c1;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t y0 = __shfl_up_sync(0xFFFFFFFFu, x0, off);
-      const uint32_t y1 = __shfl_up_sync(0xFFFFFFFFu, x1, off);
-      if (lane >= off) { x0 += y0; x1 += y1; }
-    }
-    const uint32_t tot0 = __shfl_sync(0xFFFFFFFFu, x0, 31);
-    uint32_t p0 = pos + x0 - c0, p1 = pos + tot0 + x1 - c1;
-    const int gb = lo + w_lo;
-    for (uint32_t v = w0; v; v &= v - 1) {
-      if (p0 < static_cast<uint32_t>(k_eff)) out[p0] = gb + lane * 32 + (__ffs(v) - 1);
-      else flag_error(a.status, DEVFLAG_BAD_INDEX);  // unreachable when the counts are consistent
-      ++p0;
-    }
-    for (uint32_t v = w1; v; v &= v - 1) {
-      if (p1 < static_cast<uint32_t>(k_eff)) out[p1] = gb + (lane + 32) * 32 + (__ffs(v) - 1);
-      else flag_error(a.status, DEVFLAG_BAD_INDEX);
-      ++p1;
-    }
-  } else {
-    // long lists: rescan this warp's range and compact with ballots
-    uint32_t eq_run = 0;
-    for (int base = w_lo; base < w_hi; base += 32) {
-      const int i = base + lane;
-      const uint32_t key = (i < w_hi) ? keys[i] : 0u;
-      const bool gt = i < w_hi && key > kstar;
-      const bool eq = i < w_hi && key == kstar;
-      const uint32_t eq_m = __ballot_sync(0xFFFFFFFFu, eq);
-      const bool sel = gt || (eq && (eq_run + __popc(eq_m & lt_mask)) < wquota);
-      const uint32_t sel_m = __ballot_sync(0xFFFFFFFFu, sel);
-      if (sel) {
-        const uint32_t p = pos + __popc(sel_m & lt_mask);
-        if (p < static_cast<uint32_t>(k_eff)) out[p] = lo + i;
-        else flag_error(a.status, DEVFLAG_BAD_INDEX);
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t y0 = __shfl_up_sync(0xFFFFFFFFu, x0, off);
+          const uint32_t y1 = __shfl_up_sync(0xFFFFFFFFu, x1, off);
+          if (lane >= off) { x0 += y0; x1 += y1; }
+        }
+        const uint32_t tot0 = __shfl_sync(0xFFFFFFFFu, x0, 31);
+        uint32_t p0 = pos + x0 - c0, p1 = pos + tot0 + x1 - c1;
+        const int gb = lo + w_lo;
+        for (uint32_t v = w0; v; v &= v - 1) {
+          if (p0 < static_cast<uint32_t>(k_eff)) {
+            const int t = gb + lane * 32 + (__ffs(v) - 1);
+            out[p0] = t;
+            if constexpr (D > 0) *(cluster.map_shared_rank(tok_list, p0 / L) + p0 % L) = t;
+          } else {
+            flag_error(a.status, DEVFLAG_BAD_INDEX);  // unreachable when the counts are consistent
+          }
+          ++p0;
+        }
+        for (uint32_t v = w1; v; v &= v - 1) {
+          if (p1 < static_cast<uint32_t>(k_eff)) {
+            const int t = gb + (lane + 32) * 32 + (__ffs(v) - 1);
+            out[p1] = t;
+            if constexpr (D > 0) *(cluster.map_shared_rank(tok_list, p1 / L) + p1 % L) = t;
+          } else {
+            flag_error(a.status, DEVFLAG_BAD_INDEX);
+          }
+          ++p1;
+        }
+      } else {
+        // long lists: rescan this warp's range and compact with ballots
+        uint32_t eq_run = 0;
+        for (int base = w_lo; base < w_hi; base += 32) {
+          const int i = base + lane;
+          const uint32_t key = (i < w_hi) ? keys[i] : 0u;
+          const bool gt = i < w_hi && key > kstar;
+          const bool eq = i < w_hi && key == kstar;
+          const uint32_t eq_m = __ballot_sync(0xFFFFFFFFu, eq);
+          const bool sel = gt || (eq && (eq_run + __popc(eq_m & lt_mask)) < wquota);
+          const uint32_t sel_m = __ballot_sync(0xFFFFFFFFu, sel);
+          if (sel) {
+            const uint32_t p = pos + __popc(sel_m & lt_mask);
+            if (p < static_cast<uint32_t>(k_eff)) {
+              out[p] = lo + i;
+              if constexpr (D > 0) *(cluster.map_shared_rank(tok_list, p / L) + p % L) = lo + i;
+            } else {
+              flag_error(a.status, DEVFLAG_BAD_INDEX);
+            }
+          }
+          pos += __popc(sel_m);
+          eq_run += __popc(eq_m);
+        }
       }
-      pos += __popc(sel_m);
-      eq_run += __popc(eq_m);
+    }  // selection written
+  }  // not every candidate selected
+
+  if constexpr (D > 0) {
+    // ---- attention of the row's list: this CTA takes positions [my_lo, my_lo + my_len); the
+    // selected ones were scattered into tok_list above, the window ones are filled here
+    const int my_lo = crank * L;
+    const int my_len = max(0, min(list_len, my_lo + L) - my_lo);
+    const int64_t win_start = T - Wc;
+    for (int j = tid; j < my_len; j += kSelThreads) {
+      const int p = my_lo + j;
+      if (select_all) tok_list[j] = p;  // selection [0, n) then window [n, T): token p
+      else if (p >= k_eff) tok_list[j] = static_cast<int32_t>(win_start + (p - k_eff));
     }
+    const int64_t hq0 = static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(h) * G;
+    uint32_t qf[NTILE][D / 16][2];
+    load_q_frags<D, NTILE>(a.Q, hq0, G, qf);
+    cluster_arrive_release();  // the scattered positions are in place
+    cluster_wait_acquire();
+    AttnArgs at{};
+    at.K = a.K;
+    at.V = a.V;
+    for (int i = 0; i < 3; ++i) { at.ks[i] = a.ks[i]; at.vs[i] = a.vs[i]; }
+    at.B = a.B;
+    at.Hq = a.Hq;
+    at.Hkv = a.Hkv;
+    at.dk = D;
+    at.dv = D;
+    at.T_cap = a.T_cap;
+    at.window = a.window;
+    at.sm_scale = a.sm_scale;
+    at.S = C;
+    at.split_len = L;
+    at.O = a.O;
+    at.lse = a.lse;
+    at.out_bf16 = a.out_bf16;
+    at.status = a.status;
+    attn_core<D, NTILE, false>(at, row, crank, b, h, G, hq0, qf, tok_list, win_start, my_lo, my_len, smem_raw);
   }
 }
 
 constexpr int kSelMaxSlice = 16384;    // keys per CTA kept in shared memory
-constexpr int kSelStaticBytes = 3072;  // static shared memory of the kernel, rounded up
+constexpr int kSelStaticBytes = 2048;  // static shared memory of the kernel, rounded up
 
 // Number of clusters of this shape that can be resident at once (cached per device).
 template <typename Kernel>
@@ -685,9 +750,9 @@ int active_clusters(Kernel kernel, int C, size_t smem, int rows) {
   return n;
 }
 
-template <int R>
+template <int R, int D, int NTILE>
 cudaError_t launch_select_r(SelectArgs a, int num_sms, cudaStream_t s) {
-  auto kernel = select_kernel<R>;
+  auto kernel = select_kernel<R, D, NTILE>;
   static int done[64] = {0};
   cudaError_t e = set_smem_limit_once(kernel, 227u * 1024u - kSelStaticBytes, done);
   if (e != cudaSuccess) return e;
@@ -695,42 +760,68 @@ cudaError_t launch_select_r(SelectArgs a, int num_sms, cudaStream_t s) {
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!np_done[dev]) {  // 16-CTA clusters are a non-portable size
+  if (!np_done[dev]) {  // clusters above 8 CTAs are non-portable sizes
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess)
       np_done[dev] = 1;
     else
       np_done[dev] = -1, (void)cudaGetLastError();
   }
   const int rows = a.B * a.Hkv;
-  // Cluster size and ring depth: 16 CTAs per row when 8 per row would leave SMs idle and all
-  // rows' 16-CTA clusters can be resident at once, else 8; then the deepest ring that keeps
-  // every row's cluster resident (a second wave of clusters would double the scan time).
+  // Cluster size and ring depth: the largest cluster (8..16 CTAs per row) whose clusters are
+  // all resident at once when 8 CTAs per row would leave SMs idle, 8 otherwise; then the
+  // deepest ring that keeps every row's cluster resident (a second wave of clusters would
+  // double the scan time).  With the attention inside, the ring and keys areas also hold the
+  // attention's buffers, and each CTA's share of the attended list must fit its token list.
   int C = 8, stages = 2;
   size_t fixed = 0;
-  for (int pass = 0; pass < 2; ++pass) {
-    const int c_try = (pass == 0) ? 16 : 8;
-    if (c_try == 16 && (np_done[dev] <= 0 || static_cast<int64_t>(rows) * 8 >= num_sms)) continue;
+  const int64_t list_max = a.k + min64(max64(a.window, 0), a.T_cap);
+  const int c_max = (np_done[dev] > 0 && static_cast<int64_t>(rows) * 8 < num_sms) ? kSelMaxCluster : 8;
+  for (int c_try = c_max; c_try >= 8; --c_try) {
     const int per = static_cast<int>(ceil_div(ceil_div(a.T_cap, c_try), 32) * 32);
     if (per > kSelMaxSlice) continue;
-    const size_t fx = static_cast<size_t>(max(per, kSelKeysMin / 4)) * 4 + (kSelBins1 / 2) * 4 +
-                      (kSelBins1 / 8) * 4 + kSelMaxR * 4 + static_cast<size_t>(a.n_new) * R * 8;
-    int st_ok = 0;
+    if (D > 0 && ceil_div(list_max, c_try) > kSelBins1 / 8) continue;  // token list lives in own[]
+    const size_t tail = (kSelBins1 / 2) * 4 + (kSelBins1 / 8) * 4 + kSelMaxR * 4 +
+                        static_cast<size_t>(a.n_new) * R * 8 + static_cast<size_t>((a.n_new * R + 7) & ~7) * 2;
+    int st_ok = 0, kw_ok = 0;
     for (int st = 8; st >= 2; --st) {
-      const size_t smem = static_cast<size_t>(st) * kSelStage + fx;
+      int kw = max(per, kSelKeysMin / 4);
+      if (D > 0) {
+        const int need = attn_main_bytes<D>() - st * kSelStage;
+        if (need > kw * 4) kw = (need + 3) / 4;
+      }
+      const size_t smem = static_cast<size_t>(st) * kSelStage + static_cast<size_t>(kw) * 4 + tail;
       if (smem + kSelStaticBytes > 227u * 1024u) continue;
-      if (active_clusters(kernel, c_try, smem, rows) >= rows) { st_ok = st; break; }
+      if (active_clusters(kernel, c_try, smem, rows) >= rows) { st_ok = st; kw_ok = kw; break; }
     }
-    if (st_ok == 0 && c_try == 16) continue;  // 16-CTA clusters would need two waves
+    if (st_ok == 0 && c_try > 8) continue;  // these clusters would need a second wave
+    if (st_ok == 0) {
+      kw_ok = max(per, kSelKeysMin / 4);
+      if (D > 0) kw_ok = max(kw_ok, (attn_main_bytes<D>() - 2 * kSelStage + 3) / 4);
+    }
     C = c_try;
     stages = st_ok > 0 ? st_ok : 2;
-    fixed = fx;
+    fixed = static_cast<size_t>(kw_ok) * 4 + tail;
     a.per = per;
+    a.keys_words = kw_ok;
     break;
   }
-  if (fixed == 0) return cudaErrorInvalidValue;
+  if (fixed == 0) return D > 0 ? cudaErrorNotSupported : cudaErrorInvalidValue;
   a.stages = stages;
   const size_t smem = static_cast<size_t>(stages) * kSelStage + fixed;
+  if (smem + kSelStaticBytes > 227u * 1024u) return D > 0 ? cudaErrorNotSupported : cudaErrorInvalidValue;
   return launch_ex(kernel, dim3(C, rows), dim3(kSelThreads), smem, s, C, a);
+}
+
+template <int R>
+cudaError_t launch_select_rd(const SelectArgs& a, int num_sms, cudaStream_t s) {
+  if (a.V == nullptr) return launch_select_r<R, 0, 1>(a, num_sms, s);
+  const int G = a.Hq / a.Hkv;
+  if (G > 16) return cudaErrorNotSupported;
+  switch (a.d) {
+    case 64: return G <= 8 ? launch_select_r<R, 64, 1>(a, num_sms, s) : launch_select_r<R, 64, 2>(a, num_sms, s);
+    case 128: return G <= 8 ? launch_select_r<R, 128, 1>(a, num_sms, s) : launch_select_r<R, 128, 2>(a, num_sms, s);
+    default: return cudaErrorNotSupported;
+  }
 }
 
 }  // namespace
@@ -742,10 +833,10 @@ cudaError_t launch_select(const SelectArgs& a, int num_sms, cudaStream_t s) {
   if (a.T_cap > select_max_candidates() || a.n_new > kSelMaxNew || a.n_new < 0) return cudaErrorInvalidValue;
   if (a.d % 8 != 0 || a.d / 8 > 8 * (kSelMaxDn / 8)) return cudaErrorInvalidValue;
   switch (a.r) {
-    case 8: return launch_select_r<8>(a, num_sms, s);
-    case 16: return launch_select_r<16>(a, num_sms, s);
-    case 32: return launch_select_r<32>(a, num_sms, s);
-    case 64: return launch_select_r<64>(a, num_sms, s);
+    case 8: return launch_select_rd<8>(a, num_sms, s);
+    case 16: return launch_select_rd<16>(a, num_sms, s);
+    case 32: return launch_select_rd<32>(a, num_sms, s);
+    case 64: return launch_select_rd<64>(a, num_sms, s);
     default: return cudaErrorInvalidValue;
   }
 }
