@@ -42,6 +42,7 @@ struct AttnCfg {
 template <int D>
 constexpr int attn_main_bytes() { return AttnCfg<D>::MAIN_BYTES; }
 
+
 // Combine the S split partials of query heads [hq0, hq0 + G) into O (and lse):
 // O = sum_s w_s o_s with w_s = exp(lse_s - M) / sum_s' exp(lse_s' - M), M = max lse;
 // lse = M + log(sum exp(lse_s - M)).  Run by the last CTA of a row to finish, on

@@ -38,7 +38,8 @@ constexpr int kSelMaxCluster = 16;                 // 8 (portable) or 16 CTAs pe
 constexpr int kSelBins1 = 4096;                    // digit 1: key bits [31:20]
 constexpr int kSelBins2 = 1024;                    // digits 2 and 3: bits [19:10] and [9:0]
 constexpr int kSelCapW = 64;                       // per-warp capacity of the definite / candidate lists
-constexpr int kSelMaskWords = 64;                  // per-warp output bitmap: ranges of up to 2048 keys
+constexpr int kSelMaskWords = 64;                  // per-warp bitmaps: ranges of up to 2048 keys
+static_assert(((16384 + 8) / 9 + 31) / 32 <= 64, "a slice's warp ranges fit the bitmaps");
 constexpr uint32_t kSelGather = 2048;              // in-bin keys of a row gathered into rank 0
 constexpr int kSelMaxNew = 16;                     // newest rows projected inside the kernel
 constexpr int kSelMaxR = 64;
@@ -145,6 +146,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
   uint32_t* hloc = ghist + kSelBins1;                                                    // [1024]
   uint32_t* masks = hloc + kSelBins2;                                                    // [warps][kSelMaskWords]
   uint32_t* cands = masks + kSelWarps * kSelMaskWords;                                   // [warps][kSelCapW]
+  uint32_t* cmasks = cands + kSelWarps * kSelCapW;                                       // [warps][kSelMaskWords]
   // after the row histogram is assembled the packed histogram holds the gathered keys
   uint32_t* gbuf = histp;                                                                // [kSelGather]
   uint32_t* totA = histp;                                                                // fallback totals
@@ -415,8 +417,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
     const uint32_t k1 = krem_s;
 
     // ---- one pass over the slice: each warp marks its keys above bin d1 ("definites", all
-    // selected) in a bitmap of its range and lists, in index order, its keys inside bin d1
-    // ("candidates").  A lane reads four consecutive keys per step (128 keys per warp step).
+    // selected) in a bitmap of its range and lists its keys inside bin d1 ("candidates", in
+    // any order: ties are later ranked by position).
     const int wc = ((len + kSelWarps - 1) / kSelWarps + 31) & ~31;
     const int w_lo = warp * wc, w_hi = min(len, w_lo + wc);
     const uint32_t lt_mask = (1u << lane) - 1u;
@@ -425,43 +427,46 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
     uint32_t nd = 0, nca = 0;
     const bool use_mask = wc <= 32 * kSelMaskWords;  // block-uniform
     {
+      uint32_t* my_cmask = cmasks + warp * kSelMaskWords;
       for (int base = w_lo; base < w_hi; base += 128) {
-        const int i0 = base + 4 * lane;
-        const uint4 kv = (i0 < w_hi) ? *reinterpret_cast<const uint4*>(keys + i0) : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
-        uint32_t dn = 0u, cn = 0u;
-    #pragma unroll
+        // lane L reads keys base + 32 e + L: the ballots of key-slot e are bitmap words
+        // (base - w_lo) / 32 + e of the definites and of the candidates, in index order
+        uint32_t kk[4], mdef[4], mcan[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) kk[e] = keys[min(base + 32 * e + lane, w_hi - 1)];  // all loads first
+#pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const bool valid = i0 + e < w_hi;
-          const uint32_t bin = kk[e] >> 20;
-          dn |= static_cast<uint32_t>(valid && bin > d1) << e;
-          cn |= static_cast<uint32_t>(valid && bin == d1) << e;
+          const bool ok = base + 32 * e + lane < w_hi;
+          mdef[e] = __ballot_sync(0xFFFFFFFFu, ok && (kk[e] >> 20) > d1);
+          mcan[e] = __ballot_sync(0xFFFFFFFFu, ok && (kk[e] >> 20) == d1);
         }
-        nd += __popc(dn);
-        if (use_mask) {  // word (base - w_lo) / 32 + lane / 8 gathers the nibbles of 8 lanes
-          uint32_t wv = dn << (4 * (lane & 7));
-          wv |= __shfl_xor_sync(0xFFFFFFFFu, wv, 1);
-          wv |= __shfl_xor_sync(0xFFFFFFFFu, wv, 2);
-          wv |= __shfl_xor_sync(0xFFFFFFFFu, wv, 4);
-          const int wi = (base - w_lo) / 32 + (lane >> 3);
-          if ((lane & 7) == 0 && wi < kSelMaskWords) my_mask[wi] = wv;
-        }
-        if (__any_sync(0xFFFFFFFFu, cn != 0u)) {
-          const uint32_t m0 = __ballot_sync(0xFFFFFFFFu, cn & 1u), m1 = __ballot_sync(0xFFFFFFFFu, cn & 2u);
-          const uint32_t m2 = __ballot_sync(0xFFFFFFFFu, cn & 4u), m3 = __ballot_sync(0xFFFFFFFFu, cn & 8u);
-          uint32_t p = nca + __popc(m0 & lt_mask) + __popc(m1 & lt_mask) + __popc(m2 & lt_mask) + __popc(m3 & lt_mask);
-    #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if ((cn >> e) & 1u) {
-              if (p < kSelCapW) my_cands[p] = static_cast<uint32_t>(i0 + e);
-              ++p;
-            }
-          }
-          nca += __popc(m0) + __popc(m1) + __popc(m2) + __popc(m3);
+        nd += __popc(mdef[0]) + __popc(mdef[1]) + __popc(mdef[2]) + __popc(mdef[3]);
+        // one lane stores the step's four words of each bitmap (16-byte aligned: 4 words a step)
+        const int wb = (base - w_lo) / 32;
+        if (use_mask && lane == 0 && wb < kSelMaskWords) {
+          *reinterpret_cast<uint4*>(my_mask + wb) = make_uint4(mdef[0], mdef[1], mdef[2], mdef[3]);
+          *reinterpret_cast<uint4*>(my_cmask + wb) = make_uint4(mcan[0], mcan[1], mcan[2], mcan[3]);
         }
       }
+      __syncwarp();
+      // the candidates' positions from their bitmap (lane L: words L and L + 32)
+      const int nwords = (w_hi > w_lo) ? (w_hi - w_lo + 31) / 32 : 0;
+      const uint32_t cw0 = (use_mask && lane < nwords) ? my_cmask[lane] : 0u;
+      const uint32_t cw1 = (use_mask && lane + 32 < nwords) ? my_cmask[lane + 32] : 0u;
+      const uint32_t cnt = __popc(cw0) + __popc(cw1);
+      uint32_t incl = cnt;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) nd += __shfl_xor_sync(0xFFFFFFFFu, nd, off);
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      nca = use_mask ? __shfl_sync(0xFFFFFFFFu, incl, 31) : kSelCapW + 1u;  // no bitmap: rescan later
+      uint32_t p = incl - cnt;
+      for (uint32_t v = cw0; v; v &= v - 1, ++p)
+        if (p < kSelCapW) my_cands[p] = static_cast<uint32_t>(w_lo + lane * 32 + (__ffs(v) - 1));
+      for (uint32_t v = cw1; v; v &= v - 1, ++p)
+        if (p < kSelCapW) my_cands[p] = static_cast<uint32_t>(w_lo + (lane + 32) * 32 + (__ffs(v) - 1));
+      __syncwarp();
     }
     const bool cand_list = nca <= kSelCapW;  // warp-uniform: else this warp rescans its range
     if (lane == 0) warp_nc[warp] = cand_list ? nca : (kSelGather + 1u);
@@ -488,8 +493,20 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
     uint32_t prefix = d1 << 20, mask = 0xFFF00000u, krem = k1;
     if (gtotal <= kSelGather) {
       // exact selection among the gathered keys, locally in every CTA: digits 2 and 3
-      if (crank != 0)
-        for (int j = tid; j < static_cast<int>(gtotal); j += kSelThreads) gbuf[j] = gbuf0[j];
+      if (crank != 0) {  // copy the gathered keys: all remote loads in flight before the stores
+        constexpr int kCopy = (kSelGather + kSelThreads - 1) / kSelThreads;
+        uint32_t v[kCopy];
+#pragma unroll
+        for (int u = 0; u < kCopy; ++u) {
+          const int j = tid + u * kSelThreads;
+          v[u] = (j < static_cast<int>(gtotal)) ? gbuf0[j] : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kCopy; ++u) {
+          const int j = tid + u * kSelThreads;
+          if (j < static_cast<int>(gtotal)) gbuf[j] = v[u];
+        }
+      }
 #pragma unroll 1
       for (int pass = 0; pass < 2; ++pass) {
         const int shift = (pass == 0) ? 10 : 0;
@@ -717,7 +734,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
 }
 
 constexpr int kSelMaxSlice = 16384;    // keys per CTA kept in shared memory
-constexpr int kSelStaticBytes = 2048;  // static shared memory of the kernel, rounded up
+constexpr int kSelStaticBytes = 3072;  // static shared memory of the kernel, rounded up
 
 // Number of clusters of this shape that can be resident at once (cached per device).
 template <typename Kernel>
