@@ -34,12 +34,8 @@ static size_t attn_smem_bytes() {
 template <int D, int NTILE, bool DENSE>
 __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
   using Cfg = AttnCfg<D>;
-  constexpr int STAGES = Cfg::STAGES, CPR = Cfg::CPR;
   constexpr int KSTEPS = D / 16;
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, c = lane & 3;
-  unsigned char* ring = smem_raw + warp * STAGES * Cfg::STAGE_BYTES;
   int32_t* tok_s = reinterpret_cast<int32_t*>(smem_raw + Cfg::MAIN_BYTES);
 
   const int split = blockIdx.x, row = blockIdx.y;
@@ -87,18 +83,18 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
   float* pbuf = reinterpret_cast<float*>(smem_raw + Cfg::COMBINE_BYTES);   // [16][D] (cluster merge)
   float* plse = pbuf + 16 * D;                                              // [16]
   if (my_len == 0) {  // empty split: weight zero in the merge
-    if (!DENSE) {
+    if constexpr (!DENSE) {
       for (int i = threadIdx.x; i < G * D; i += kAttnThreads) pbuf[i] = 0.f;
       if (threadIdx.x < G) plse[threadIdx.x] = -INFINITY;
       cluster_merge<D>(a, hq0, G, pbuf, plse);
-      return;
+    } else {
+      for (int i = threadIdx.x; i < G * D; i += kAttnThreads) {
+        const int head = i / D, dim = i % D;
+        a.part_o[((hq0 + head) * a.S + split) * D + dim] = 0.f;
+        if (dim == 0) a.part_lse[(hq0 + head) * a.S + split] = -INFINITY;
+      }
+      finish_split<D>(a, row, hq0, G, reinterpret_cast<float*>(smem_raw));
     }
-    for (int i = threadIdx.x; i < G * D; i += kAttnThreads) {
-      const int head = i / D, dim = i % D;
-      a.part_o[((hq0 + head) * a.S + split) * D + dim] = 0.f;
-      if (dim == 0) a.part_lse[(hq0 + head) * a.S + split] = -INFINITY;
-    }
-    finish_split<D>(a, row, hq0, G, reinterpret_cast<float*>(smem_raw));
     return;
   }
   if (!DENSE) {
