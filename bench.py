@@ -183,6 +183,7 @@ class Setup:
         tb = torch.zeros(w.B, dtype=torch.int32, device=device)
         jssa.project_keys(self.L, self.K, self.P, self.Kp, self.T_cap, t_begin=tb)   # prefill fill
         self.ws = jssa.alloc_workspace(self.L, w.k, w.window)
+        self.gbuf = jssa.alloc_gather_buffer(self.L, w.k, w.window) if w.mode != "mla" else None
         self.O = torch.empty(w.B, w.Hq, w.dv, dtype=torch.bfloat16, device=device)
         self.idx = torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=device)
         self.nsel = torch.empty(w.B, w.Hkv, dtype=torch.int32, device=device)
@@ -225,7 +226,8 @@ def stage_times(st, Q, reps=50):
     """Device time of the public entry points that make up the step, each replayed from a
     CUDA graph of `reps` calls (CUDA events on the replay stream).  select = the selection
     half of the step (projections, score scan, top-k: one kernel when the cache fits a
-    cluster); attention = indexed attention with its merge; dense = the full-KV comparator."""
+    cluster); attention = indexed attention with its merge; dense = the full-KV comparator;
+    gather_then_attend = the same attention done the gather-based way (copy, then dense)."""
     jssa, w = st.jssa, st.w
     calls = {
         "select_us": lambda: jssa.select(st.L, Q, st.K, st.Kp, st.P, st.seq_lens, 1, w.k, w.window, st.idx,
@@ -235,6 +237,10 @@ def stage_times(st, Q, reps=50):
     }
     if st.w.mode != "mla":  # the MLA path is indexed only
         calls["dense_us"] = lambda: st.dense(Q)
+        # the gather-based baseline of the pages: copy the attended rows, then dense decode on them
+        calls["gather_then_attend_us"] = lambda: jssa.gather_decode(st.L, Q, st.K, st.V, st.idx, w.k, st.nsel,
+                                                                    st.seq_lens, w.window, w.sm_scale, st.O, None,
+                                                                    st.gbuf, st.ws)
     out = {}
     for name, fn in calls.items():
         fn()

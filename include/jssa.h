@@ -219,6 +219,22 @@ JSSA_API jssa_status jssa_decode_step(const jssa_layout* L, const void* Q, const
                              size_t ws_bytes, void* stream);
 
 /*
+ * Gather-then-attend comparator (§2.2, §3.3, §4.7): not the method's path, but the
+ * gather-based baseline its gather-free kernel is measured against.  The attended rows of every
+ * (sequence, KV head), exactly as jssa_indexed_attn defines them, are first copied into a compact
+ * buffer; then the dense flash-decode runs over that buffer.  GQA only.
+ * jssa_gather_size gives the bytes of the caller-owned gather buffer (16-byte aligned):
+ * gathered K and V [B*Hkv, Lmax, d] bf16 with Lmax = k + min(window, T_cap), plus the row
+ * lengths.  The workspace is the one jssa_workspace_size(L, k, window) sizes.
+ */
+JSSA_API jssa_status jssa_gather_size(const jssa_layout* L, int32_t k, int32_t window, size_t* bytes);
+JSSA_API jssa_status jssa_gather_decode(const jssa_layout* L, const void* Q, const void* K, const void* V,
+                                        const int32_t* idx, int32_t k, const int32_t* n_sel,
+                                        const int32_t* seq_lens, int32_t window, float sm_scale, void* O,
+                                        float* lse, void* gather_buf, size_t gather_bytes, void* workspace,
+                                        size_t ws_bytes, void* stream);
+
+/*
  * Dense full-KV flash-decode (the full-KV baseline of §4.5), same kernel family as
  * jssa_indexed_attn with the index list replaced by the contiguous range
  * [T_b - W, T_b) (W = window clamped to T_b; window = 0 means all of [0, T_b)).

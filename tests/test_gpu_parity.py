@@ -238,6 +238,39 @@ def test_indexed_attention_matches_oracle(name, kw, seq, k, window, out):
     _assert_status_clean(ws)
 
 
+@pytest.mark.parametrize("name,kw,seq,k,window", [
+    ("tiny", {}, None, 128, 0),
+    ("h128k", dict(B=2, T=9000), [9000, 4000], 2048, 0),
+    ("hybrid", dict(B=2, T=6000), [6000, 1500], 1024, 1024),    # d = 256 + window
+    ("h128k", dict(B=1, T=3000, Hq=32, Hkv=2), [3000], 257, 0),  # G = 16
+])
+def test_gather_then_attend_comparator_matches_oracle(name, kw, seq, k, window):
+    w = W[name].with_(**kw)
+    p = Problem(w, seq_lens=seq)
+    seq = seq or [w.T] * w.B
+    ncand = [T - min(window, T) for T in seq]
+    idx = synth.random_index_sets(w.B * w.Hkv, [n for n in ncand for _ in range(w.Hkv)], k, seed=k + 1)
+    nsel = (idx >= 0).sum(-1).to(torch.int32).view(w.B, w.Hkv).cuda()
+    idx = idx.view(w.B, w.Hkv, k).cuda()
+    ws = p.workspace(k, window)
+    gbuf = jssa.alloc_gather_buffer(p.L, k, window)
+    O = torch.full((w.B, w.Hq, w.dv), float("nan"), device="cuda")
+    lse = torch.full((w.B, w.Hq), float("nan"), device="cuda")
+    jssa.gather_decode(p.L, p.Q, p.K, p.V, idx, k, nsel, p.seq_lens, window, w.sm_scale, O, lse, gbuf, ws)
+    torch.cuda.synchronize()
+    G = w.G
+    for b in range(w.B):
+        T = seq[b]
+        for h in range(w.Hkv):
+            hst = p.host(b, h)
+            n = int(nsel[b, h])
+            toks = np.concatenate([idx[b, h, :n].cpu().numpy(), np.arange(T - min(window, T), T)])
+            O_ref, lse_ref = oracle.attention(hst["Q"], hst["K"], hst["V"], toks, w.sm_scale)
+            check_attention(O[b, h * G:(h + 1) * G].cpu().numpy().astype(np.float64), O_ref, f"gather b={b} h={h}")
+            np.testing.assert_allclose(lse[b, h * G:(h + 1) * G].cpu().numpy(), lse_ref, atol=1e-4, rtol=1e-5)
+    _assert_status_clean(ws)
+
+
 @pytest.mark.parametrize("name,kw,seq,window", [
     ("tiny", {}, None, 0),
     ("h128k", dict(B=2, T=7000), [7000, 333], 0),

@@ -25,7 +25,7 @@ DEV_BAD_SEQ_LEN, DEV_BAD_INDEX, DEV_BAD_NSEL, DEV_TIMEOUT = 1, 2, 4, 8
 
 EXPORTS = ("jssa_status_string", "jssa_version", "jssa_workspace_size", "jssa_project_keys", "jssa_score",
            "jssa_topk", "jssa_topk_noalloc", "jssa_select", "jssa_indexed_attn", "jssa_decode_step",
-           "jssa_dense_decode",
+           "jssa_dense_decode", "jssa_gather_size", "jssa_gather_decode",
            "jssa_workspace_init", "jssa_read_device_status")
 
 
@@ -67,6 +67,8 @@ def load(path: str = LIB_PATH):
         "jssa_select": (C.c_int, [LP, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
         "jssa_indexed_attn": (C.c_int, [LP, vp, vp, vp, vp, i32, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
         "jssa_decode_step": (C.c_int, [LP, vp, vp, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, vp, vp, sz, vp]),
+        "jssa_gather_size": (C.c_int, [LP, i32, i32, C.POINTER(sz)]),
+        "jssa_gather_decode": (C.c_int, [LP, vp, vp, vp, vp, i32, vp, vp, i32, f32, vp, vp, vp, sz, vp, sz, vp]),
         "jssa_dense_decode": (C.c_int, [LP, vp, vp, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
         "jssa_workspace_init": (C.c_int, [vp, sz, vp]),
         "jssa_read_device_status": (C.c_int, [vp, sz, C.POINTER(i32), vp]),
@@ -195,6 +197,21 @@ def decode_step(L, Q, K, V, Kp, P, seq_lens, n_new: int, k: int, window: int, sm
     _check("jssa_decode_step", load().jssa_decode_step(C.byref(L), _c(Q), _p(K), _p(V), _p(Kp), _c(P),
                                                        _c(seq_lens), n_new, k, window, sm_scale, _c(O), _c(lse),
                                                        _c(idx_out), _c(n_sel_out), w, n, _stream(stream)))
+
+
+def alloc_gather_buffer(L, k: int, window: int = 0, device="cuda"):
+    """Device buffer for gather_decode (the gather-then-attend comparator)."""
+    n = C.c_size_t(0)
+    _check("jssa_gather_size", load().jssa_gather_size(C.byref(L), k, window, C.byref(n)))
+    return torch.empty(n.value, dtype=torch.uint8, device=device)
+
+
+def gather_decode(L, Q, K, V, idx, k: int, n_sel, seq_lens, window: int, sm_scale: float, O, lse, gbuf, ws,
+                  stream=None):
+    w, n = _ws(ws)
+    _check("jssa_gather_decode", load().jssa_gather_decode(C.byref(L), _c(Q), _p(K), _p(V), _c(idx), k, _c(n_sel),
+                                                           _c(seq_lens), window, sm_scale, _c(O), _c(lse), _c(gbuf),
+                                                           gbuf.numel(), w, n, _stream(stream)))
 
 
 def dense_decode(L, Q, K, V, seq_lens, window: int, sm_scale: float, O, lse=None, ws=None, stream=None):

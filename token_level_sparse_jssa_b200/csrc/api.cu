@@ -507,6 +507,88 @@ jssa_status jssa_decode_step(const jssa_layout* L, const void* Q, const void* K,
   return run_attention(L, Q, K, V, idx, k, nsel, seq_lens, window, sm_scale, O, lse, w, true, s);
 }
 
+namespace {
+// Bytes of the gather buffer and its pieces: K and V [rows, Lmax, d] bf16, then the row lengths.
+size_t gather_layout(const jssa_layout* L, int64_t k, int64_t window, int64_t* Lmax, size_t* off_v,
+                     size_t* off_len) {
+  *Lmax = k + min64(window, L->T_cap);
+  const size_t rows = static_cast<size_t>(L->B) * L->Hkv;
+  const size_t kv = align_up(rows * static_cast<size_t>(*Lmax) * L->d_k * 2);
+  *off_v = kv;
+  *off_len = 2 * kv;
+  return 2 * kv + align_up(rows * sizeof(int32_t));
+}
+}  // namespace
+
+jssa_status jssa_gather_size(const jssa_layout* L, int32_t k, int32_t window, size_t* bytes) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  if (L->mode == JSSA_MODE_MLA) return JSSA_ERR_UNSUPPORTED;
+  if (!bytes || k < 1 || k > kMaxK || window < 0) return JSSA_ERR_INVALID_ARG;
+  int64_t Lmax;
+  size_t ov, ol;
+  *bytes = gather_layout(L, k, window, &Lmax, &ov, &ol);
+  return JSSA_OK;
+}
+
+jssa_status jssa_gather_decode(const jssa_layout* L, const void* Q, const void* K, const void* V, const int32_t* idx,
+                               int32_t k, const int32_t* n_sel, const int32_t* seq_lens, int32_t window,
+                               float sm_scale, void* O, float* lse, void* gather_buf, size_t gather_bytes,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  if (L->mode == JSSA_MODE_MLA) return JSSA_ERR_UNSUPPORTED;
+  if (!Q || !K || !V || !idx || !n_sel || !seq_lens || !O || !gather_buf || k < 1 || k > kMaxK || window < 0)
+    return JSSA_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 4) || !aligned(gather_buf, 16))
+    return JSSA_ERR_INVALID_ARG;
+  int64_t Lmax;
+  size_t off_v, off_len;
+  const size_t need = gather_layout(L, k, window, &Lmax, &off_v, &off_len);
+  if (gather_bytes < need) return JSSA_ERR_WORKSPACE;
+  Workspace w{};
+  st = get_ws(L, k, window, workspace, ws_bytes, &w);
+  if (st != JSSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* gb = static_cast<char*>(gather_buf);
+  GatherArgs g{};
+  g.K = K;
+  memcpy(g.ks, L->k_stride, sizeof g.ks);
+  g.V = V;
+  memcpy(g.vs, L->v_stride, sizeof g.vs);
+  g.idx = idx;
+  g.idx_ld = k;
+  g.n_sel = n_sel;
+  g.seq_lens = seq_lens;
+  g.B = L->B;
+  g.Hkv = L->Hkv;
+  g.d = L->d_k;
+  g.window = window;
+  g.T_cap = L->T_cap;
+  g.Lmax = Lmax;
+  g.Kg = gb;
+  g.Vg = gb + off_v;
+  g.glen = reinterpret_cast<int32_t*>(gb + off_len);
+  g.status = w.status;
+  st = cu(launch_gather_rows(g, s));
+  if (st != JSSA_OK) return st;
+  // the buffer as a cache of B*Hkv sequences with one KV head and G query heads each
+  jssa_layout Lg = *L;
+  Lg.B = L->B * L->Hkv;
+  Lg.Hkv = 1;
+  Lg.Hq = L->Hq / L->Hkv;
+  Lg.T_cap = Lmax;
+  const int64_t kst[3] = {Lmax * L->d_k, Lmax * L->d_k, L->d_k};
+  memcpy(Lg.k_stride, kst, sizeof kst);
+  memcpy(Lg.v_stride, kst, sizeof kst);
+  const int64_t pst[3] = {Lmax * L->r, Lmax * L->r, L->r};
+  memcpy(Lg.kp_stride, pst, sizeof pst);
+  int S = 0, len = 0;
+  attn_split_policy(Lg.mode, false, Lg.B * Lg.Hkv, Lmax, num_sms_current(), &S, &len);
+  if (S > w.S_cap) return JSSA_ERR_WORKSPACE;
+  return run_attention(&Lg, Q, gb, gb + off_v, nullptr, 0, nullptr, g.glen, 0, sm_scale, O, lse, w, false, s);
+}
+
 jssa_status jssa_dense_decode(const jssa_layout* L, const void* Q, const void* K, const void* V,
                               const int32_t* seq_lens, int32_t window, float sm_scale, void* O, float* lse,
                               void* workspace, size_t ws_bytes, void* stream) {

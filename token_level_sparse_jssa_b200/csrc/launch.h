@@ -132,6 +132,25 @@ cudaError_t launch_select(const SelectArgs& a, int num_sms, cudaStream_t s);
 int64_t select_max_candidates();
 int select_max_new_rows();
 
+// Gather-then-attend comparator: copy each row's attended K/V rows into [B*Hkv, Lmax, d] buffers.
+struct GatherArgs {
+  const void* K;
+  int64_t ks[3];
+  const void* V;
+  int64_t vs[3];
+  const int32_t* idx;
+  int idx_ld;
+  const int32_t* n_sel;
+  const int32_t* seq_lens;
+  int B, Hkv, d, window;
+  int64_t T_cap, Lmax;
+  void* Kg;
+  void* Vg;
+  int32_t* glen;   // [B*Hkv] attended positions per row
+  int* status;
+};
+cudaError_t launch_gather_rows(const GatherArgs& a, cudaStream_t s);
+
 // Split policy shared by the workspace sizing and the launch.
 void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int num_sms, int* S, int* split_len);
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);   // GQA path
