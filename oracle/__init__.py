@@ -37,6 +37,13 @@ def _load():
         lib.or_double_to_bf16_array.argtypes = [f64p, C.c_int64, u16p]
         lib.or_project_rows.argtypes = [u16p, C.c_int64, C.c_int, f32p, C.c_int, C.c_int64,
                                         u16p, C.c_int64, f64p]
+        u8p = C.POINTER(C.c_uint8)
+        lib.or_e4m3_to_double.argtypes = [C.c_uint8]
+        lib.or_e4m3_to_double.restype = C.c_double
+        lib.or_double_to_e4m3.argtypes = [C.c_double]
+        lib.or_double_to_e4m3.restype = C.c_uint8
+        lib.or_project_rows_e4m3.argtypes = [u16p, C.c_int64, C.c_int, f32p, C.c_int, C.c_int64, u8p, C.c_int64, f64p]
+        lib.or_scores_e4m3.argtypes = [f64p, C.c_int, u8p, C.c_int64, C.c_int64, f64p]
         lib.or_query_proj.argtypes = [u16p, C.c_int, C.c_int, f32p, C.c_int, f64p]
         lib.or_scores.argtypes = [f64p, C.c_int, u16p, C.c_int64, C.c_int64, f64p]
         lib.or_topk.argtypes = [f64p, C.c_int64, C.c_int64, i32p]
@@ -100,6 +107,40 @@ def project_rows(K: np.ndarray, P: np.ndarray):
     _load().or_project_rows(_ptr(K, C.c_uint16), k_ld, d, _ptr(P, C.c_float), r, n,
                             _ptr(Kp, C.c_uint16), r, _ptr(ex, C.c_double))
     return Kp[:n], ex[:n]
+
+
+def e4m3_to_double(c: int) -> float:
+    """Value of one FP8 E4M3 code."""
+    return _load().or_e4m3_to_double(int(c))
+
+
+def double_to_e4m3(x: float) -> int:
+    """FP8 E4M3 code of x: round to nearest even, saturate to +-448."""
+    return int(_load().or_double_to_e4m3(float(x)))
+
+
+def project_rows_e4m3(K: np.ndarray, P: np.ndarray):
+    """FP8 projected scoring cache rows: Kp8 = e4m3(K . P) from the exact product (the paper's
+    deployed precision, §A.3 / §E.2).  Returns (Kp8 uint8 [n, r], exact float64 [n, r])."""
+    K, k_ld = _rows(K, np.uint16)
+    P = np.ascontiguousarray(P, np.float32)
+    d, r = P.shape
+    n = K.shape[0] if K.shape[1] == d else 0
+    Kp = np.zeros((max(n, 1), r), np.uint8)
+    ex = np.zeros((max(n, 1), r), np.float64)
+    _load().or_project_rows_e4m3(_ptr(K, C.c_uint16), k_ld, d, _ptr(P, C.c_float), r, n,
+                                 _ptr(Kp, C.c_uint8), r, _ptr(ex, C.c_double))
+    return Kp[:n], ex[:n]
+
+
+def scores_e4m3(qs: np.ndarray, Kp8: np.ndarray) -> np.ndarray:
+    """fp64 scores against an FP8 projected cache: s_t = qs . value(Kp8_t)."""
+    qs = np.ascontiguousarray(qs, np.float64)
+    Kp8 = np.ascontiguousarray(Kp8, np.uint8)
+    n, r = Kp8.shape
+    s = np.zeros(max(n, 1), np.float64)
+    _load().or_scores_e4m3(_ptr(qs, C.c_double), r, _ptr(Kp8, C.c_uint8), r, n, _ptr(s, C.c_double))
+    return s[:n]
 
 
 def query_proj(Qg: np.ndarray, P: np.ndarray) -> np.ndarray:

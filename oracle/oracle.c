@@ -106,6 +106,69 @@ void or_project_rows(const uint16_t* K, int64_t k_ld, int d,
 /*   qs[j] = sum_g sum_i P[i, j] * q_g[i]                                      */
 /* Q holds the G query heads of one KV group, each of length d (bf16).         */
 /* ------------------------------------------------------------------------- */
+/* ---------------------------------------------------------------------------------------
+ * FP8 E4M3 projected cache (the paper's deployed projected-cache precision, §A.3 / §E.2).
+ * Format (OCP 8-bit floating point, "E4M3"): 1 sign bit, 4 exponent bits with bias 7, 3
+ * mantissa bits; exponent 0 encodes subnormals m * 2^-9; no infinities; S.1111.111 is NaN, so
+ * the largest finite magnitude is 1.75 * 2^8 = 448.  Encoding here: round to nearest, ties to
+ * even, and magnitudes that round beyond 448 saturate to 448 (the cache never holds NaN).
+ * Unit scale: the stored code is the rounding of the exact product itself.
+ * --------------------------------------------------------------------------------------- */
+double or_e4m3_to_double(uint8_t c)
+{
+    const int sign = (c >> 7) & 1, e = (c >> 3) & 15, m = c & 7;
+    double a;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) a = ldexp((double)m, -9);                 /* subnormal: m / 8 * 2^-6 */
+    else a = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -a : a;
+}
+
+uint8_t or_double_to_e4m3(double x)
+{
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs(x);
+    if (isnan(x)) return 0x7F;
+    if (a >= 464.0) return (uint8_t)(sign | 0x7E);        /* 464 = midpoint of 448 and 480 */
+    if (a < ldexp(1.0, -6)) {                             /* subnormal spacing 2^-9 */
+        double q = nearbyint(a / ldexp(1.0, -9));         /* ties to even (default mode) */
+        return (uint8_t)(sign | (uint8_t)q);              /* q = 8 is the smallest normal 0x08 */
+    }
+    int E;
+    frexp(a, &E);                                         /* a = f * 2^E, 0.5 <= f < 1 */
+    int e = E - 1;                                        /* a in [2^e, 2^(e+1)) */
+    double q = nearbyint((a / ldexp(1.0, e) - 1.0) * 8.0);/* mantissa in eighths, ties even */
+    if (q == 8.0) { q = 0.0; e += 1; }
+    if (e > 8 || (e == 8 && q == 7.0)) return (uint8_t)(sign | 0x7E);  /* beyond 448: saturate */
+    return (uint8_t)(sign | (uint8_t)((e + 7) << 3) | (uint8_t)q);
+}
+
+/* Kp8[t, j] = e4m3(sum_i K[t, i] * P[i, j]) from the exact (fp64) product. */
+void or_project_rows_e4m3(const uint16_t* K, int64_t k_ld, int d, const float* P, int r, int64_t n,
+                          uint8_t* Kp, int64_t kp_ld, double* kp_exact)
+{
+    for (int64_t t = 0; t < n; ++t) {
+        const uint16_t* krow = K + t * k_ld;
+        for (int j = 0; j < r; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < d; ++i)
+                acc += or_bf16_to_double(krow[i]) * (double)P[(int64_t)i * r + j];
+            Kp[t * kp_ld + j] = or_double_to_e4m3(acc);
+            if (kp_exact) kp_exact[t * r + j] = acc;
+        }
+    }
+}
+
+/* s[t] = sum_j qs[j] * e4m3_value(Kp8[t, j]) in fp64. */
+void or_scores_e4m3(const double* qs, int r, const uint8_t* Kp, int64_t kp_ld, int64_t n, double* s)
+{
+    for (int64_t t = 0; t < n; ++t) {
+        double acc = 0.0;
+        for (int j = 0; j < r; ++j) acc += qs[j] * or_e4m3_to_double(Kp[t * kp_ld + j]);
+        s[t] = acc;
+    }
+}
+
 void or_query_proj(const uint16_t* Q, int G, int d, const float* P, int r, double* qs)
 {
     for (int j = 0; j < r; ++j) {

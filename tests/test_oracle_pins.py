@@ -346,3 +346,65 @@ def test_whole_batch_decode_step_on_tiny_workload():
     assert np.all(out["idx"] < 500) and np.all(np.diff(out["idx"], axis=-1) > 0)
     # heavy (x4) rows dominate the selection of this generator
     assert np.isfinite(out["O"]).all()
+
+
+# ----------------------------------------------------------------------------- FP8 E4M3 projected cache
+def test_e4m3_decodes_the_format_constants():
+    # OCP E4M3: bias 7, 3 mantissa bits, subnormals m * 2^-9, S.1111.111 is NaN, max 448
+    assert oracle.e4m3_to_double(0x7E) == 448.0
+    assert oracle.e4m3_to_double(0x08) == 2.0 ** -6      # smallest normal
+    assert oracle.e4m3_to_double(0x07) == 7 * 2.0 ** -9  # largest subnormal
+    assert oracle.e4m3_to_double(0x01) == 2.0 ** -9      # smallest subnormal
+    assert oracle.e4m3_to_double(0x38) == 1.0
+    assert oracle.e4m3_to_double(0x40) == 2.0
+    assert oracle.e4m3_to_double(0x3C) == 1.5
+    assert oracle.e4m3_to_double(0xB8) == -1.0
+    assert oracle.e4m3_to_double(0x00) == 0.0 and math.copysign(1.0, oracle.e4m3_to_double(0x80)) == -1.0
+    assert math.isnan(oracle.e4m3_to_double(0x7F)) and math.isnan(oracle.e4m3_to_double(0xFF))
+
+
+def test_e4m3_agrees_with_torch_float8_on_every_code_and_on_in_range_rounding():
+    codes = torch.arange(256, dtype=torch.uint8)
+    tvals = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for c in range(256):
+        v = oracle.e4m3_to_double(c)
+        if math.isnan(v):
+            assert math.isnan(tvals[c])
+        else:
+            assert v == tvals[c], (c, v, tvals[c])
+    g = torch.Generator().manual_seed(7)
+    x = torch.cat([torch.randn(4000, generator=g, dtype=torch.float64) * s for s in (1e-3, 0.05, 1.0, 30.0)])
+    x = x[x.abs() < 440]
+    mids = torch.tensor([1 + 1 / 16, 1 + 3 / 16, 2 ** -9 * 0.5, 2 ** -9 * 1.5, 2 ** -9 * 2.5, 240 + 8], dtype=torch.float64)
+    x = torch.cat([x, mids, -mids])
+    ref = x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.double_to_e4m3(float(v)) for v in x.numpy()], np.uint8)
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_e4m3_encoding_ties_to_even_and_saturates():
+    assert oracle.double_to_e4m3(1 + 1 / 16) == 0x38           # midway 1.0 / 1.125 -> even mantissa
+    assert oracle.double_to_e4m3(1 + 3 / 16) == 0x3A           # midway 1.125 / 1.25 -> even
+    assert oracle.double_to_e4m3(0.5 * 2.0 ** -9) == 0x00      # midway 0 / 2^-9 -> 0
+    assert oracle.double_to_e4m3(1.5 * 2.0 ** -9) == 0x02      # midway 1 / 2 subnormal steps -> 2
+    assert oracle.double_to_e4m3(460.0) == 0x7E and oracle.double_to_e4m3(1e9) == 0x7E
+    assert oracle.double_to_e4m3(-1e9) == 0xFE
+    for c in list(range(0, 0x7F)) + list(range(0x80, 0xFF)):   # every finite code round-trips
+        assert oracle.double_to_e4m3(oracle.e4m3_to_double(c)) == c
+
+
+def test_e4m3_projection_is_the_rounded_exact_product():
+    rng = np.random.default_rng(3)
+    d, r, n = 64, 16, 50
+    K = rng.standard_normal((n, d)).astype(np.float32)
+    Kb = (K.view(np.uint32) >> 16).astype(np.uint16)        # bf16 truncation of the inputs
+    P = np.linalg.qr(rng.standard_normal((d, r)))[0].astype(np.float32)
+    Kp8, ex = oracle.project_rows_e4m3(Kb, P)
+    Kd = oracle.bf16_to_f64(Kb)
+    exact = Kd @ P.astype(np.float64)
+    np.testing.assert_allclose(ex, exact, rtol=1e-12, atol=1e-12)
+    want = np.array([[oracle.double_to_e4m3(v) for v in row] for row in exact], np.uint8)
+    np.testing.assert_array_equal(Kp8, want)
+    qs = rng.standard_normal(r)
+    vals = np.vectorize(oracle.e4m3_to_double)(Kp8)
+    np.testing.assert_allclose(oracle.scores_e4m3(qs, Kp8), vals @ qs, rtol=1e-13)
