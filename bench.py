@@ -9,7 +9,11 @@ T projected keys, select the top-k per (sequence, KV head), attend over the sele
 rows in place and merge the split partials.  Every timed step uses a fresh query
 batch, so every step selects a different token set.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME] [--kp bf16|e4m3]
+
+``--kp e4m3`` stores the projected scoring cache in FP8 E4M3 (the paper's deployed
+configuration) instead of bf16; the default line also reports the step over an E4M3 cache
+as a stage time.
 
 N > 1 runs under torchrun: each rank owns an independent batch of sequences (weak
 scaling, no collective on the data path); time is the max over ranks.
@@ -60,23 +64,26 @@ def parse():
     ap.add_argument("--workload", default="h128k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--kp", default="bf16", choices=["bf16", "e4m3"], help="projected scoring cache type")
     return ap.parse_args()
 
 
 # --------------------------------------------------------------------------- helpers
-def byte_model(w, T, k, window, out_bytes=2):
-    """Algorithmic bytes of one step and of the dense step (HBM roofline numerator)."""
+def byte_model(w, T, k, window, out_bytes=2, kp_bytes=2):
+    """Algorithmic bytes of one step and of the dense step (HBM roofline numerator);
+    kp_bytes = bytes per projected-cache element (2 bf16, 1 E4M3)."""
     n = T - min(window, T)
     keff = min(k, n)
     rows = w.B * w.Hkv
-    kp = rows * n * w.r * 2
+    kp = rows * n * w.r * kp_bytes
     kv_row = (w.dk if w.mode == "mla" else w.dk + w.dv) * 2
     sel = rows * (keff + min(window, T)) * kv_row
     qo = w.B * w.Hq * (w.dk * 2 + w.dv * out_bytes)
     dense = rows * T * kv_row + qo
     # the selection kernel: Kp scan, queries, bases, the newest key row in and its Kp row
     # out, indices and counts out (the scores and histograms stay on chip)
-    select = kp + w.B * w.Hq * w.dk * 2 + w.Hkv * w.dk * w.r * 4 + rows * (w.dk * 2 + w.r * 2) + rows * (k * 4 + 4)
+    select = (kp + w.B * w.Hq * w.dk * 2 + w.Hkv * w.dk * w.r * 4 + rows * (w.dk * 2 + w.r * kp_bytes)
+              + rows * (k * 4 + 4))
     return dict(kp=kp, selected=sel, qo=qo, step=kp + sel + qo, dense=dense, scores=rows * n * 4, select=select)
 
 
@@ -166,7 +173,7 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- workload setup
 class Setup:
-    def __init__(self, w, device, seed_offset=0):
+    def __init__(self, w, device, seed_offset=0, kp="bf16"):
         import token_level_sparse_jssa_b200 as jssa
         from token_level_sparse_jssa_b200 import synth
         self.jssa, self.w = jssa, w
@@ -177,11 +184,8 @@ class Setup:
         self.P = x["P"].contiguous()
         self.seq_lens = x["seq_lens"]
         self.A = x["A"]
-        self.Kp = torch.empty(w.B, w.Hkv, self.T_cap, w.r, dtype=torch.bfloat16, device=device)
-        self.L = jssa.make_layout(self.K, self.V, self.Kp, w.Hq, w.r,
-                                  jssa.MODE_MLA if w.mode == "mla" else jssa.MODE_GQA, jssa.OUT_BF16)
-        tb = torch.zeros(w.B, dtype=torch.int32, device=device)
-        jssa.project_keys(self.L, self.K, self.P, self.Kp, self.T_cap, t_begin=tb)   # prefill fill
+        self.Kp, self.L = self.scoring_cache(kp)
+        self.kp = kp
         self.ws = jssa.alloc_workspace(self.L, w.k, w.window)
         self.gbuf = jssa.alloc_gather_buffer(self.L, w.k, w.window) if w.mode != "mla" else None
         self.O = torch.empty(w.B, w.Hq, w.dv, dtype=torch.bfloat16, device=device)
@@ -189,10 +193,21 @@ class Setup:
         self.nsel = torch.empty(w.B, w.Hkv, dtype=torch.int32, device=device)
         torch.cuda.synchronize()
 
-    def step(self, Q):
+    def scoring_cache(self, kp):
+        """A projected scoring cache of this workload (bf16 or E4M3) filled from K, and its layout."""
+        jssa, w = self.jssa, self.w
+        Kp = torch.empty(w.B, w.Hkv, self.T_cap, w.r, dtype=torch.uint8 if kp == "e4m3" else torch.bfloat16,
+                         device=self.K.device)
+        L = jssa.make_layout(self.K, self.V, Kp, w.Hq, w.r, jssa.MODE_MLA if w.mode == "mla" else jssa.MODE_GQA,
+                             jssa.OUT_BF16)
+        tb = torch.zeros(w.B, dtype=torch.int32, device=self.K.device)
+        jssa.project_keys(L, self.K, self.P, Kp, self.T_cap, t_begin=tb)   # prefill fill
+        return Kp, L
+
+    def step(self, Q, Kp=None, L=None):
         w = self.w
-        self.jssa.decode_step(self.L, Q, self.K, self.V, self.Kp, self.P, self.seq_lens, 1, w.k, w.window,
-                              w.sm_scale, self.O, None, self.idx, self.nsel, self.ws)
+        self.jssa.decode_step(self.L if L is None else L, Q, self.K, self.V, self.Kp if Kp is None else Kp, self.P, self.seq_lens,
+                              1, w.k, w.window, w.sm_scale, self.O, None, self.idx, self.nsel, self.ws)
 
     def dense(self, Q):
         self.jssa.dense_decode(self.L, Q, self.K, self.V, self.seq_lens, 0, self.w.sm_scale, self.O, None, self.ws)
@@ -227,7 +242,8 @@ def stage_times(st, Q, reps=50):
     CUDA graph of `reps` calls (CUDA events on the replay stream).  select = the selection
     half of the step (projections, score scan, top-k: one kernel when the cache fits a
     cluster); attention = indexed attention with its merge; dense = the full-KV comparator;
-    gather_then_attend = the same attention done the gather-based way (copy, then dense)."""
+    gather_then_attend = the same attention done the gather-based way (copy, then dense);
+    step_other_kp = the whole step over the other scoring-cache type (E4M3 when the run is bf16)."""
     jssa, w = st.jssa, st.w
     calls = {
         "select_us": lambda: jssa.select(st.L, Q, st.K, st.Kp, st.P, st.seq_lens, 1, w.k, w.window, st.idx,
@@ -241,6 +257,9 @@ def stage_times(st, Q, reps=50):
         calls["gather_then_attend_us"] = lambda: jssa.gather_decode(st.L, Q, st.K, st.V, st.idx, w.k, st.nsel,
                                                                     st.seq_lens, w.window, w.sm_scale, st.O, None,
                                                                     st.gbuf, st.ws)
+    other = "bf16" if st.kp == "e4m3" else "e4m3"
+    Kp2, L2 = st.scoring_cache(other)
+    calls[f"step_kp_{other}_us"] = lambda: st.step(Q, Kp2, L2)
     out = {}
     for name, fn in calls.items():
         fn()
@@ -250,11 +269,12 @@ def stage_times(st, Q, reps=50):
         torch.cuda.synchronize()
         out[name] = timed_graph(g, lambda: None) * 1000.0 / reps
         del g
+    del Kp2
     return out
 
 
 # --------------------------------------------------------------------------- CPU oracle timing
-def cpu_oracle_rate(w, seconds: float, data=None):
+def cpu_oracle_rate(w, seconds: float, data=None, kp="bf16"):
     """Time the fp64 oracle's decode step on sampled (sequence, KV head) rows of the workload
     on this host (single thread) for about ``seconds``; returns (steps/s, description)."""
     import numpy as np
@@ -268,18 +288,20 @@ def cpu_oracle_rate(w, seconds: float, data=None):
     else:
         K, V, Q, P = data
     rows = [(0, h) for h in range(min(2, w.Hkv))]
+    proj = oracle.project_rows_e4m3 if kp == "e4m3" else oracle.project_rows
+    head = oracle.decode_head_e4m3 if kp == "e4m3" else oracle.decode_head
     G, T = w.G, w.T
     host = []
     for (b, h) in rows:
         Kh, Vh = u16(K[b, h, :T]), u16(V[b, h, :T])
         Ph = f32(P[h])
-        Kp, _ = oracle.project_rows(Kh, Ph)       # cache state before the step (not timed)
+        Kp, _ = proj(Kh, Ph)                      # cache state before the step (not timed)
         host.append((u16(Q[b, h * G:(h + 1) * G]), Kh, Vh, Kp, Ph))
     n, t0 = 0, time.perf_counter()
     while True:
         for (Qg, Kh, Vh, Kp, Ph) in host:
-            oracle.project_rows(Kh[T - 1:T], Ph)  # the newest key, projected on write
-            oracle.decode_head(Qg, Kh, Vh, Kp, Ph, T, w.k, w.window, w.sm_scale)
+            proj(Kh[T - 1:T], Ph)                 # the newest key, projected on write
+            head(Qg, Kh, Vh, Kp, Ph, T, w.k, w.window, w.sm_scale)
             n += 1
         el = time.perf_counter() - t0
         if el >= seconds:
@@ -318,7 +340,7 @@ def run_reference(args, w, cfg):
     rank, _, _ = rank_env()
     if rank != 0:
         return 0
-    rate, desc = cpu_oracle_rate(w, max(0.2, args.cpu_seconds))
+    rate, desc = cpu_oracle_rate(w, max(0.2, args.cpu_seconds), kp=args.kp)
     line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / rate, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
@@ -333,11 +355,12 @@ def main():
     from token_level_sparse_jssa_b200 import synth
     w = synth.WORKLOADS[args.workload]
     rank, world, local = rank_env()
-    bm = byte_model(w, w.T, w.k, w.window)
+    bm = byte_model(w, w.T, w.k, w.window, kp_bytes=1 if args.kp == "e4m3" else 2)
     cfg = {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} d_k={w.dk} d_v={w.dv} r={w.r} T={w.T} k={w.k}"
                        + (f" W={w.window}" if w.window else "") + f" ({w.mode.upper()})",
            "global_batch": w.B * max(world, args.gpus), "seq_len": w.T, "k": w.k, "r": w.r,
            "parallelism": f"dp{max(world, args.gpus)} (independent sequences per rank, no collective)",
+           "kp": "FP8 E4M3 (unit scale)" if args.kp == "e4m3" else "bf16",
            "l2": "inputs larger than L2 (the projected cache alone is %.0f MB per step) and a fresh query every step"
                  % (bm["kp"] / 1e6)}
     if args.impl == "reference":
@@ -357,7 +380,7 @@ def main():
         if dist is not None:
             dist.barrier()
 
-    st = Setup(w, "cuda", seed_offset=rank)
+    st = Setup(w, "cuda", seed_offset=rank, kp=args.kp)
     nq = args.warmup + args.steps
     Qs = synth.fresh_queries(w, nq, st.A, device="cuda", seed=7 + rank)
     # warm-up (untimed), then exactly `steps` timed steps, each in one CUDA graph
@@ -387,7 +410,7 @@ def main():
     n_kernels, fused = step_kernels(w)
     sel_bytes = bm["step"] if fused else bm["select"]
     sel_s = stages["select_us"] * 1e-6
-    shash = source_hash("select.cu", "attn_core.cuh", "common.cuh")
+    shash = source_hash("select_kernel.cuh", "attn_core.cuh", "common.cuh")
 
     # end to end through the public API with host buffers: per step, H2D of the query and of
     # the newest token's K/V rows from pinned memory, the step, and D2H of the output
@@ -423,7 +446,7 @@ def main():
     if rank == 0:
         cpu = None
         if not args.no_cpu_baseline and world == 1:
-            rate, desc = cpu_oracle_rate(w, args.cpu_seconds, data=(st.K, st.V, Qs[0], st.P))
+            rate, desc = cpu_oracle_rate(w, args.cpu_seconds, data=(st.K, st.V, Qs[0], st.P), kp=args.kp)
             cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
         # the dominant kernel: with the attention inside, the step is that one kernel and its
         # launch time is the step time measured above; otherwise the selection kernel alone
@@ -445,7 +468,8 @@ def main():
                                    "select_kernel (query and newest-key projection, score scan, top-k)",
                          "bound": "hbm", "achieved": achieved, "peak": hbm,
                          "unit": "GB/s", "frac": achieved / hbm, "peak_kind": peak_kind,
-                         "traffic": traffic_for("select_kernel", w.name, shash),
+                         "traffic": traffic_for("select_kernel", w.name + ("-e4m3" if args.kp == "e4m3" else ""),
+                                                shash),
                          "algorithmic_bytes_per_launch": sel_bytes},
             "cpu_baseline": cpu,
             "e2e": {"value": whole_job_rate(world, ne, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,

@@ -18,9 +18,14 @@
  *     Kp[t] — the projected query is formed in fp32 from bf16 Q and fp32 P;
  *   - ties in the top-k break toward the lower token index; selected indices are
  *     written in ascending order; unused slots are -1;
- *   - Kp is stored in bf16, rounded to nearest-even once from an fp64 accumulation
- *     of K P (bit-identical to rounding the exact product, except in cases where
- *     the exact value lies within ~1e-16 relative of a rounding midpoint);
+ *   - Kp is stored in bf16 or, with kp_dtype = JSSA_KP_FP8_E4M3, in FP8 E4M3 (the
+ *     paper's deployed scoring cache, §A.3, §E.2), rounded to nearest-even once
+ *     from an fp64 accumulation of K P (bit-identical to rounding the exact product,
+ *     except in cases where the exact value lies within ~1e-16 relative of a
+ *     rounding midpoint).  E4M3 is the OCP format (bias 7, subnormals, max 448)
+ *     with a unit scale and saturation to +-448; a per-head scale s_h is expressed
+ *     by passing P_h / s_h, which scales every score of the (sequence, head) row by
+ *     the same positive factor and leaves the selection unchanged;
  *   - attention uses an explicit softmax scale sm_scale (logit = sm_scale * q . k);
  *     split partials are combined by a log-sum-exp merge;
  *   - with a sliding window W > 0 (hybrid local/global models, §A.1/§A.3), the
@@ -77,6 +82,7 @@ typedef enum {
 
 enum { JSSA_MODE_GQA = 0, JSSA_MODE_MLA = 1 };
 enum { JSSA_OUT_F32 = 0, JSSA_OUT_BF16 = 1 };
+enum { JSSA_KP_BF16 = 0, JSSA_KP_FP8_E4M3 = 1 };
 
 /* Device status bits reported by jssa_read_device_status(). */
 enum {
@@ -91,15 +97,17 @@ enum {
  *   Q    [B, Hq, d_k]      bf16, contiguous
  *   K    element (b, h, t, i) at K[b*k_stride[0] + h*k_stride[1] + t*k_stride[2] + i], i < d_k
  *   V    element (b, h, t, i) at V[b*v_stride[0] + h*v_stride[1] + t*v_stride[2] + i], i < d_v
- *   Kp   element (b, h, t, j) at Kp[b*kp_stride[0] + h*kp_stride[1] + t*kp_stride[2] + j], j < r
+ *   Kp   element (b, h, t, j) at Kp[b*kp_stride[0] + h*kp_stride[1] + t*kp_stride[2] + j], j < r,
+ *        bf16 or E4M3 bytes (kp_dtype); kp_stride[2] = r (rows contiguous)
  *   P    [Hkv, d_k, r]     fp32, contiguous (column j of P_h is the j-th basis vector)
  *   O    [B, Hq, d_v]      fp32 or bf16 (out_dtype), contiguous
  *   lse  [B, Hq]           fp32 natural-log log-sum-exp of the scaled logits (optional)
  * GQA: Hq = G * Hkv; query head hq belongs to KV head hq / G.  Supported: d_k = d_v in
  * {64, 128, 256}, G in {1, 2, 4, 8, 16}, r in {8, 16, 32, 64} (r <= d_k).
  * MLA: Hkv = 1, d_k = 576, d_v = 512, Hq = 128, r in {16, 32, 64}; V may alias K.
+ * An E4M3 Kp needs r >= 16 (rows of at least 16 bytes).
  * Q, P, K, V and Kp base pointers and the K/V/Kp strides (except the unit inner
- * stride) must be multiples of 16 bytes.
+ * stride) must be multiples of 16 bytes.  A zero-initialised kp_dtype means bf16.
  */
 typedef struct {
   int32_t mode;      /* JSSA_MODE_GQA or JSSA_MODE_MLA                    */
@@ -110,6 +118,7 @@ typedef struct {
   int64_t k_stride[3];
   int64_t v_stride[3];
   int64_t kp_stride[3];
+  int32_t kp_dtype;  /* JSSA_KP_BF16 or JSSA_KP_FP8_E4M3                   */
 } jssa_layout;
 
 /* Human-readable name of a status code (static string). */
@@ -127,7 +136,8 @@ JSSA_API jssa_status jssa_workspace_size(const jssa_layout* L, int32_t k, int32_
 
 /*
  * Projected scoring cache on write (§3.1, §3.4, §E.1):
- *   Kp[b, h, t, :] = bf16(K[b, h, t, :] . P_h)   for t in [t_begin[b], t_begin[b] + n_tokens)
+ *   Kp[b, h, t, :] = rnd(K[b, h, t, :] . P_h)   for t in [t_begin[b], t_begin[b] + n_tokens)
+ * with rnd = bf16 or E4M3 (saturating) rounding to nearest even, by kp_dtype.
  * t_begin: device int32 [B] (rows past T_cap are skipped), or NULL to mean
  * t_begin[b] = seq_lens[b] - n_tokens (the last n_tokens rows; then seq_lens is
  * required).  n_tokens = 0 is a no-op.

@@ -223,6 +223,20 @@ def decode_head(Qg, K, V, Kp, P, T: int, k: int, W: int, scale: float):
     return dict(idx=idx[:k], k_eff=int(k_eff), O=O, lse=lse, scores=s[:T - Wc])
 
 
+def decode_head_e4m3(Qg, K, V, Kp8, P, T: int, k: int, W: int, scale: float):
+    """One decode step for one (sequence, KV head) problem over an FP8 E4M3 projected cache
+    (§A.3, §E.2: only the scoring cache is FP8; attention reads the bf16 rows).  The steps of
+    Figure 1 in order: projected group query, scores against the decoded codes, exact top-k,
+    attention over the selection plus the window [T-W, T).  Same return as decode_head."""
+    Wc = min(max(W, 0), T)
+    n = T - Wc
+    s = scores_e4m3(query_proj(Qg, P), np.asarray(Kp8, np.uint8)[:n])
+    idx, k_eff = topk(s, k)
+    toks = np.concatenate([idx[:k_eff].astype(np.int64), np.arange(n, T, dtype=np.int64)])
+    O, lse = attention(Qg, K, V, toks, scale)
+    return dict(idx=idx, k_eff=k_eff, O=O, lse=lse, scores=s)
+
+
 # --------------------------------------------------------------------------- whole tensors
 def project_cache(K: np.ndarray, P: np.ndarray, T: int | None = None) -> np.ndarray:
     """Kp for rows [0, T) of every (b, h) of a [B, Hkv, T_cap, d] cache; rows >= T stay 0."""

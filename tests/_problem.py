@@ -8,7 +8,7 @@ import numpy as np
 import torch
 
 import oracle
-from tests._util import u16, f32, rel_l2
+from tests._util import u16, u8, f32, rel_l2
 import token_level_sparse_jssa_b200 as jssa
 from token_level_sparse_jssa_b200 import synth
 
@@ -24,7 +24,7 @@ class Problem:
     """Device caches (K, V, Kp, Q, P, seq_lens) of one workload plus its layout."""
 
     def __init__(self, w: synth.Workload, T_cap=None, seq_lens=None, out_dtype=jssa.OUT_F32, device="cuda",
-                 gen_device="cuda", seed=None):
+                 gen_device="cuda", seed=None, kp_fp8=False):
         self.w = w
         x = synth.make_inputs(w, device=gen_device, T_cap=T_cap, seq_lens=seq_lens, seed=seed)
         self.T_cap = x["T_cap"]
@@ -36,7 +36,9 @@ class Problem:
             self.V = x["V"].to(device)
         self.P = x["P"].to(device).contiguous()
         self.seq_lens = x["seq_lens"].to(device)
-        self.Kp = torch.zeros(w.B, w.Hkv, self.T_cap, w.r, dtype=torch.bfloat16, device=device)
+        self.kp_fp8 = kp_fp8
+        self.Kp = torch.zeros(w.B, w.Hkv, self.T_cap, w.r, dtype=torch.uint8 if kp_fp8 else torch.bfloat16,
+                              device=device)
         self.L = jssa.make_layout(self.K, self.V, self.Kp, w.Hq, w.r,
                                   jssa.MODE_MLA if w.mode == "mla" else jssa.MODE_GQA, out_dtype)
 
@@ -52,7 +54,11 @@ class Problem:
     def host(self, b, h):
         G = self.w.G
         return dict(Q=u16(self.Q[b, h * G:(h + 1) * G]), K=u16(self.K[b, h]), V=u16(self.V[b, h]),
-                    Kp=u16(self.Kp[b, h]), P=f32(self.P[h]))
+                    Kp=u8(self.Kp[b, h]) if self.kp_fp8 else u16(self.Kp[b, h]), P=f32(self.P[h]))
+
+    def project(self, K_rows, P):
+        """The oracle's scoring-cache rows for these key rows, in this problem's Kp type."""
+        return (oracle.project_rows_e4m3 if self.kp_fp8 else oracle.project_rows)(K_rows, P)[0]
 
 
 def check_selection(gpu_idx: np.ndarray, gpu_nsel: int, s: np.ndarray, k: int):
@@ -84,7 +90,8 @@ def check_attention(O_gpu: np.ndarray, O_ref: np.ndarray, what=""):
 def score_error_bound(Qg: np.ndarray, P: np.ndarray, Kp: np.ndarray) -> np.ndarray:
     """Rigorous bound on |fp32 score - exact score| for the GPU's evaluation order family:
     the group sum (G terms), the d-term projection and the r-term dot product, each in
-    fp32 with any summation order (gamma_n = n u / (1 - n u), u = 2^-24)."""
+    fp32 with any summation order (gamma_n = n u / (1 - n u), u = 2^-24).  Kp: bf16 codes
+    (uint16) or the decoded values (float64)."""
     u = 2.0 ** -24
     gam = lambda n: n * u / (1 - n * u)
     q = oracle.bf16_to_f64(Qg)                 # [G, d]
@@ -93,7 +100,7 @@ def score_error_bound(Qg: np.ndarray, P: np.ndarray, Kp: np.ndarray) -> np.ndarr
     qsum_abs = np.abs(q).sum(0)                # bound on |sum_g q| and on its rounding base
     qs_exact = P.astype(np.float64).T @ q.sum(0)
     err_qs = (gam(d) + gam(G) * (1 + gam(d))) * (absP.T @ qsum_abs)   # [r]
-    kp = oracle.bf16_to_f64(Kp)                # [n, r]
+    kp = oracle.bf16_to_f64(Kp) if Kp.dtype == np.uint16 else np.asarray(Kp, np.float64)   # [n, r]
     r = kp.shape[1]
     qs_abs = np.abs(qs_exact) + err_qs
     return gam(r) * (np.abs(kp) @ qs_abs) + np.abs(kp) @ err_qs
@@ -110,10 +117,11 @@ def check_step_rows(p: Problem, k: int, window: int, O, idx, nsel, rows, what=""
     for (b, h) in rows:
         T = int(p.seq_lens[b])
         hst = p.host(b, h)
-        Kp_or, _ = oracle.project_rows(hst["K"][:T], hst["P"])
+        Kp_or = p.project(hst["K"][:T], hst["P"])
         if kp_checked:  # the scoring cache the step read is the oracle's projection, bit for bit
             np.testing.assert_array_equal(hst["Kp"][:T], Kp_or)
-        res = oracle.decode_head(hst["Q"], hst["K"][:T], hst["V"][:T], Kp_or, hst["P"], T, k, window, w.sm_scale)
+        head = oracle.decode_head_e4m3 if p.kp_fp8 else oracle.decode_head
+        res = head(hst["Q"], hst["K"][:T], hst["V"][:T], Kp_or, hst["P"], T, k, window, w.sm_scale)
         g_idx = idx[b, h].cpu().numpy()
         _, same = check_selection(g_idx, int(nsel[b, h]), res["scores"], k)
         O_gpu = O[b, h * G:(h + 1) * G].float().cpu().numpy().astype(np.float64)

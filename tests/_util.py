@@ -9,6 +9,12 @@ def u16(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
+def u8(t: torch.Tensor) -> np.ndarray:
+    """uint8 / float8_e4m3fn tensor -> numpy uint8 codes (contiguous copy)."""
+    assert t.dtype in (torch.uint8, torch.float8_e4m3fn)
+    return t.detach().cpu().contiguous().view(torch.uint8).numpy()
+
+
 def f32(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().contiguous().to(torch.float32).numpy()
 

@@ -76,6 +76,7 @@ def _layout(**kw):
     L.mode, L.B, L.Hq, L.Hkv, L.d_k, L.d_v, L.r, L.out_dtype = kw.get("mode", 0), B, Hq, Hkv, d, kw.get("dv", d), r, \
         kw.get("out", 0)
     L.T_cap = T
+    L.kp_dtype = kw.get("kp", 0)
     for i, v in enumerate((Hkv * T * d, T * d, d)):
         L.k_stride[i] = v
         L.v_stride[i] = v
@@ -105,6 +106,9 @@ FAKE = 0x10000  # a 16-byte aligned non-null value; validation rejects the call 
     (dict(T=0), 1),
     (dict(k_stride=(8, 8, 100)), 1),  # stride not a multiple of 16 bytes
     (dict(kp_stride=(0, 0, 64)), 2),  # Kp rows must be contiguous
+    (dict(kp=2), 1),                  # unknown Kp storage type
+    (dict(kp=1, r=8, d=64), 2),       # E4M3 rows of 8 bytes
+    (dict(kp=1, r=16, kp_stride=(24, 24, 16)), 1),  # E4M3 strides must be multiples of 16 bytes
 ])
 def test_bad_layouts_are_rejected_on_the_host(lib, kw, code):
     L = _layout(**kw)

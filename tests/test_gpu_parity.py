@@ -410,7 +410,9 @@ def test_select_matches_the_oracle_selection(name, kw, seq, window):
         T = int(p.seq_lens[b])
         for h in range(w.Hkv):
             hst = p.host(b, h)
-            res = oracle.decode_head(hst["Q"], hst["K"][:T], hst["V"][:T], hst["Kp"][:T], hst["P"], T, w.k, window,
+            Kp_or = p.project(hst["K"][:T], hst["P"])   # the oracle's own cache; the GPU's must equal it
+            np.testing.assert_array_equal(hst["Kp"][:T], Kp_or)
+            res = oracle.decode_head(hst["Q"], hst["K"][:T], hst["V"][:T], Kp_or, hst["P"], T, w.k, window,
                                      w.sm_scale)
             check_selection(idx[b, h].cpu().numpy(), int(nsel[b, h]), res["scores"], w.k)
     _assert_status_clean(ws)

@@ -408,3 +408,23 @@ def test_e4m3_projection_is_the_rounded_exact_product():
     qs = rng.standard_normal(r)
     vals = np.vectorize(oracle.e4m3_to_double)(Kp8)
     np.testing.assert_allclose(oracle.scores_e4m3(qs, Kp8), vals @ qs, rtol=1e-13)
+
+
+def test_e4m3_decode_head_equals_the_bf16_step_on_the_same_values():
+    # every finite E4M3 value is exactly a bf16 value, so the FP8 step on codes c must equal the
+    # bf16 step (the C decode_head) on bf16(value(c)): same scores, selection and output
+    rng = np.random.default_rng(11)
+    G, d, r, T, k, W = 4, 32, 16, 300, 20, 16
+    bf = lambda a: oracle.bf16_round(np.asarray(a, np.float64))
+    Qg, K, V = bf(rng.standard_normal((G, d))), bf(rng.standard_normal((T, d))), bf(rng.standard_normal((T, d)))
+    P = np.linalg.qr(rng.standard_normal((d, r)))[0].astype(np.float32)
+    codes = rng.integers(0, 256, (T, r)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x38                    # no NaN codes
+    vals = np.vectorize(oracle.e4m3_to_double)(codes)
+    a = oracle.decode_head_e4m3(Qg, K, V, codes, P, T, k, W, 0.125)
+    b = oracle.decode_head(Qg, K, V, bf(vals), P, T, k, W, 0.125)
+    np.testing.assert_array_equal(a["scores"], b["scores"])
+    assert a["k_eff"] == b["k_eff"] == k
+    np.testing.assert_array_equal(a["idx"], b["idx"])
+    np.testing.assert_allclose(a["O"], b["O"], rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(a["lse"], b["lse"], rtol=1e-13)

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libjssa.so")
 
 MODE_GQA, MODE_MLA = 0, 1
 OUT_F32, OUT_BF16 = 0, 1
+KP_BF16, KP_FP8_E4M3 = 0, 1
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape or mode", 3: "workspace missing, misaligned or too small",
           4: "CUDA error", 5: "device-side check failed", 6: "bounded wait timed out",
@@ -39,7 +40,7 @@ class Layout(C.Structure):
     _fields_ = [("mode", C.c_int32), ("B", C.c_int32), ("Hq", C.c_int32), ("Hkv", C.c_int32),
                 ("d_k", C.c_int32), ("d_v", C.c_int32), ("r", C.c_int32), ("out_dtype", C.c_int32),
                 ("T_cap", C.c_int64), ("k_stride", C.c_int64 * 3), ("v_stride", C.c_int64 * 3),
-                ("kp_stride", C.c_int64 * 3)]
+                ("kp_stride", C.c_int64 * 3), ("kp_dtype", C.c_int32)]
 
 
 _lib = None
@@ -118,12 +119,19 @@ def _ws(ws):
 def make_layout(K: torch.Tensor, V: torch.Tensor, Kp: torch.Tensor, Hq: int, r: int, mode: int = MODE_GQA,
                 out_dtype: int = OUT_F32) -> Layout:
     """Layout from 4-D caches K [B, Hkv, T_cap, d_k], V [B, Hkv, T_cap, d_v] and
-    Kp [B, Hkv, T_cap, r] (any strides with a contiguous last dimension)."""
+    Kp [B, Hkv, T_cap, r] (any strides with a contiguous last dimension).  A Kp of
+    dtype bfloat16 is a bf16 cache; float8_e4m3fn or uint8 (the raw codes) an E4M3 one."""
     B, Hkv, T_cap, d_k = K.shape
     L = Layout()
     L.mode, L.B, L.Hq, L.Hkv = mode, B, Hq, Hkv
     L.d_k, L.d_v, L.r, L.out_dtype = d_k, V.shape[-1], r, out_dtype
     L.T_cap = T_cap
+    if Kp.dtype == torch.bfloat16:
+        L.kp_dtype = KP_BF16
+    elif Kp.dtype in (torch.float8_e4m3fn, torch.uint8):
+        L.kp_dtype = KP_FP8_E4M3
+    else:
+        raise TypeError(f"Kp must be bfloat16, float8_e4m3fn or uint8, not {Kp.dtype}")
     for i in range(3):
         L.k_stride[i] = K.stride(i)
         L.v_stride[i] = V.stride(i)

@@ -43,10 +43,14 @@ jssa_status check_layout(const jssa_layout* L) {
   if (L->Hq % L->Hkv != 0) return JSSA_ERR_INVALID_ARG;
   if (L->r > L->d_k || L->d_v > L->d_k) return JSSA_ERR_INVALID_ARG;
   if (L->out_dtype != JSSA_OUT_F32 && L->out_dtype != JSSA_OUT_BF16) return JSSA_ERR_INVALID_ARG;
+  if (L->kp_dtype != JSSA_KP_BF16 && L->kp_dtype != JSSA_KP_FP8_E4M3) return JSSA_ERR_INVALID_ARG;
+  if (L->kp_dtype == JSSA_KP_FP8_E4M3 && L->r < 16) return JSSA_ERR_UNSUPPORTED;  // rows under 16 bytes
+  const int64_t kp_align = (L->kp_dtype == JSSA_KP_FP8_E4M3) ? 16 : 8;  // elements per 16 bytes
   if (L->B > 1024) return JSSA_ERR_UNSUPPORTED;
   for (int i = 0; i < 3; ++i) {
     if (L->k_stride[i] < 0 || L->v_stride[i] < 0 || L->kp_stride[i] < 0) return JSSA_ERR_INVALID_ARG;
-    if (L->k_stride[i] % 8 || L->v_stride[i] % 8 || L->kp_stride[i] % 8) return JSSA_ERR_INVALID_ARG;
+    if (L->k_stride[i] % 8 || L->v_stride[i] % 8) return JSSA_ERR_INVALID_ARG;
+    if (L->kp_stride[i] % kp_align) return JSSA_ERR_INVALID_ARG;
   }
   if (L->k_stride[2] < L->d_k || L->v_stride[2] < L->d_v) return JSSA_ERR_INVALID_ARG;
   if (L->kp_stride[2] != L->r) return JSSA_ERR_UNSUPPORTED;  // Kp rows are streamed as one block
@@ -148,6 +152,7 @@ ProjectArgs project_args(const jssa_layout* L, const void* K, const float* P, vo
   a.P = P;
   a.Kp = Kp;
   memcpy(a.ps, L->kp_stride, sizeof a.ps);
+  a.kp_fp8 = (L->kp_dtype == JSSA_KP_FP8_E4M3);
   a.t_begin = t_begin;
   a.seq_lens = seq_lens;
   a.n_tokens = n;
@@ -170,6 +175,7 @@ jssa_status run_prologue(const jssa_layout* L, const void* Q, const float* P, co
   memcpy(q.ks, L->k_stride, sizeof q.ks);
   q.Kp = Kp;
   memcpy(q.ps, L->kp_stride, sizeof q.ps);
+  q.kp_fp8 = (L->kp_dtype == JSSA_KP_FP8_E4M3);
   q.seq_lens = seq_lens;
   q.counters = w.counters;
   q.n_new = n_new;
@@ -188,6 +194,7 @@ jssa_status run_score(const jssa_layout* L, const void* Kp, const int32_t* seq_l
   ScoreArgs a{};
   a.Kp = Kp;
   memcpy(a.ps, L->kp_stride, sizeof a.ps);
+  a.kp_fp8 = (L->kp_dtype == JSSA_KP_FP8_E4M3);
   a.qs = w.qs;
   a.scores = scores;
   a.sc_ld = sc_ld;
@@ -302,6 +309,7 @@ jssa_status run_select(const jssa_layout* L, const void* Q, const void* K, void*
     memcpy(sa.ks, L->k_stride, sizeof sa.ks);
     sa.Kp = Kp;
     memcpy(sa.ps, L->kp_stride, sizeof sa.ps);
+    sa.kp_fp8 = (L->kp_dtype == JSSA_KP_FP8_E4M3);
     sa.seq_lens = seq_lens;
     sa.n_new = n_in;
     sa.B = L->B;
@@ -362,7 +370,7 @@ const char* jssa_status_string(jssa_status s) {
   return "unknown status";
 }
 
-int32_t jssa_version(void) { return 10000; }
+int32_t jssa_version(void) { return 10100; }
 
 jssa_status jssa_workspace_size(const jssa_layout* L, int32_t k, int32_t window, size_t* bytes) {
   jssa_status st = check_layout(L);

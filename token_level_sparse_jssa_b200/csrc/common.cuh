@@ -9,6 +9,8 @@
 #include <cstdint>
 #include <utility>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 namespace jssa {
@@ -163,6 +165,77 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
   }
   const double q = rint(__longlong_as_double(static_cast<long long>(a)) * 0x1p133);  // whole quanta of 2^-133
   return uint16_t(sign | static_cast<uint16_t>(q));
+}
+
+// fp64 -> FP8 E4M3 (the OCP format: bias 7, 3 fraction bits, subnormals in steps of
+// 2^-9, largest finite 448 = 0x7E, 0x7F NaN), nearest with ties to even, saturated to
+// +-448 (infinities too).  Worked on the bits of the double: a result of 2^-6 or more keeps
+// the exponent and the top 3 fraction bits and rounds on the 49 bits below (a carry out of
+// the fraction steps the exponent, which is the right code); a smaller one counts whole
+// 2^-9 quanta (a count of 8 is the code of 2^-6).
+__device__ __forceinline__ uint8_t f64_to_e4m3_rne_sat(double x) {
+  const unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(x));
+  const uint8_t sign = static_cast<uint8_t>((u >> 56) & 0x80u);
+  const unsigned long long a = u & 0x7FFFFFFFFFFFFFFFull;
+  if (a > 0x7FF0000000000000ull) return static_cast<uint8_t>(sign | 0x7Fu);   // NaN
+  if (a >= 0x407C000000000000ull) return static_cast<uint8_t>(sign | 0x7Eu);  // |x| >= 448
+  const int e = static_cast<int>(a >> 52) - 1023;
+  const unsigned long long m = (a & ((1ull << 52) - 1)) | (1ull << 52);
+  if (e >= -6) {
+    const unsigned long long rem = m & ((1ull << 49) - 1), half = 1ull << 48;
+    const uint32_t f = static_cast<uint32_t>(m >> 49) & 7u;
+    uint32_t code = (static_cast<uint32_t>(e + 7) << 3) | f;
+    if (rem > half || (rem == half && (f & 1u))) code += 1;
+    return static_cast<uint8_t>(sign | code);
+  }
+  const int sh = 43 - e;  // |x| / 2^-9 = m * 2^-sh
+  if (sh >= 54) return sign;  // |x| <= 2^-10: rounds to zero (2^-10 itself is a tie to 0)
+  uint32_t q = static_cast<uint32_t>(m >> sh);
+  const unsigned long long rem = m & ((1ull << sh) - 1), half = 1ull << (sh - 1);
+  if (rem > half || (rem == half && (q & 1u))) q += 1;
+  return static_cast<uint8_t>(sign | q);
+}
+
+// Rotation of a scan thread's 16-byte Kp vectors: VPT vectors per thread, read in the order
+// (j + rot) % VPT, so that each 8-thread phase of a 16-byte shared-memory load covers 8
+// different 16-byte bank groups for every row size the scans use (rows of 1, 2, 4 or 8
+// vectors with one or two threads per token).
+template <int VPT>
+__device__ __forceinline__ int kp_vector_rotation(int tid) {
+  if constexpr (VPT == 1) return 0;
+  else if constexpr (VPT == 2) return (tid >> 2) & 1;
+  else return (tid >> 1) & 3;
+}
+
+// Dot product of one 16-byte vector of a projected-key row with the matching slice of the
+// projected query (fp32), the products added in element order.  bf16: 8 elements, widened by
+// a shift.  E4M3: 16 elements (element 0 in the lowest byte), each pair widened exactly to
+// f16x2 by the hardware conversion and then to fp32.
+template <bool F8>
+__device__ __forceinline__ float kp_vector_dot(const float* q, uint4 raw) {
+  if constexpr (!F8) {
+    float x = q[0] * __uint_as_float(raw.x << 16);
+    x = fmaf(q[1], __uint_as_float(raw.x & 0xFFFF0000u), x);
+    x = fmaf(q[2], __uint_as_float(raw.y << 16), x);
+    x = fmaf(q[3], __uint_as_float(raw.y & 0xFFFF0000u), x);
+    x = fmaf(q[4], __uint_as_float(raw.z << 16), x);
+    x = fmaf(q[5], __uint_as_float(raw.z & 0xFFFF0000u), x);
+    x = fmaf(q[6], __uint_as_float(raw.w << 16), x);
+    x = fmaf(q[7], __uint_as_float(raw.w & 0xFFFF0000u), x);
+    return x;
+  } else {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    float x = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>((w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu), __NV_E4M3);
+      const float2 f = __half22float2(__half2(hr));
+      x = (i == 0) ? q[0] * f.x : fmaf(q[2 * i], f.x, x);
+      x = fmaf(q[2 * i + 1], f.y, x);
+    }
+    return x;
+  }
 }
 
 // Order-preserving map of an fp32 value to uint32 (larger value -> larger key);

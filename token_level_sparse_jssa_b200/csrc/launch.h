@@ -13,6 +13,7 @@ struct ProjectArgs {
   const float* P;
   void* Kp;
   int64_t ps[3];
+  int kp_fp8;               // Kp elements are E4M3 bytes (else bf16)
   const int32_t* t_begin;   // nullable: then seq_lens[b] - n_tokens
   const int32_t* seq_lens;
   int64_t n_tokens;
@@ -32,6 +33,7 @@ struct PrologueArgs {
   int64_t ks[3];
   void* Kp;
   int64_t ps[3];
+  int kp_fp8;       // Kp elements are E4M3 bytes (else bf16)
   const int32_t* seq_lens;
   int* counters;    // nullable: [B*Hkv] attention arrival counters zeroed here
   int n_new;
@@ -44,6 +46,7 @@ cudaError_t launch_step_prologue(const PrologueArgs& a, cudaStream_t s);
 struct ScoreArgs {
   const void* Kp;
   int64_t ps[3];
+  int kp_fp8;        // Kp elements are E4M3 bytes (else bf16)
   const float* qs;   // [B*Hkv, r] projected group queries (from the step prologue)
   float* scores;     // [B*Hkv, sc_ld]
   int64_t sc_ld;
@@ -109,6 +112,7 @@ struct SelectArgs {
   int64_t ks[3];
   void* Kp;
   int64_t ps[3];
+  int kp_fp8;        // Kp elements are E4M3 bytes (else bf16)
   const int32_t* seq_lens;
   int n_new;         // <= select_max_new_rows()
   int B, Hq, Hkv, d, r;
@@ -129,6 +133,7 @@ struct SelectArgs {
   int out_bf16;
 };
 cudaError_t launch_select(const SelectArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_select_fp8(const SelectArgs& a, int num_sms, cudaStream_t s);  // E4M3 Kp, r >= 16
 int64_t select_max_candidates();
 int select_max_new_rows();
 

@@ -5,9 +5,10 @@
 // (one basis for queries and keys) and §E.1 (the newly generated key is projected on
 // write; at most 3.2 % of the step).
 //
-// Kp[t] = bf16(K[t] . P_h): the products K[t,i] * P[i,j] (bf16 x fp32) are exact in
-// fp64 and are accumulated in fp64, then rounded once to bf16 (nearest, ties to
-// even), so the stored cache equals the rounding of the exact product except when
+// Kp[t] = rnd(K[t] . P_h): the products K[t,i] * P[i,j] (bf16 x fp32) are exact in fp64
+// and are accumulated in fp64, then rounded once to the cache's type (bf16, or FP8 E4M3
+// saturated to +-448 as in the paper's deployed scoring cache, §A.3 and §E.2; nearest,
+// ties to even), so the stored cache equals the rounding of the exact product except when
 // that product lies within about 1e-16 relative of a rounding midpoint.
 //
 // Two kernels:
@@ -29,6 +30,12 @@ __device__ __forceinline__ void stage_basis(float* Psm, const float* Ph, int n) 
   const float4* src = reinterpret_cast<const float4*>(Ph);
   float4* dst = reinterpret_cast<float4*>(Psm);
   for (int i = threadIdx.x; i < n / 4; i += blockDim.x) dst[i] = __ldg(src + i);
+}
+
+// Store one projected value, rounded to the cache's element type, at element offset `off`.
+__device__ __forceinline__ void store_kp(void* Kp, int fp8, int64_t off, double v) {
+  if (fp8) static_cast<uint8_t*>(Kp)[off] = f64_to_e4m3_rne_sat(v);
+  else static_cast<uint16_t*>(Kp)[off] = f64_to_bf16_rne(v);
 }
 
 constexpr int kProjRows = 32;     // rows of K per CTA
@@ -79,12 +86,12 @@ __global__ void __launch_bounds__(kProjThreads) project_keys_kernel(ProjectArgs 
     for (int q = 0; q < kMaxRowsPerThread; ++q)
       if (q < my_rows) acc[q] = fma(static_cast<double>(__bfloat162float(krows[(g + q * groups) * d + i])), p, acc[q]);
   }
-  __nv_bfloat16* Kpb = static_cast<__nv_bfloat16*>(a.Kp) + b * a.ps[0] + h * a.ps[1];
+  const int64_t kp0 = b * a.ps[0] + h * a.ps[1];
 #pragma unroll
   for (int q = 0; q < kMaxRowsPerThread; ++q) {
     if (q < my_rows) {
       const int64_t t = tb + row0 + g + q * groups;
-      if (t >= 0 && t < a.T_cap) reinterpret_cast<uint16_t*>(Kpb)[t * a.ps[2] + j] = f64_to_bf16_rne(acc[q]);
+      if (t >= 0 && t < a.T_cap) store_kp(a.Kp, a.kp_fp8, kp0 + t * a.ps[2] + j, acc[q]);
     }
   }
 }
@@ -186,7 +193,7 @@ __global__ void __launch_bounds__(kPrologueThreads) step_prologue_kernel(Prologu
   __syncthreads();
   ok = mbar_wait_bounded(&bars[1], 0, a.status) && ok;
   const int64_t t0 = tb_s;
-  uint16_t* Kpb = reinterpret_cast<uint16_t*>(a.Kp) + b * a.ps[0] + h * a.ps[1];
+  const int64_t kp0 = b * a.ps[0] + h * a.ps[1];
   for (int64_t t = t0; t < t0 + n_new; ++t) {
     int64_t T = a.seq_lens[b];
     T = T < 0 ? 0 : (T > a.T_cap ? a.T_cap : T);
@@ -200,7 +207,7 @@ __global__ void __launch_bounds__(kPrologueThreads) step_prologue_kernel(Prologu
     if (tid < r && ok) {
       double t2 = 0.0;
       for (int q = 0; q < parts; ++q) t2 += red[q * r + tid];
-      Kpb[t * a.ps[2] + tid] = f64_to_bf16_rne(t2);
+      store_kp(a.Kp, a.kp_fp8, kp0 + t * a.ps[2] + tid, t2);
     }
     __syncthreads();
   }

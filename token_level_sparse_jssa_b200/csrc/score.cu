@@ -12,7 +12,7 @@
 // a shared-memory histogram per CTA, flushed to the row's global histogram with one
 // atomic add per non-zero bin whenever the CTA moves to another row.
 //
-// The scan is HBM-bound (r*2 bytes read and 4 bytes written per token).  A persistent
+// The scan is HBM-bound (r*2 bytes of bf16 Kp, or r of E4M3, read and 4 bytes written per token).  A persistent
 // grid walks the flattened (row, token) space in 16 KB chunks, each CTA a contiguous
 // range of chunks.  One producer warp streams chunks into a shared-memory ring with
 // 1-D bulk copies (TMA engine, L2 evict-first) and full/empty mbarrier pairs; eight
@@ -56,12 +56,15 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-template <int R>
+template <int R, bool F8>
 __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
-  constexpr int CH = kChunkBytes / (R * 2);           // tokens per chunk
-  constexpr int V = R / 8;                            // 16-byte vectors per token
+  constexpr int EB = F8 ? 1 : 2;                      // bytes per Kp element (E4M3 or bf16)
+  constexpr int EPV = 16 / EB;                        // Kp elements per 16-byte vector
+  constexpr int CH = kChunkBytes / (R * EB);          // tokens per chunk
+  constexpr int V = R * EB / 16;                      // 16-byte vectors per token
   constexpr int TPT = (R >= 64) ? 2 : 1;              // threads per token
   constexpr int VPT = V / TPT;                        // vectors per thread (<= 4)
+  static_assert(V >= 1 && V % TPT == 0, "Kp rows of at least 16 bytes");
   constexpr int TOK_PER_PASS = kScoreConsumers / TPT;
   constexpr int PASSES = CH / TOK_PER_PASS;
   static_assert(PASSES >= 1 && CH % TOK_PER_PASS == 0, "chunk / thread mapping");
@@ -124,7 +127,7 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
   if (producer) {
     if ((tid & 31) == 0) {
       const uint64_t policy = l2_policy_evict_first();
-      const __nv_bfloat16* Kp = static_cast<const __nv_bfloat16*>(a.Kp);
+      const unsigned char* Kp = static_cast<const unsigned char*>(a.Kp);
       ChunkIter c = it0;
       for (int64_t it = 0; it < n_mine; ++it) {
         const int s = static_cast<int>(it % kScoreStages);
@@ -135,9 +138,9 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
         }
         const int64_t t0 = c.ci * CH;
         const uint32_t cnt = static_cast<uint32_t>(min64(CH, nb[c.b] - t0));
-        const __nv_bfloat16* src = Kp + c.b * a.ps[0] + c.h * a.ps[1] + t0 * a.ps[2];
-        mbar_arrive_expect_tx(&full[s], cnt * R * 2);
-        bulk_g2s(ring + s * kChunkBytes, src, cnt * R * 2, &full[s], policy);
+        const unsigned char* src = Kp + (c.b * a.ps[0] + c.h * a.ps[1] + t0 * a.ps[2]) * EB;
+        mbar_arrive_expect_tx(&full[s], cnt * R * EB);
+        bulk_g2s(ring + s * kChunkBytes, src, cnt * R * EB, &full[s], policy);
         chunk_advance(c, per_head, a.B, a.Hkv);
       }
     }
@@ -152,8 +155,8 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
     // this thread's token within a pass, its slice of the token and its rotation
     const int sub = (TPT == 2) ? (tid & 1) : 0;
     const int tok_in_pass = tid / TPT;
-    const int rot = (V == 1) ? 0 : (TPT == 2 ? ((tid >> 1) & 3) : ((tid >> (V == 2 ? 2 : 1)) & (V - 1)));
-    float q[VPT][8];
+    const int rot = kp_vector_rotation<VPT>(tid);
+    float q[VPT][EPV];
     ChunkIter c = it0;
     int cur_row = -1;
     bool dead = false;  // a wait gave up: keep the loop's barrier structure, skip the work
@@ -176,10 +179,12 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
         const float* qsrc = (row - row0 < kQRows) ? qtab + (row - row0) * R : a.qs + static_cast<int64_t>(row) * R;
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
-          const float4* qp = reinterpret_cast<const float4*>(qsrc + (sub * VPT + (j + rot) % VPT) * 8);
-          const float4 q0 = qp[0], q1 = qp[1];
-          q[j][0] = q0.x; q[j][1] = q0.y; q[j][2] = q0.z; q[j][3] = q0.w;
-          q[j][4] = q1.x; q[j][5] = q1.y; q[j][6] = q1.z; q[j][7] = q1.w;
+          const float4* qp = reinterpret_cast<const float4*>(qsrc + (sub * VPT + (j + rot) % VPT) * EPV);
+#pragma unroll
+          for (int u = 0; u < EPV / 4; ++u) {
+            const float4 q4 = qp[u];
+            q[j][4 * u] = q4.x; q[j][4 * u + 1] = q4.y; q[j][4 * u + 2] = q4.z; q[j][4 * u + 3] = q4.w;
+          }
         }
       }
       if (!dead && !mbar_wait_bounded(&full[s], static_cast<uint32_t>((it / kScoreStages) & 1), a.status)) {
@@ -194,20 +199,12 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
 #pragma unroll
         for (int p = 0; p < PASSES; ++p) {
           const int tok = p * TOK_PER_PASS + tok_in_pass;
-          const unsigned char* trow = buf + tok * (R * 2);
+          const unsigned char* trow = buf + tok * (R * EB);
           float acc[VPT];
 #pragma unroll
           for (int j = 0; j < VPT; ++j) {
             const uint4 raw = *reinterpret_cast<const uint4*>(trow + (sub * VPT + (j + rot) % VPT) * 16);
-            float x = q[j][0] * __uint_as_float(raw.x << 16);
-            x = fmaf(q[j][1], __uint_as_float(raw.x & 0xFFFF0000u), x);
-            x = fmaf(q[j][2], __uint_as_float(raw.y << 16), x);
-            x = fmaf(q[j][3], __uint_as_float(raw.y & 0xFFFF0000u), x);
-            x = fmaf(q[j][4], __uint_as_float(raw.z << 16), x);
-            x = fmaf(q[j][5], __uint_as_float(raw.z & 0xFFFF0000u), x);
-            x = fmaf(q[j][6], __uint_as_float(raw.w << 16), x);
-            x = fmaf(q[j][7], __uint_as_float(raw.w & 0xFFFF0000u), x);
-            acc[j] = x;
+            acc[j] = kp_vector_dot<F8>(q[j], raw);
           }
           float sc = acc[0];
 #pragma unroll
@@ -241,24 +238,32 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
   }
 }
 
-template <int R>
+template <int R, bool F8>
 static cudaError_t launch_score_r(const ScoreArgs& a, int num_sms, cudaStream_t s) {
   const size_t smem = kScoreStages * kChunkBytes + 2 * kScoreStages * sizeof(uint64_t) +
                       kHistBins * sizeof(uint32_t) + kQRows * R * sizeof(float) + (3 * a.B + 1) * sizeof(int64_t);
   static int done[64] = {0};
-  cudaError_t e = set_smem_limit_once(score_kernel<R>, smem, done);
+  cudaError_t e = set_smem_limit_once(score_kernel<R, F8>, smem, done);
   if (e != cudaSuccess) return e;
   const int grid = num_sms * 3;
-  return launch_ex(score_kernel<R>, dim3(grid), dim3(kScoreThreads), smem, s, 0, a);
+  return launch_ex(score_kernel<R, F8>, dim3(grid), dim3(kScoreThreads), smem, s, 0, a);
 }
 
 cudaError_t launch_score(const ScoreArgs& a, int num_sms, cudaStream_t s) {
   if (a.B > kMaxBatch) return cudaErrorInvalidValue;
+  if (a.kp_fp8) {
+    switch (a.r) {  // E4M3 rows of at least 16 bytes
+      case 16: return launch_score_r<16, true>(a, num_sms, s);
+      case 32: return launch_score_r<32, true>(a, num_sms, s);
+      case 64: return launch_score_r<64, true>(a, num_sms, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (a.r) {
-    case 8: return launch_score_r<8>(a, num_sms, s);
-    case 16: return launch_score_r<16>(a, num_sms, s);
-    case 32: return launch_score_r<32>(a, num_sms, s);
-    case 64: return launch_score_r<64>(a, num_sms, s);
+    case 8: return launch_score_r<8, false>(a, num_sms, s);
+    case 16: return launch_score_r<16, false>(a, num_sms, s);
+    case 32: return launch_score_r<32, false>(a, num_sms, s);
+    case 64: return launch_score_r<64, false>(a, num_sms, s);
     default: return cudaErrorInvalidValue;
   }
 }
