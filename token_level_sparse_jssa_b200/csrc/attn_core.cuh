@@ -122,44 +122,41 @@ __device__ __forceinline__ void finish_split(const AttnArgs& a, int row, int64_t
 
 // Split merge inside a thread-block cluster (one CTA per split of the row, S <= 16):
 // every CTA keeps its normalised partial (o, lse) in its own shared memory; after a
-// cluster barrier CTA c combines output slice c of the row, reading the S partials
-// through distributed shared memory, and a second barrier keeps the partials alive
-// until every CTA has read them.
+// cluster barrier CTA c combines output slice c of the row.  Each thread reads, in one
+// round of distributed-shared-memory loads, the S partials of its element and the S
+// log-sum-exps of its head, forms the weights itself and writes the element (and the
+// head's lse, from the thread of the head's first element).  A second barrier keeps the
+// partials alive until every CTA has read them.
 template <int D>
 __device__ __forceinline__ void cluster_merge(const AttnArgs& a, int64_t hq0, int G, const float* pbuf,
                                               const float* plse) {
-  __shared__ float wts[16 * 16];
   cg::cluster_group cl = cg::this_cluster();
   const int S = static_cast<int>(cl.num_blocks());
   const int c = static_cast<int>(cl.block_rank());
   cl.sync();
-  for (int i = threadIdx.x; i < G * S; i += blockDim.x) wts[i] = cl.map_shared_rank(plse, i % S)[i / S];
-  __syncthreads();
-  if (threadIdx.x < G) {
-    float* w = wts + threadIdx.x * S;
-    float M = -INFINITY;
-    for (int q = 0; q < S; ++q) M = fmaxf(M, w[q]);
-    float L = 0.f;
-    for (int q = 0; q < S; ++q) {
-      w[q] = (M == -INFINITY) ? 0.f : expf(w[q] - M);
-      L += w[q];
-    }
-    for (int q = 0; q < S; ++q) w[q] = (L > 0.f) ? w[q] / L : 0.f;
-    if (a.lse && c == 0) a.lse[hq0 + threadIdx.x] = (M == -INFINITY) ? -INFINITY : M + logf(L);
-  }
-  __syncthreads();
   const int per = (G * D + S - 1) / S;
   const int lo = c * per, hi = min(G * D, lo + per);
   for (int i = lo + threadIdx.x; i < hi; i += blockDim.x) {
     const int head = i / D;
-    float v[16];
+    float v[16], l[16];
 #pragma unroll
-    for (int q = 0; q < 16; ++q) v[q] = (q < S) ? cl.map_shared_rank(pbuf, q)[i] : 0.f;
-    float o = 0.f;
+    for (int q = 0; q < 16; ++q) {  // all remote loads in flight before the first use
+      v[q] = (q < S) ? cl.map_shared_rank(pbuf, q)[i] : 0.f;
+      l[q] = (q < S) ? cl.map_shared_rank(plse, q)[head] : -INFINITY;
+    }
+    float M = -INFINITY;
 #pragma unroll
-    for (int q = 0; q < 16; ++q)
-      if (q < S) o = fmaf(wts[head * S + q], v[q], o);
+    for (int q = 0; q < 16; ++q) M = fmaxf(M, l[q]);
+    float L = 0.f, o = 0.f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const float w = (M == -INFINITY || q >= S) ? 0.f : expf(l[q] - M);
+      L += w;
+      o = fmaf(w, v[q], o);
+    }
+    o = (L > 0.f) ? o / L : 0.f;
     const int64_t qi = hq0 + head;
+    if (a.lse && i % D == 0) a.lse[qi] = (M == -INFINITY) ? -INFINITY : M + logf(L);
     if (a.out_bf16) static_cast<__nv_bfloat16*>(a.O)[qi * D + (i % D)] = __float2bfloat16_rn(o);
     else static_cast<float*>(a.O)[qi * D + (i % D)] = o;
   }
