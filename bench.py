@@ -184,6 +184,7 @@ class Setup:
         self.P = x["P"].contiguous()
         self.seq_lens = x["seq_lens"]
         self.A = x["A"]
+        self.T_cap = x["T_cap"]
         self.Kp, self.L = self.scoring_cache(kp)
         self.kp = kp
         self.ws = jssa.alloc_workspace(self.L, w.k, w.window)
@@ -243,13 +244,17 @@ def stage_times(st, Q, reps=50):
     half of the step (projections, score scan, top-k: one kernel when the cache fits a
     cluster); attention = indexed attention with its merge; dense = the full-KV comparator;
     gather_then_attend = the same attention done the gather-based way (copy, then dense);
-    step_other_kp = the whole step over the other scoring-cache type (E4M3 when the run is bf16)."""
+    step_other_kp = the whole step over the other scoring-cache type (E4M3 when the run is bf16);
+    vote_select = the head-shared soft-voting selection."""
     jssa, w = st.jssa, st.w
     calls = {
         "select_us": lambda: jssa.select(st.L, Q, st.K, st.Kp, st.P, st.seq_lens, 1, w.k, w.window, st.idx,
                                          st.nsel, st.ws),
         "attention_us": lambda: jssa.indexed_attn(st.L, Q, st.K, st.V, st.idx, w.k, st.nsel, st.seq_lens,
                                                   w.window, w.sm_scale, st.O, None, st.ws),
+        # the head-shared soft-voting variant of the selection (unfused kernels)
+        "vote_select_us": lambda: jssa.vote_select(st.L, Q, st.K, st.Kp, st.P, st.seq_lens, 1, w.k, w.window,
+                                                   w.sm_scale, st.idx, st.nsel, st.ws),
     }
     if st.w.mode != "mla":  # the MLA path is indexed only
         calls["dense_us"] = lambda: st.dense(Q)
@@ -271,6 +276,54 @@ def stage_times(st, Q, reps=50):
         del g
     del Kp2
     return out
+
+
+# --------------------------------------------------------------------------- basis calibration
+def calibration_leg(st, reps=3):
+    """Offline calibration of the basis (jssa_calibrate) on calibration queries drawn with the
+    workload's recipe at n positions of every sequence, timed with CUDA events (best of
+    `reps`), and the selection quality it buys: the fraction of the exact full-dimensional
+    top-k (group-mean query . key over all candidates) that the selection contains, with the
+    calibrated basis and with the workload's random orthonormal basis, on two fresh queries."""
+    from token_level_sparse_jssa_b200 import synth
+    jssa, w = st.jssa, st.w
+    n = min(w.T, 32768) if w.mode != "mla" else 1024
+    Qc = synth.fresh_queries(w, n, st.A, device="cuda", seed=99).permute(1, 2, 0, 3).contiguous()
+    P = torch.empty_like(st.P)
+    ws = jssa.alloc_calibration_workspace(st.L)
+    jssa.calibrate(st.L, Qc, st.K, n, P, ws)
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        jssa.calibrate(st.L, Qc, st.K, n, P, ws)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    code, _ = jssa.read_device_status(ws)
+    del Qc, ws
+    Qs = synth.fresh_queries(w, 2, st.A, device="cuda", seed=98)
+    rec = {}
+    for name, basis in (("calibrated", P), ("random", st.P)):
+        Kp = torch.empty(w.B, w.Hkv, st.T_cap, w.r, dtype=torch.bfloat16, device="cuda")
+        L = jssa.make_layout(st.K, st.V, Kp, w.Hq, w.r, jssa.MODE_MLA if w.mode == "mla" else jssa.MODE_GQA,
+                             jssa.OUT_BF16)
+        jssa.project_keys(L, st.K, basis, Kp, st.T_cap, t_begin=torch.zeros(w.B, dtype=torch.int32, device="cuda"))
+        got = []
+        for Q in Qs:
+            jssa.select(L, Q, st.K, Kp, basis, st.seq_lens, 0, w.k, w.window, st.idx, st.nsel, st.ws)
+            n_cand = w.T - min(w.window, w.T)
+            qbar = Q.float().view(w.B, w.Hkv, w.G, w.dk).mean(2)
+            s = torch.einsum("bhd,bhtd->bht", qbar, st.K[:, :, :n_cand].float())
+            truth = torch.topk(s, min(w.k, n_cand), dim=2).indices
+            sel = torch.zeros_like(s, dtype=torch.bool).scatter_(2, st.idx.long().clamp(min=0), True)
+            got.append(sel.gather(2, truth).float().mean().item())
+            del s, sel
+        rec[name] = sum(got) / len(got)
+        del Kp
+    return {"calibration_ms": best, "calibration_tokens_per_head": w.B * n, "status": code,
+            "recall_at_k": rec}
 
 
 # --------------------------------------------------------------------------- CPU oracle timing
@@ -406,6 +459,7 @@ def main():
         del g_dw, g_d
 
     stages = stage_times(st, Qs[0])
+    calib = calibration_leg(st)
     hbm, peak_kind = peaks()
     n_kernels, fused = step_kernels(w)
     sel_bytes = bm["step"] if fused else bm["select"]
@@ -463,6 +517,7 @@ def main():
             "byte_ratio": bm["dense"] / bm["step"],
             "dense_hbm_frac": bm["dense"] / (dense_ms * 1e-3) / 1e9 / hbm if dense_ms else None,
             "stage_us": stages,
+            "calibration": calib,
             "roofline": {"kernel": ("select_kernel (the whole step: query and newest-key projection, score scan, "
                                     "top-k, attention, merge)") if fused else
                                    "select_kernel (query and newest-key projection, score scan, top-k)",

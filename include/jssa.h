@@ -216,6 +216,21 @@ JSSA_API jssa_status jssa_select(const jssa_layout* L, const void* Q, const void
                                  int32_t* n_sel, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Head-shared soft voting (§1, §E.3 / Table 15: the variant that per-KV-head selection is
+ * compared with; the vote is not defined on the pages, this is the library's reading):
+ * the same projections and score scan as jssa_select, then per (sequence, KV head) the
+ * distribution p_h(t) = softmax_t(c * s_h(t)) over the candidates [0, T_b - W) with
+ * c = sm_scale / G (the logit of the group-mean query), the vote v(t) = sum_h p_h(t), and
+ * the top-k of v (ties to the lower index, ascending, -1 padded) written to EVERY KV head's
+ * row of idx.  Runs the unfused kernels (score scan, vote statistics and combination,
+ * top-k, broadcast) for any T_cap.  Arguments as jssa_select, plus sm_scale > 0.
+ */
+JSSA_API jssa_status jssa_vote_select(const jssa_layout* L, const void* Q, const void* K, void* Kp, const float* P,
+                                      const int32_t* seq_lens, int32_t n_new, int32_t k, int32_t window,
+                                      float sm_scale, int32_t* idx, int32_t* n_sel, void* workspace, size_t ws_bytes,
+                                      void* stream);
+
+/*
  * One fused decode step (Figure 1): project the last n_new rows of each sequence
  * into Kp (n_new may be 0 when Kp is already current), score, select the top-k per
  * (sequence, KV head), attend over the selection (plus the window) and merge.
@@ -252,6 +267,28 @@ JSSA_API jssa_status jssa_gather_decode(const jssa_layout* L, const void* Q, con
 JSSA_API jssa_status jssa_dense_decode(const jssa_layout* L, const void* Q, const void* K, const void* V,
                               const int32_t* seq_lens, int32_t window, float sm_scale, void* O,
                               float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Spectral calibration of the basis (§3.2, §A.4, §B.1-§B.3; offline, once per layer):
+ *   P_h = the top-r eigenvectors of M_h = S_q / tr S_q + S_k / tr S_k, where
+ *   S_q = sum_t qbar_t qbar_t^T over the calibration tokens, qbar_t the mean of KV head h's
+ *   G query heads at token t, and S_k = sum_t k_t k_t^T (a moment with zero trace
+ *   contributes nothing).  This is the library's reading of the marginal bound's closed
+ *   form, which the summary does not print: Cauchy-Schwarz on the product of marginals
+ *   and the arithmetic-geometric mean of the two unit-trace residuals give the surrogate
+ *   2 - tr(P^T M P), minimised by those eigenvectors.
+ *   Qc  device bf16 [B, Hq, n_tokens, d_k], contiguous: the calibration queries;
+ *   K   the layout's key cache; rows [0, n_tokens) of every sequence (n_tokens <= T_cap);
+ *   P   device fp32 [Hkv, d_k, r] out: columns in descending eigenvalue order, each
+ *       column's largest-magnitude entry positive (lowest index on ties);
+ *   eigvals  device fp64 [Hkv, d_k] out (nullable): the eigenvalues of M_h, descending.
+ * Moments in fp64 (exact products of bf16), eigenvectors by cyclic Jacobi in fp64 (one
+ * 8-CTA cluster per KV head).  d_k must be a multiple of 64.  The workspace holds the
+ * status word: a diagonalisation that did not converge raises JSSA_DEV_TIMEOUT there.
+ */
+JSSA_API jssa_status jssa_calibrate_workspace_size(const jssa_layout* L, size_t* bytes);
+JSSA_API jssa_status jssa_calibrate(const jssa_layout* L, const void* Qc, const void* K, int64_t n_tokens,
+                                    float* P, double* eigvals, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Zero a freshly allocated workspace (asynchronously on `stream`): required once before

@@ -26,7 +26,8 @@ DEV_BAD_SEQ_LEN, DEV_BAD_INDEX, DEV_BAD_NSEL, DEV_TIMEOUT = 1, 2, 4, 8
 
 EXPORTS = ("jssa_status_string", "jssa_version", "jssa_workspace_size", "jssa_project_keys", "jssa_score",
            "jssa_topk", "jssa_topk_noalloc", "jssa_select", "jssa_indexed_attn", "jssa_decode_step",
-           "jssa_dense_decode", "jssa_gather_size", "jssa_gather_decode",
+           "jssa_dense_decode", "jssa_gather_size", "jssa_gather_decode", "jssa_calibrate_workspace_size",
+           "jssa_calibrate", "jssa_vote_select",
            "jssa_workspace_init", "jssa_read_device_status")
 
 
@@ -71,6 +72,9 @@ def load(path: str = LIB_PATH):
         "jssa_gather_size": (C.c_int, [LP, i32, i32, C.POINTER(sz)]),
         "jssa_gather_decode": (C.c_int, [LP, vp, vp, vp, vp, i32, vp, vp, i32, f32, vp, vp, vp, sz, vp, sz, vp]),
         "jssa_dense_decode": (C.c_int, [LP, vp, vp, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
+        "jssa_calibrate_workspace_size": (C.c_int, [LP, C.POINTER(sz)]),
+        "jssa_calibrate": (C.c_int, [LP, vp, vp, i64, vp, vp, vp, sz, vp]),
+        "jssa_vote_select": (C.c_int, [LP, vp, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, sz, vp]),
         "jssa_workspace_init": (C.c_int, [vp, sz, vp]),
         "jssa_read_device_status": (C.c_int, [vp, sz, C.POINTER(i32), vp]),
     }
@@ -220,6 +224,31 @@ def gather_decode(L, Q, K, V, idx, k: int, n_sel, seq_lens, window: int, sm_scal
     _check("jssa_gather_decode", load().jssa_gather_decode(C.byref(L), _c(Q), _p(K), _p(V), _c(idx), k, _c(n_sel),
                                                            _c(seq_lens), window, sm_scale, _c(O), _c(lse), _c(gbuf),
                                                            gbuf.numel(), w, n, _stream(stream)))
+
+
+def vote_select(L, Q, K, Kp, P, seq_lens, n_new: int, k: int, window: int, sm_scale: float, idx, n_sel, ws,
+                stream=None):
+    """Head-shared soft voting: one index set per sequence, written to every KV head's row."""
+    w, n = _ws(ws)
+    _check("jssa_vote_select", load().jssa_vote_select(C.byref(L), _c(Q), _p(K), _p(Kp), _c(P), _c(seq_lens), n_new,
+                                                       k, window, sm_scale, _c(idx), _c(n_sel), w, n,
+                                                       _stream(stream)))
+
+
+def alloc_calibration_workspace(L, device="cuda"):
+    """Workspace of calibrate (status word zeroed)."""
+    n = C.c_size_t(0)
+    _check("jssa_calibrate_workspace_size", load().jssa_calibrate_workspace_size(C.byref(L), C.byref(n)))
+    ws = torch.empty(n.value, dtype=torch.uint8, device=device)
+    workspace_init(ws)
+    return ws
+
+
+def calibrate(L, Qc, K, n_tokens: int, P, ws, eigvals=None, stream=None):
+    """Spectral basis from calibration queries Qc [B, Hq, n_tokens, d_k] and cache rows [0, n_tokens)."""
+    w, n = _ws(ws)
+    _check("jssa_calibrate", load().jssa_calibrate(C.byref(L), _c(Qc), _p(K), n_tokens, _c(P), _c(eigvals), w, n,
+                                                   _stream(stream)))
 
 
 def dense_decode(L, Q, K, V, seq_lens, window: int, sm_scale: float, O, lse=None, ws=None, stream=None):

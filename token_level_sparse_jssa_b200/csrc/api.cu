@@ -190,7 +190,7 @@ jssa_status run_prologue(const jssa_layout* L, const void* Q, const float* P, co
 }
 
 jssa_status run_score(const jssa_layout* L, const void* Kp, const int32_t* seq_lens, int window, float* scores,
-                      int64_t sc_ld, const Workspace& w, cudaStream_t s) {
+                      int64_t sc_ld, const Workspace& w, cudaStream_t s, bool with_hist = true) {
   ScoreArgs a{};
   a.Kp = Kp;
   memcpy(a.ps, L->kp_stride, sizeof a.ps);
@@ -198,7 +198,7 @@ jssa_status run_score(const jssa_layout* L, const void* Kp, const int32_t* seq_l
   a.qs = w.qs;
   a.scores = scores;
   a.sc_ld = sc_ld;
-  a.hist = w.hist;
+  a.hist = with_hist ? w.hist : nullptr;
   a.seq_lens = seq_lens;
   a.B = L->B;
   a.Hkv = L->Hkv;
@@ -490,6 +490,57 @@ jssa_status jssa_select(const jssa_layout* L, const void* Q, const void* K, void
   return run_select(L, Q, K, Kp, P, seq_lens, n_new, k, window, idx, n_sel, w, static_cast<cudaStream_t>(stream));
 }
 
+jssa_status jssa_vote_select(const jssa_layout* L, const void* Q, const void* K, void* Kp, const float* P,
+                             const int32_t* seq_lens, int32_t n_new, int32_t k, int32_t window, float sm_scale,
+                             int32_t* idx, int32_t* n_sel, void* workspace, size_t ws_bytes, void* stream) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  if (!Q || !K || !Kp || !P || !seq_lens || !idx || !n_sel || k < 1 || k > kMaxK || window < 0 || n_new < 0 ||
+      !(sm_scale > 0.f))
+    return JSSA_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(Kp, 16) || !aligned(P, 16) || !aligned(idx, 4) ||
+      !aligned(n_sel, 4))
+    return JSSA_ERR_INVALID_ARG;
+  Workspace w{};
+  st = get_ws(L, k, window, workspace, ws_bytes, &w);
+  if (st != JSSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n_new > kMaxPrologueRows) {
+    ProjectArgs pa = project_args(L, K, P, Kp, nullptr, seq_lens, n_new, w.status);
+    st = cu(launch_project_keys(pa, s));
+    if (st != JSSA_OK) return st;
+  }
+  st = run_prologue(L, Q, P, K, Kp, seq_lens, n_new > kMaxPrologueRows ? 0 : n_new, w, s);
+  if (st != JSSA_OK) return st;
+  st = run_score(L, Kp, seq_lens, window, w.scores, w.sc_ld, w, s, false);
+  if (st != JSSA_OK) return st;
+  VoteArgs v{};
+  v.scores = w.scores;
+  v.sc_ld = w.sc_ld;
+  v.stats = reinterpret_cast<double*>(w.qs);  // the projected queries are consumed by the scan
+  v.seq_lens = seq_lens;
+  v.B = L->B;
+  v.Hkv = L->Hkv;
+  v.T_cap = L->T_cap;
+  v.window = window;
+  v.k = k;
+  v.c = sm_scale / static_cast<float>(L->Hq / L->Hkv);
+  v.idx_shared = w.idx;
+  v.nsel_shared = w.n_sel;
+  v.idx = idx;
+  v.n_sel = n_sel;
+  v.status = w.status;
+  st = cu(launch_vote_stats(v, s));
+  if (st != JSSA_OK) return st;
+  // top-k over the B vote rows (row b of the vote layout is score row b * Hkv)
+  jssa_layout Lv = *L;
+  Lv.Hkv = 1;
+  Lv.Hq = L->Hq / L->Hkv;
+  st = run_topk(&Lv, w.scores, w.sc_ld * L->Hkv, seq_lens, k, window, w.idx, w.n_sel, w, true, s);
+  if (st != JSSA_OK) return st;
+  return cu(launch_vote_broadcast(v, s));
+}
+
 jssa_status jssa_decode_step(const jssa_layout* L, const void* Q, const void* K, const void* V, void* Kp,
                              const float* P, const int32_t* seq_lens, int32_t n_new, int32_t k, int32_t window,
                              float sm_scale, void* O, float* lse, int32_t* idx_out, int32_t* n_sel_out, void* workspace,
@@ -610,6 +661,51 @@ jssa_status jssa_dense_decode(const jssa_layout* L, const void* Q, const void* K
   if (st != JSSA_OK) return st;
   return run_attention(L, Q, K, V, nullptr, 0, nullptr, seq_lens, window, sm_scale, O, lse, w, false,
                        static_cast<cudaStream_t>(stream));
+}
+
+namespace {
+size_t calib_bytes(const jssa_layout* L) {
+  return align_up(sizeof(int)) + align_up(calib_workspace_doubles(L->Hkv, L->d_k) * sizeof(double));
+}
+}  // namespace
+
+jssa_status jssa_calibrate_workspace_size(const jssa_layout* L, size_t* bytes) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  if (!bytes) return JSSA_ERR_INVALID_ARG;
+  if (L->d_k % 64 != 0) return JSSA_ERR_UNSUPPORTED;
+  *bytes = calib_bytes(L);
+  return JSSA_OK;
+}
+
+jssa_status jssa_calibrate(const jssa_layout* L, const void* Qc, const void* K, int64_t n_tokens, float* P,
+                           double* eigvals, void* workspace, size_t ws_bytes, void* stream) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  if (L->d_k % 64 != 0) return JSSA_ERR_UNSUPPORTED;
+  if (!Qc || !K || !P || n_tokens < 1 || n_tokens > L->T_cap) return JSSA_ERR_INVALID_ARG;
+  if (!aligned(Qc, 16) || !aligned(K, 16) || !aligned(P, 4) || (eigvals && !aligned(eigvals, 8)))
+    return JSSA_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, kAlign) || ws_bytes < calib_bytes(L)) return JSSA_ERR_WORKSPACE;
+  unsigned char* base = static_cast<unsigned char*>(workspace);
+  double* scratch = reinterpret_cast<double*>(base + align_up(sizeof(int)));
+  CalibArgs a{};
+  a.Qc = Qc;
+  a.K = K;
+  memcpy(a.ks, L->k_stride, sizeof a.ks);
+  a.n_tokens = n_tokens;
+  a.B = L->B;
+  a.Hq = L->Hq;
+  a.Hkv = L->Hkv;
+  a.d = L->d_k;
+  a.r = L->r;
+  a.P = P;
+  a.eigvals = eigvals;
+  a.acc = scratch;
+  a.jac = scratch + static_cast<size_t>(L->Hkv) * 2 * L->d_k * L->d_k;
+  a.jac_off = a.jac + static_cast<size_t>(L->Hkv) * 3 * L->d_k * L->d_k;
+  a.status = reinterpret_cast<int*>(base);
+  return cu(launch_calibrate(a, static_cast<cudaStream_t>(stream)));
 }
 
 jssa_status jssa_workspace_init(void* workspace, size_t ws_bytes, void* stream) {

@@ -156,6 +156,43 @@ struct GatherArgs {
 };
 cudaError_t launch_gather_rows(const GatherArgs& a, cudaStream_t s);
 
+// Spectral calibration of the basis: second moments of the group-mean query and of the key
+// over calibration tokens, then the top-r eigenvectors of their unit-trace sum.
+struct CalibArgs {
+  const void* Qc;     // [B, Hq, n_tokens, d] bf16, contiguous
+  const void* K;      // cache rows [0, n_tokens) of every sequence
+  int64_t ks[3];
+  int64_t n_tokens;
+  int B, Hq, Hkv, d, r;
+  float* P;           // [Hkv, d, r] out
+  double* eigvals;    // nullable: [Hkv, d] out, descending
+  double* acc;        // [Hkv, 2, d, d] scratch
+  double* jac;        // [Hkv, 3, d, d] scratch
+  double* jac_off;    // [Hkv, 2, 8] scratch
+  int* status;
+};
+size_t calib_workspace_doubles(int Hkv, int d);
+cudaError_t launch_calibrate(const CalibArgs& a, cudaStream_t s);
+
+// Head-shared soft voting over the fp32 score rows of the unfused scan.
+struct VoteArgs {
+  float* scores;          // [B*Hkv, sc_ld]; row b*Hkv receives the votes of sequence b
+  int64_t sc_ld;
+  double* stats;          // [B*Hkv, 2] (max logit, sum of exponentials)
+  const int32_t* seq_lens;
+  int B, Hkv;
+  int64_t T_cap;
+  int window, k;
+  float c;                // logit scale: sm_scale / G
+  const int32_t* idx_shared;    // [B, k] the selection over the vote rows
+  const int32_t* nsel_shared;   // [B]
+  int32_t* idx;           // [B*Hkv, k] out
+  int32_t* n_sel;         // [B*Hkv] out
+  int* status;
+};
+cudaError_t launch_vote_stats(const VoteArgs& a, cudaStream_t s);      // stats, then the votes
+cudaError_t launch_vote_broadcast(const VoteArgs& a, cudaStream_t s);
+
 // Split policy shared by the workspace sizing and the launch.
 void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int num_sms, int* S, int* split_len);
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);   // GQA path
