@@ -4,8 +4,9 @@ App. C: selection at indexer layers, indices reused by the adjacent layers).
 
 The vote's error band is derived from the rigorous fp32 score bound: a score error e shifts a
 head's logit by c*e, which moves p_h(t) by at most a factor exp(+-(c e(t) + max_u c e(u)));
-the fp32 subtraction, exponential, reciprocal and product add a few units in the last place,
-and the fp32 sum over the KV heads one more per head.  Selections may differ only by swaps
+the fp32 subtraction, the exponentials (also those that merge the statistics' slices), the
+reciprocal and the product add at most ten units in the last place, and the fp32 sum over the
+KV heads one more per head.  Selections may differ only by swaps
 among tokens whose oracle vote lies within that band of the k-th vote.
 """
 import numpy as np
@@ -48,7 +49,7 @@ def _vote_band(p, b, n):
     v = ph.sum(axis=0)
     x = c * s
     eps = c * np.stack(bands) + np.abs(x) * U
-    rel = np.exp(eps + eps.max(axis=1, keepdims=True) + np.abs(x - x.max(axis=1, keepdims=True)) * U + 6 * U) - 1
+    rel = np.exp(eps + eps.max(axis=1, keepdims=True) + np.abs(x - x.max(axis=1, keepdims=True)) * U + 10 * U) - 1
     band = (ph * rel).sum(axis=0) + Hkv * U * v
     return v, band
 

@@ -517,7 +517,7 @@ jssa_status jssa_vote_select(const jssa_layout* L, const void* Q, const void* K,
   VoteArgs v{};
   v.scores = w.scores;
   v.sc_ld = w.sc_ld;
-  v.stats = reinterpret_cast<double*>(w.qs);  // the projected queries are consumed by the scan
+  v.stats = reinterpret_cast<double*>(w.hist);  // free until the vote rows' histograms are built
   v.seq_lens = seq_lens;
   v.B = L->B;
   v.Hkv = L->Hkv;

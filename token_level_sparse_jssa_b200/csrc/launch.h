@@ -178,7 +178,7 @@ cudaError_t launch_calibrate(const CalibArgs& a, cudaStream_t s);
 struct VoteArgs {
   float* scores;          // [B*Hkv, sc_ld]; row b*Hkv receives the votes of sequence b
   int64_t sc_ld;
-  double* stats;          // [B*Hkv, 2] (max logit, sum of exponentials)
+  double* stats;          // [B*Hkv, 8 slices, 2] (max logit, sum of exponentials)
   const int32_t* seq_lens;
   int B, Hkv;
   int64_t T_cap;

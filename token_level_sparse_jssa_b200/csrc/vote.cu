@@ -10,11 +10,11 @@
 // ascending) is copied to every KV head's row of the index list.
 //
 // Kernels (after the score scan has written the fp32 scores of every (b, h) row):
-//   vote_stats_kernel   — one CTA per (b, h) row: m_h (fp32 max) and Z_h (fp64 sum of the
-//                         fp32 exponentials), written over the row's projected query;
-//   vote_combine_kernel — grid (token blocks, b): v(t) for every candidate, written over
-//                         the score row of KV head 0 (the thread that reads s_0(t) writes
-//                         v(t));
+//   vote_stats_kernel   — grid (8 slices, b * Hkv + h): the slice's max logit and fp64 sum
+//                         of the fp32 exponentials relative to it;
+//   vote_combine_kernel — grid (token blocks, b): merges the slices into m_h and Z_h, then
+//                         v(t) for every candidate, written over the score row of KV head 0
+//                         (the thread that reads s_0(t) writes v(t));
 //   then the standalone top-k over the B vote rows, and
 //   vote_broadcast_kernel — the B index sets copied to all B * Hkv rows.
 #include <cfloat>
@@ -25,7 +25,9 @@
 namespace jssa {
 namespace {
 
-constexpr int kVoteThreads = 512;
+constexpr int kVoteThreads = 256;
+constexpr int kVoteSlices = 8;   // CTAs per (b, h) row of the statistics
+constexpr int kVoteMaxHkv = 64;  // KV heads merged in shared memory by the combine kernel
 constexpr int kCombineThreads = 256;
 constexpr int kCombineTok = 4;  // tokens per thread
 
@@ -41,9 +43,10 @@ __device__ __forceinline__ int64_t vote_candidates(const VoteArgs& a, int b, boo
 __global__ void __launch_bounds__(kVoteThreads) vote_stats_kernel(VoteArgs a) {
   __shared__ float smax[kVoteThreads / 32];
   __shared__ double ssum[kVoteThreads / 32];
-  const int row = blockIdx.x, b = row / a.Hkv;
-  const int64_t n = vote_candidates(a, b, threadIdx.x == 0 && row % a.Hkv == 0);
-  const float* s = a.scores + static_cast<int64_t>(row) * a.sc_ld;
+  const int row = blockIdx.y, b = row / a.Hkv;
+  const int64_t n_all = vote_candidates(a, b, threadIdx.x == 0 && blockIdx.x == 0 && row % a.Hkv == 0);
+  const int64_t lo = n_all * blockIdx.x / kVoteSlices, n = n_all * (blockIdx.x + 1) / kVoteSlices - lo;
+  const float* s = a.scores + static_cast<int64_t>(row) * a.sc_ld + lo;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float m = -FLT_MAX;
   for (int64_t t = threadIdx.x; t < n; t += kVoteThreads) m = fmaxf(m, a.c * s[t]);
@@ -60,22 +63,33 @@ __global__ void __launch_bounds__(kVoteThreads) vote_stats_kernel(VoteArgs a) {
   if (threadIdx.x == 0) {
     double t = 0.0;
     for (int w = 0; w < kVoteThreads / 32; ++w) t += ssum[w];
-    a.stats[2 * row] = static_cast<double>(m);
-    a.stats[2 * row + 1] = t;
+    a.stats[2 * (row * kVoteSlices + blockIdx.x)] = static_cast<double>(m);
+    a.stats[2 * (row * kVoteSlices + blockIdx.x) + 1] = t;
   }
 }
 
 __global__ void __launch_bounds__(kCombineThreads) vote_combine_kernel(VoteArgs a) {
+  __shared__ float mh[kVoteMaxHkv], invz[kVoteMaxHkv];
   const int b = blockIdx.y;
   const int64_t n = vote_candidates(a, b, false);
+  // merge the slices of each head: m = max m_i, Z = sum_i Z_i exp(m_i - m) (slices in order)
+  for (int h = threadIdx.x; h < a.Hkv; h += blockDim.x) {
+    const double* st = a.stats + 2 * static_cast<int64_t>(b * a.Hkv + h) * kVoteSlices;
+    float m = -FLT_MAX;
+    for (int i = 0; i < kVoteSlices; ++i) m = fmaxf(m, static_cast<float>(st[2 * i]));
+    double Z = 0.0;
+    for (int i = 0; i < kVoteSlices; ++i)
+      if (st[2 * i + 1] > 0.0) Z += st[2 * i + 1] * static_cast<double>(expf(static_cast<float>(st[2 * i]) - m));
+    mh[h] = m;
+    invz[h] = Z > 0.0 ? static_cast<float>(1.0 / Z) : 0.f;
+  }
+  __syncthreads();
   const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * kCombineThreads + threadIdx.x) * kCombineTok;
   if (t0 >= n) return;
   float v[kCombineTok] = {0.f, 0.f, 0.f, 0.f};
   float* s0 = a.scores + static_cast<int64_t>(b) * a.Hkv * a.sc_ld;
   for (int h = 0; h < a.Hkv; ++h) {
-    const float m = static_cast<float>(a.stats[2 * (b * a.Hkv + h)]);
-    const double Z = a.stats[2 * (b * a.Hkv + h) + 1];
-    const float inv = Z > 0.0 ? static_cast<float>(1.0 / Z) : 0.f;
+    const float m = mh[h], inv = invz[h];
     const float* s = s0 + static_cast<int64_t>(h) * a.sc_ld;
 #pragma unroll
     for (int j = 0; j < kCombineTok; ++j)
@@ -99,7 +113,8 @@ __global__ void vote_broadcast_kernel(VoteArgs a) {
 }  // namespace
 
 cudaError_t launch_vote_stats(const VoteArgs& a, cudaStream_t s) {
-  vote_stats_kernel<<<a.B * a.Hkv, kVoteThreads, 0, s>>>(a);
+  if (a.Hkv > kVoteMaxHkv) return cudaErrorInvalidValue;
+  vote_stats_kernel<<<dim3(kVoteSlices, a.B * a.Hkv), kVoteThreads, 0, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t per_cta = static_cast<int64_t>(kCombineThreads) * kCombineTok;
