@@ -167,3 +167,33 @@ def test_package_import_does_not_load_the_library_and_fails_loudly_when_missing(
             "try:\n    b.load(r'%s')\nexcept RuntimeError as e:\n    print('LOUD', e)\n" % (tmp_path / "missing.so"))
     out = subprocess.run(["python", "-c", code], capture_output=True, text=True, cwd=ROOT, check=True).stdout
     assert "LOUD" in out and "no fallback" in out
+
+
+def test_calibration_entry_points_validate_on_the_host(lib):
+    L = _layout(B=2, Hq=8, Hkv=2, d=128, r=32, T=1024)
+    n = C.c_size_t(0)
+    assert lib.jssa_calibrate_workspace_size(C.byref(L), C.byref(n)) == 0
+    # status word (256 B) + [Hkv][2 moments + 3 Jacobi matrices][d][d] doubles + [Hkv][2][8] doubles
+    assert n.value == 256 + ((2 * 5 * 128 * 128 + 2 * 2 * 8) * 8 + 255) // 256 * 256
+    assert lib.jssa_calibrate_workspace_size(C.byref(L), None) == 1
+    ws = C.c_void_p(FAKE)
+    big = n.value
+    assert lib.jssa_calibrate(C.byref(L), None, FAKE, 100, FAKE, None, ws, big, None) == 1       # no queries
+    assert lib.jssa_calibrate(C.byref(L), FAKE, FAKE, 0, FAKE, None, ws, big, None) == 1         # no tokens
+    assert lib.jssa_calibrate(C.byref(L), FAKE, FAKE, 1025, FAKE, None, ws, big, None) == 1      # beyond T_cap
+    assert lib.jssa_calibrate(C.byref(L), FAKE + 8, FAKE, 100, FAKE, None, ws, big, None) == 1   # misaligned
+    assert lib.jssa_calibrate(C.byref(L), FAKE, FAKE, 100, FAKE, None, ws, big - 256, None) == 3  # small workspace
+    assert lib.jssa_calibrate(C.byref(L), FAKE, FAKE, 100, FAKE, None, C.c_void_p(FAKE + 64), big, None) == 3
+
+
+def test_voting_and_gather_entry_points_validate_on_the_host(lib):
+    L = _layout()
+    ws = C.c_void_p(FAKE)
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, 0, 16, 0]
+    assert lib.jssa_vote_select(C.byref(L), *args, C.c_float(0.0), FAKE, FAKE, ws, 1 << 30, None) == 1   # sm_scale
+    assert lib.jssa_vote_select(C.byref(L), *args, C.c_float(-1.0), FAKE, FAKE, ws, 1 << 30, None) == 1
+    bad_k = [FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, 0]
+    assert lib.jssa_vote_select(C.byref(L), *bad_k, C.c_float(0.1), FAKE, FAKE, ws, 1 << 30, None) == 1   # k = 0
+    assert lib.jssa_vote_select(C.byref(L), None, *args[1:], C.c_float(0.1), FAKE, FAKE, ws, 1 << 30, None) == 1
+    n = C.c_size_t(0)
+    assert lib.jssa_gather_size(C.byref(L), 0, 0, C.byref(n)) == 1

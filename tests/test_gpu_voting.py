@@ -42,8 +42,14 @@ def _vote_band(p, b, n):
         hst = p.host(b, h)
         Kp_or = p.project(hst["K"][:n], hst["P"])
         np.testing.assert_array_equal(hst["Kp"][:n], Kp_or)       # the GPU cache is the oracle's
-        s.append(oracle.scores(oracle.query_proj(hst["Q"], hst["P"]), Kp_or))
-        bands.append(score_error_bound(hst["Q"], hst["P"], Kp_or))
+        qs = oracle.query_proj(hst["Q"], hst["P"])
+        if p.kp_fp8:
+            vals = np.vectorize(oracle.e4m3_to_double, otypes=[np.float64])(Kp_or)
+            s.append(oracle.scores_e4m3(qs, Kp_or))
+            bands.append(score_error_bound(hst["Q"], hst["P"], vals))
+        else:
+            s.append(oracle.scores(qs, Kp_or))
+            bands.append(score_error_bound(hst["Q"], hst["P"], Kp_or))
     s = np.stack(s)
     ph = voting.head_distributions(s, c)
     v = ph.sum(axis=0)
@@ -68,16 +74,19 @@ def _check_vote_selection(g_idx, g_n, v, band, k):
     return False
 
 
-@pytest.mark.parametrize("name,kw,seq,window", [
-    ("tiny", {}, None, 0),
-    ("h128k", dict(B=2, T=5000, k=256), [5000, 3001], 0),
-    ("hybrid", dict(B=2, T=4000, k=300), [4000, 1200], 1024),
-    ("h128k", dict(B=1, Hq=32, Hkv=2, T=3000, k=100), [3000], 0),     # G = 16
-    ("h128k", dict(B=2, T=600, k=1024), [600, 2000], 0),             # k above the candidates in one row
+@pytest.mark.parametrize("name,kw,seq,window,fp8", [
+    ("tiny", {}, None, 0, False),
+    ("h128k", dict(B=2, T=5000, k=256), [5000, 3001], 0, False),
+    ("hybrid", dict(B=2, T=4000, k=300), [4000, 1200], 1024, False),
+    ("h128k", dict(B=1, Hq=32, Hkv=2, T=3000, k=100), [3000], 0, False),     # G = 16
+    ("h128k", dict(B=2, T=600, k=1024), [600, 2000], 0, False),             # k above the candidates in one row
+    ("mla", dict(B=2, T=3000, k=300), [3000, 2222], 0, False),              # one latent head: the score ranking
+    ("h128k", dict(B=2, T=5000, k=256), [5000, 4000], 0, True),             # E4M3 scoring cache
+    ("h128k", dict(B=1, Hq=8, Hkv=2, T=140000, k=1024), [140000], 0, False),  # longer than one cluster's slices
 ])
-def test_vote_select_matches_the_oracle(name, kw, seq, window):
+def test_vote_select_matches_the_oracle(name, kw, seq, window, fp8):
     w = W[name].with_(**kw)
-    p = Problem(w, T_cap=max(seq) if seq else None, seq_lens=seq)
+    p = Problem(w, T_cap=max(seq) if seq else None, seq_lens=seq, kp_fp8=fp8)
     p.fill_kp()
     ws = p.workspace(w.k, window)
     idx = torch.full((w.B, w.Hkv, w.k), -7, dtype=torch.int32, device="cuda")

@@ -40,7 +40,8 @@ constexpr int kSelConsumers = 256;                 // 8 consumer warps
 constexpr int kSelThreads = kSelConsumers + 32;    // + 1 producer warp
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelStage = 16384;                   // bytes per ring stage
-constexpr int kSelMaxCluster = 16;                 // 8 (portable) or 16 CTAs per row
+constexpr int kSelMaxCluster = 16;                 // up to 8 (portable) or 16 CTAs per row
+constexpr int kSelMinCluster = 2;                  // fewer than 8 only to keep every row in one wave
 constexpr int kSelBins1 = 4096;                    // digit 1: key bits [31:20]
 constexpr int kSelBins2 = 1024;                    // digits 2 and 3: bits [19:10] and [9:0]
 constexpr int kSelCapW = 64;                       // per-warp capacity of the definite / candidate lists
@@ -51,6 +52,14 @@ constexpr int kSelMaxNew = 16;                     // newest rows projected insi
 constexpr int kSelMaxR = 64;
 constexpr int kSelKeysMin = 16384;                 // the keys area also holds the projection scratch
 constexpr int kSelMaxDn = 72;                      // dims per CTA of the split projections (576 / 8)
+
+// Words of the owned-bins area: the CTA's share of the row's first-digit histogram (an even
+// number of bins), later its share of the attended token list; at least 512 words, so that
+// clusters of 8 or more CTAs share one layout.
+__host__ __device__ constexpr int sel_own_bins(int C) { return (((kSelBins1 + C - 1) / C) + 1) & ~1; }
+__host__ __device__ constexpr int sel_own_words(int C) {
+  return sel_own_bins(C) > kSelBins1 / 8 ? sel_own_bins(C) : kSelBins1 / 8;
+}
 
 __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kSelConsumers) : "memory"); }
 
@@ -139,7 +148,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
   const int C = static_cast<int>(cluster.num_blocks());  // 8 or 16
-  const int own_bins = (((kSelBins1 + C - 1) / C) + 1) & ~1;  // even: a packed bin pair has one owner
+  const int own_bins = sel_own_bins(C);  // even: a packed bin pair has one owner
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const int S = a.stages;
   const int keys_words = a.keys_words;
@@ -147,7 +156,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
   uint32_t* keys = reinterpret_cast<uint32_t*>(ring + S * kSelStage);                   // [keys_words]
   uint32_t* histp = keys + keys_words;                                                   // [2048] packed 16-bit bins
   uint32_t* own = histp + kSelBins1 / 2;                                                 // [4096 / C] owned row bins
-  float* qpart = reinterpret_cast<float*>(own + kSelBins1 / 8);                         // [R] this CTA's share of qs
+  float* qpart = reinterpret_cast<float*>(own + sel_own_words(C));                     // [R] this CTA's share of qs
   double* npart = reinterpret_cast<double*>(qpart + kSelMaxR);                          // [n_new][R] newest-row shares
   unsigned char* kpn = reinterpret_cast<unsigned char*>(npart + a.n_new * R);           // [n_new][R] newest Kp rows
   // after the scan the ring holds the row histogram copy and the selection scratch
@@ -790,20 +799,26 @@ cudaError_t launch_select_r(SelectArgs a, int num_sms, cudaStream_t s) {
       np_done[dev] = -1, (void)cudaGetLastError();
   }
   const int rows = a.B * a.Hkv;
-  // Cluster size and ring depth: the largest cluster (8..16 CTAs per row) whose clusters are
-  // all resident at once when 8 CTAs per row would leave SMs idle, 8 otherwise; then the
-  // deepest ring that keeps every row's cluster resident (a second wave of clusters would
-  // double the scan time).  With the attention inside, the ring and keys areas also hold the
-  // attention's buffers, and each CTA's share of the attended list must fit its token list.
-  int C = 8, stages = 2;
+  // Cluster size and ring depth.  Sizes are tried from the largest down: 9..16 CTAs per row
+  // only when 8 per row would leave SMs idle, fewer than 8 (down to 2) only when 8 per row
+  // cannot all be resident at once.  The first size whose clusters are all resident wins, with
+  // the deepest ring that keeps them so: a second wave of clusters would pay the scan and the
+  // selection's serial tail twice.  If no size fits in one wave, 8 CTAs per row run in two.
+  // With the attention inside, the ring and keys areas also hold the attention's buffers, and
+  // each CTA's share of the attended list must fit its token list.
+  int C = 0, stages = 2, per_c = 0, kw_c = 0;
   size_t fixed = 0;
+  int fb_per = 0, fb_kw = 0;  // the two-wave fallback at 8 CTAs per row
+  size_t fb_fixed = 0;
   const int64_t list_max = a.k + min64(max64(a.window, 0), a.T_cap);
   const int c_max = (np_done[dev] > 0 && static_cast<int64_t>(rows) * 8 < num_sms) ? kSelMaxCluster : 8;
-  for (int c_try = c_max; c_try >= 8; --c_try) {
+  for (int c_try = c_max; c_try >= kSelMinCluster; --c_try) {
     const int per = static_cast<int>(ceil_div(ceil_div(a.T_cap, c_try), 32) * 32);
     if (per > kSelMaxSlice) continue;
-    if (D > 0 && ceil_div(list_max, c_try) > kSelBins1 / 8) continue;  // token list lives in own[]
-    const size_t tail = (kSelBins1 / 2) * 4 + (kSelBins1 / 8) * 4 + kSelMaxR * 4 +
+    if (ceil_div(a.d / 8, c_try) * 8 > kSelMaxDn) continue;                    // share of the projections
+    const int own_words = sel_own_words(c_try);
+    if (D > 0 && ceil_div(list_max, c_try) > own_words) continue;             // token list lives in own[]
+    const size_t tail = (kSelBins1 / 2) * 4 + static_cast<size_t>(own_words) * 4 + kSelMaxR * 4 +
                         static_cast<size_t>(a.n_new) * R * 8 + static_cast<size_t>((a.n_new * R + 7) & ~7) * 2;
     int st_ok = 0, kw_ok = 0;
     for (int st = 8; st >= 2; --st) {
@@ -816,19 +831,32 @@ cudaError_t launch_select_r(SelectArgs a, int num_sms, cudaStream_t s) {
       if (smem + kSelStaticBytes > 227u * 1024u) continue;
       if (active_clusters(kernel, c_try, smem, rows) >= rows) { st_ok = st; kw_ok = kw; break; }
     }
-    if (st_ok == 0 && c_try > 8) continue;  // these clusters would need a second wave
-    if (st_ok == 0) {
-      kw_ok = max(per, kSelKeysMin / 4);
-      if (D > 0) kw_ok = max(kw_ok, (attn_main_bytes<D>() - 2 * kSelStage + 3) / 4);
+    if (st_ok == 0) {  // these clusters would need a second wave
+      if (c_try == 8) {
+        fb_kw = max(per, kSelKeysMin / 4);
+        if (D > 0) fb_kw = max(fb_kw, (attn_main_bytes<D>() - 2 * kSelStage + 3) / 4);
+        fb_per = per;
+        fb_fixed = static_cast<size_t>(fb_kw) * 4 + tail;
+      }
+      continue;
     }
     C = c_try;
-    stages = st_ok > 0 ? st_ok : 2;
+    stages = st_ok;
     fixed = static_cast<size_t>(kw_ok) * 4 + tail;
-    a.per = per;
-    a.keys_words = kw_ok;
+    per_c = per;
+    kw_c = kw_ok;
     break;
   }
+  if (C == 0 && fb_fixed > 0) {
+    C = 8;
+    stages = 2;
+    fixed = fb_fixed;
+    per_c = fb_per;
+    kw_c = fb_kw;
+  }
   if (fixed == 0) return D > 0 ? cudaErrorNotSupported : cudaErrorInvalidValue;
+  a.per = per_c;
+  a.keys_words = kw_c;
   a.stages = stages;
   const size_t smem = static_cast<size_t>(stages) * kSelStage + fixed;
   if (smem + kSelStaticBytes > 227u * 1024u) return D > 0 ? cudaErrorNotSupported : cudaErrorInvalidValue;
