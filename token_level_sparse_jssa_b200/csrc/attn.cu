@@ -32,9 +32,10 @@ static size_t attn_smem_bytes() {
 }
 
 template <int D, int NTILE, bool DENSE>
-__global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(AttnCfg<D>::THREADS) attn_kernel(AttnArgs a) {
   using Cfg = AttnCfg<D>;
-  constexpr int KSTEPS = D / 16;
+  constexpr int KSTEPS = Cfg::DW / 16;  // Q fragments of this warp's head dims
+  constexpr int NT = Cfg::THREADS;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   int32_t* tok_s = reinterpret_cast<int32_t*>(smem_raw + Cfg::MAIN_BYTES);
 
@@ -48,18 +49,18 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
   // below) and the query fragments.
   int64_t T = a.seq_lens[b];
   int64_t nsel = DENSE ? 0 : a.n_sel[row];
-  constexpr int kPre = 4;  // index entries per thread loaded up front (splits up to 512 tokens)
+  constexpr int kPre = 4;  // index entries per thread loaded up front (4 x block size tokens)
   int32_t pre[kPre];
   if (!DENSE) {
     const int32_t* irow = a.idx + static_cast<int64_t>(row) * a.idx_ld;
 #pragma unroll
     for (int u = 0; u < kPre; ++u) {
-      const int64_t pos = my_lo + threadIdx.x + u * kAttnThreads;
-      pre[u] = (threadIdx.x + u * kAttnThreads < a.split_len && pos < a.idx_ld) ? __ldg(irow + pos) : -1;
+      const int64_t pos = my_lo + threadIdx.x + u * NT;
+      pre[u] = (threadIdx.x + u * NT < a.split_len && pos < a.idx_ld) ? __ldg(irow + pos) : -1;
     }
   }
   uint32_t qf[NTILE][KSTEPS][2];
-  load_q_frags<D, NTILE>(a.Q, hq0, G, qf);
+  load_q_frags<D, NTILE, KSTEPS>(a.Q, hq0, G, qf, ((threadIdx.x >> 5) / kAttnWarps % Cfg::HALVES) * Cfg::DW);
   if (T < 0 || T > a.T_cap) {
     if (split == 0 && threadIdx.x == 0) flag_error(a.status, DEVFLAG_BAD_SEQ_LEN);
     T = T < 0 ? 0 : a.T_cap;
@@ -84,11 +85,11 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
   float* plse = pbuf + 16 * D;                                              // [16]
   if (my_len == 0) {  // empty split: weight zero in the merge
     if constexpr (!DENSE) {
-      for (int i = threadIdx.x; i < G * D; i += kAttnThreads) pbuf[i] = 0.f;
+      for (int i = threadIdx.x; i < G * D; i += NT) pbuf[i] = 0.f;
       if (threadIdx.x < G) plse[threadIdx.x] = -INFINITY;
       cluster_merge<D>(a, hq0, G, pbuf, plse);
     } else {
-      for (int i = threadIdx.x; i < G * D; i += kAttnThreads) {
+      for (int i = threadIdx.x; i < G * D; i += NT) {
         const int head = i / D, dim = i % D;
         a.part_o[((hq0 + head) * a.S + split) * D + dim] = 0.f;
         if (dim == 0) a.part_lse[(hq0 + head) * a.S + split] = -INFINITY;
@@ -113,10 +114,10 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(AttnArgs a) {
     };
 #pragma unroll
     for (int u = 0; u < kPre; ++u) {
-      const int j = threadIdx.x + u * kAttnThreads;
+      const int j = threadIdx.x + u * NT;
       if (j < my_len) resolve(j, pre[u]);
     }
-    for (int j = threadIdx.x + kPre * kAttnThreads; j < my_len; j += kAttnThreads)
+    for (int j = threadIdx.x + kPre * NT; j < my_len; j += NT)
       resolve(j, (my_lo + j < nsel) ? irow[my_lo + j] : 0);
     __syncthreads();
   }
@@ -243,7 +244,7 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
   cudaError_t e = set_smem_limit_once(attn_kernel<D, NTILE, DENSE>, smem, done);
   if (e != cudaSuccess) return e;
   // indexed: the S (<= 8) splits of a row form one cluster and merge through shared memory
-  return launch_ex(attn_kernel<D, NTILE, DENSE>, dim3(a.S, a.B * a.Hkv), dim3(kAttnThreads), smem, s,
+  return launch_ex(attn_kernel<D, NTILE, DENSE>, dim3(a.S, a.B * a.Hkv), dim3(AttnCfg<D>::THREADS), smem, s,
                    DENSE ? 0 : a.S, a);
 }
 

@@ -20,23 +20,32 @@ namespace cg = cooperative_groups;
 namespace jssa {
 
 constexpr int kAttnWarps = 4;
-constexpr int kAttnThreads = kAttnWarps * 32;
 constexpr int kSub = 16;                 // tokens per warp subtile
 constexpr int kMaxTokList = 4096;        // indexed mode: split length bound (token list in smem)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+// Per head dimension D: kAttnWarps warp groups stream the subtiles; a group is one warp, or,
+// for D = 256, a pair of warps that each take half of the head dims (the score partials of
+// the two halves are added through shared memory, then both warps run the same softmax and
+// each accumulates its half of the output), which halves the dependency chain of a warp and
+// doubles the warps that hide each other's latency.
 template <int D>
 struct AttnCfg {
-  static constexpr int STAGES = (D <= 64) ? 4 : (D <= 128 ? 3 : 2);
-  static constexpr int CPR = D / 8;                    // 16-byte chunks per row
-  static constexpr int SUB_BYTES = kSub * D * 2;       // one K or V subtile
+  static constexpr int HALVES = (D >= 256) ? 2 : 1;    // warps per group
+  static constexpr int DW = D / HALVES;                // head dims per warp
+  static constexpr int WARPS = kAttnWarps * HALVES;
+  static constexpr int THREADS = WARPS * 32;
+  static constexpr int STAGES = (DW <= 64) ? 4 : 3;
+  static constexpr int CPR = DW / 8;                   // 16-byte chunks per row and warp
+  static constexpr int SUB_BYTES = kSub * DW * 2;      // one K or V subtile (this warp's dims)
   static constexpr int STAGE_BYTES = 2 * SUB_BYTES;
-  static constexpr int RING_BYTES = kAttnWarps * STAGES * STAGE_BYTES;
+  static constexpr int RING_BYTES = WARPS * STAGES * STAGE_BYTES;
+  static constexpr int XCH_BYTES = (HALVES > 1) ? WARPS * 2 * 32 * 8 * 4 : 0;  // [warp][parity][lane][<= 8]
   static constexpr int COMBINE_BYTES = kAttnWarps * 16 * D * 4 + 2 * kAttnWarps * 16 * 4;
   static constexpr int PART_BYTES = 16 * D * 4 + 16 * 4;   // this CTA's partial (o, lse) for the cluster merge
-  static constexpr int MAIN_BYTES =
-      RING_BYTES > COMBINE_BYTES + PART_BYTES ? RING_BYTES : COMBINE_BYTES + PART_BYTES;
+  static constexpr int MAIN_BYTES = RING_BYTES + XCH_BYTES > COMBINE_BYTES + PART_BYTES ? RING_BYTES + XCH_BYTES
+                                                                                        : COMBINE_BYTES + PART_BYTES;
 };
 
 template <int D>
@@ -163,9 +172,11 @@ __device__ __forceinline__ void cluster_merge(const AttnArgs& a, int64_t hq0, in
   cl.sync();
 }
 
-// Q^T as MMA B fragments: head nt*8 + g, dims kk*16 + 2c (+8) (g = lane / 4, c = lane % 4).
-template <int D, int NTILE>
-__device__ __forceinline__ void load_q_frags(const void* Q, int64_t hq0, int G, uint32_t (&qf)[NTILE][D / 16][2]) {
+// Q^T as MMA B fragments: head nt*8 + g, dims dim0 + kk*16 + 2c (+8) (g = lane / 4, c = lane % 4),
+// for the KS K-steps of 16 dims from dim0.
+template <int D, int NTILE, int KS = D / 16>
+__device__ __forceinline__ void load_q_frags(const void* Q, int64_t hq0, int G, uint32_t (&qf)[NTILE][KS][2],
+                                             int dim0 = 0) {
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const __nv_bfloat16* Qg = static_cast<const __nv_bfloat16*>(Q) + hq0 * D;
@@ -173,9 +184,10 @@ __device__ __forceinline__ void load_q_frags(const void* Q, int64_t hq0, int G, 
   for (int nt = 0; nt < NTILE; ++nt) {
     const int head = nt * 8 + g;
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
+    for (int kk = 0; kk < KS; ++kk) {
       if (head < G) {
-        const uint32_t* qp = reinterpret_cast<const uint32_t*>(Qg + static_cast<int64_t>(head) * D + kk * 16 + 2 * c);
+        const uint32_t* qp =
+            reinterpret_cast<const uint32_t*>(Qg + static_cast<int64_t>(head) * D + dim0 + kk * 16 + 2 * c);
         qf[nt][kk][0] = __ldg(qp);
         qf[nt][kk][1] = __ldg(qp + 4);
       } else {
@@ -187,20 +199,23 @@ __device__ __forceinline__ void load_q_frags(const void* Q, int64_t hq0, int G, 
 }
 
 // One split of a row: the attended tokens are tok_s[0, my_len) (indexed) or the contiguous
-// range win_start + my_lo + [0, my_len) (dense).  The first kAttnWarps warps stream and
-// multiply; every thread of the block must call this (it holds block and cluster barriers).
+// range win_start + my_lo + [0, my_len) (dense).  The first AttnCfg<D>::WARPS warps stream and
+// multiply (qf holds the Q fragments of the warp's dims); every thread of the block must call
+// this (it holds block and cluster barriers).
 // Writes the split's partial through the cluster merge (indexed) or the workspace and the
 // row's last CTA (dense).  smem_raw: AttnCfg<D>::MAIN_BYTES of shared memory.
 template <int D, int NTILE, bool DENSE>
 __device__ __forceinline__ void attn_core(const AttnArgs& a, int row, int split, int b, int h, int G, int64_t hq0,
-                                          const uint32_t (&qf)[NTILE][D / 16][2], const int32_t* tok_s,
+                                          const uint32_t (&qf)[NTILE][AttnCfg<D>::DW / 16][2], const int32_t* tok_s,
                                           int64_t win_start, int64_t my_lo, int my_len, unsigned char* smem_raw) {
   using Cfg = AttnCfg<D>;
-  constexpr int STAGES = Cfg::STAGES, CPR = Cfg::CPR;
-  constexpr int KSTEPS = D / 16;
+  constexpr int STAGES = Cfg::STAGES, CPR = Cfg::CPR, HALVES = Cfg::HALVES, DW = Cfg::DW;
+  constexpr int KSTEPS = DW / 16;  // K-steps of the score MMA and M-tiles of the output, this warp's dims
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
-  unsigned char* ring = smem_raw + (warp < kAttnWarps ? warp : 0) * STAGES * Cfg::STAGE_BYTES;
+  const bool streams = warp < Cfg::WARPS;
+  const int grp = warp % kAttnWarps, hf = (warp / kAttnWarps) % HALVES;  // warp group, half of the dims
+  unsigned char* ring = smem_raw + (streams ? warp : 0) * STAGES * Cfg::STAGE_BYTES;
   float* pbuf = reinterpret_cast<float*>(smem_raw + Cfg::COMBINE_BYTES);   // [16][D] (cluster merge)
   float* plse = pbuf + 16 * D;                                              // [16]
   const float scale_log2 = a.sm_scale * kLog2e;
@@ -216,18 +231,18 @@ __device__ __forceinline__ void attn_core(const AttnArgs& a, int row, int split,
       for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
   }
 
-  const __nv_bfloat16* Kb = static_cast<const __nv_bfloat16*>(a.K) + b * a.ks[0] + h * a.ks[1];
-  const __nv_bfloat16* Vb = static_cast<const __nv_bfloat16*>(a.V) + b * a.vs[0] + h * a.vs[1];
+  const __nv_bfloat16* Kb = static_cast<const __nv_bfloat16*>(a.K) + b * a.ks[0] + h * a.ks[1] + hf * DW;
+  const __nv_bfloat16* Vb = static_cast<const __nv_bfloat16*>(a.V) + b * a.vs[0] + h * a.vs[1] + hf * DW;
   const int nsub = (my_len + kSub - 1) / kSub;
-  // warps beyond the first kAttnWarps (a larger block) only join the barriers
-  const int my_count = (warp < kAttnWarps && nsub > warp) ? (nsub - warp + kAttnWarps - 1) / kAttnWarps : 0;
+  // warps beyond the streaming ones (a larger block) only join the barriers
+  const int my_count = (streams && nsub > grp) ? (nsub - grp + kAttnWarps - 1) / kAttnWarps : 0;
 
   auto token_at = [&](int j) -> int64_t {
     if (j >= my_len) return -1;
     return DENSE ? (win_start + my_lo + j) : static_cast<int64_t>(tok_s[j]);
   };
-  auto issue = [&](int i) {  // i-th subtile of this warp into stage i % STAGES
-    const int sub = warp + i * kAttnWarps;
+  auto issue = [&](int i) {  // i-th subtile of this warp's group into stage i % STAGES
+    const int sub = grp + i * kAttnWarps;
     unsigned char* kbuf = ring + (i % STAGES) * Cfg::STAGE_BYTES;
     unsigned char* vbuf = kbuf + Cfg::SUB_BYTES;
 #pragma unroll
@@ -253,16 +268,17 @@ __device__ __forceinline__ void attn_core(const AttnArgs& a, int row, int split,
     cp_async_commit();
     cp_async_wait<STAGES - 1>();
     __syncwarp();
-    const int sub = warp + i * kAttnWarps;
+    const int sub = grp + i * kAttnWarps;
     const unsigned char* kbuf = ring + (i % STAGES) * Cfg::STAGE_BYTES;
     const unsigned char* vbuf = kbuf + Cfg::SUB_BYTES;
 
     // ---- S^T = K_sub . Q^T
-    float sacc[NTILE][4];
+    // (even and odd K-steps accumulate separately: two dependency chains of D/32 MMAs)
+    float sacc[NTILE][4], sacc_odd[NTILE][4];
 #pragma unroll
     for (int nt = 0; nt < NTILE; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+      for (int e = 0; e < 4; ++e) sacc[nt][e] = sacc_odd[nt][e] = 0.f;
     {
       const int tin = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
@@ -271,8 +287,32 @@ __device__ __forceinline__ void attn_core(const AttnArgs& a, int row, int split,
         uint32_t af[4];
         ldmatrix_x4(af, kbuf + (tin * CPR + (ch ^ (tin & 7))) * 16);
 #pragma unroll
-        for (int nt = 0; nt < NTILE; ++nt) mma_bf16_16816(sacc[nt], af, qf[nt][kk][0], qf[nt][kk][1]);
+        for (int nt = 0; nt < NTILE; ++nt)
+          mma_bf16_16816((kk & 1) ? sacc_odd[nt] : sacc[nt], af, qf[nt][kk][0], qf[nt][kk][1]);
       }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] += sacc_odd[nt][e];
+    if constexpr (HALVES > 1) {
+      // add the other half's score partial (double-buffered by subtile parity; the pair's
+      // barrier orders every write before the partner's read, and a buffer is written again
+      // only after the partner has passed the next barrier, i.e. finished reading it)
+      static_assert(NTILE * 4 <= 8, "exchange slot of 8 floats per lane");
+      float* xch = reinterpret_cast<float*>(smem_raw + Cfg::RING_BYTES);
+      const int partner = grp + (1 - hf) * kAttnWarps;
+      float* mine = xch + ((warp * 2 + (i & 1)) * 32 + lane) * 8;
+      const float* theirs = xch + ((partner * 2 + (i & 1)) * 32 + lane) * 8;
+#pragma unroll
+      for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mine[nt * 4 + e] = sacc[nt][e];
+      asm volatile("bar.sync %0, 64;" ::"r"(8 + grp) : "memory");
+#pragma unroll
+      for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[nt][e] += theirs[nt * 4 + e];
     }
     // ---- online softmax over the 16 tokens of this subtile
     const bool v0 = token_at(sub * kSub + g) >= 0;
@@ -347,21 +387,21 @@ __device__ __forceinline__ void attn_core(const AttnArgs& a, int row, int split,
     }
   __syncthreads();  // ring no longer needed
   float* o_w = reinterpret_cast<float*>(smem_raw);           // [warps][16 heads][D]
-  float* m_w = o_w + kAttnWarps * 16 * D;                     // [warps][16]
-  float* l_w = m_w + kAttnWarps * 16;                         // [warps][16]
+  float* m_w = o_w + kAttnWarps * 16 * D;                     // [groups][16]
+  float* l_w = m_w + kAttnWarps * 16;                         // [groups][16]
 #pragma unroll
-  for (int nt = 0; nt < NTILE && warp < kAttnWarps; ++nt) {
+  for (int nt = 0; nt < NTILE && streams; ++nt) {
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int head = nt * 8 + 2 * c + e;
-      if (g == 0) {
-        m_w[warp * 16 + head] = m_run[nt][e];
-        l_w[warp * 16 + head] = l_run[nt][e];
+      if (g == 0 && hf == 0) {  // both halves hold the same softmax state
+        m_w[grp * 16 + head] = m_run[nt][e];
+        l_w[grp * 16 + head] = l_run[nt][e];
       }
 #pragma unroll
       for (int mt = 0; mt < KSTEPS; ++mt) {
-        o_w[(warp * 16 + head) * D + mt * 16 + g] = acc[mt][nt][e];
-        o_w[(warp * 16 + head) * D + mt * 16 + g + 8] = acc[mt][nt][2 + e];
+        o_w[(grp * 16 + head) * D + hf * DW + mt * 16 + g] = acc[mt][nt][e];
+        o_w[(grp * 16 + head) * D + hf * DW + mt * 16 + g + 8] = acc[mt][nt][2 + e];
       }
     }
   }
