@@ -206,8 +206,9 @@ JSSA_API jssa_status jssa_indexed_attn(const jssa_layout* L, const void* Q, cons
  * projected group query, score every candidate [0, T_b - W) and select the top-k per
  * (sequence, KV head), with the ties, ordering and padding rules of jssa_topk.
  *   idx    device int32 [B, Hkv, k]      n_sel  device int32 [B, Hkv]
- * When T_cap <= 131072 all of this runs in one kernel with one 8-CTA cluster per
- * (sequence, KV head), the scores never leaving shared memory; longer caches take the
+ * When T_cap <= 131072 all of this runs in one kernel with one thread-block cluster per
+ * (sequence, KV head) of 2 to 16 CTAs (the largest size that keeps every row's cluster
+ * resident at once), the scores never leaving shared memory; longer caches take the
  * jssa_score + jssa_topk kernels.  Up to 16 appended rows are projected inside the
  * selection; more are projected by the bulk projection kernel first.
  */

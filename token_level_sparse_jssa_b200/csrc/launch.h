@@ -104,7 +104,7 @@ struct AttnArgs {
   int* status;
 };
 // Fused selection (query projection, newest-key projection, score scan, top-k) with one
-// 8-CTA cluster per (sequence, KV head); rows of up to select_max_candidates() tokens.
+// 2-16 CTA cluster per (sequence, KV head); rows of up to select_max_candidates() tokens.
 struct SelectArgs {
   const void* Q;     // [B, Hq, d]
   const float* P;    // [Hkv, d, r]

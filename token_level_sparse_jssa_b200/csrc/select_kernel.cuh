@@ -12,15 +12,15 @@
 // the lower index, output ascending; §3.2 (keys projected on write): the newest key rows
 // are projected into the scoring cache inside the same step.
 //
-// The cluster's C = 8 CTAs split the row's candidates into contiguous slices of at most
-// `per` tokens.  Each CTA streams its slice of Kp through a ring of 16 KB stages (one
-// producer warp, 1-D bulk copies, full/empty mbarriers; eight consumer warps), keeps the
-// order-preserving score keys of its slice in shared memory and counts the top 12 key
-// bits in a packed 16-bit histogram.  The row's histogram is then assembled in distributed
-// shared memory (CTA c owns bins [512c, 512c + 512)); each CTA finds the first radix digit,
-// lists its keys above and inside that bin, gathers the row's in-bin keys into rank 0,
-// resolves digits 2 and 3 locally and writes its selected positions in order.  Neither the
-// scores nor the histogram leave the chip.
+// The cluster's C CTAs (2 to 16, chosen at launch) split the row's candidates into
+// contiguous slices of at most `per` tokens.  Each CTA streams its slice of Kp through a
+// ring of 16 KB stages (one producer warp, 1-D bulk copies, full/empty mbarriers; eight
+// consumer warps), keeps the order-preserving score keys of its slice in shared memory and
+// counts the top 12 key bits in a packed 16-bit histogram.  The row's histogram is then
+// assembled in distributed shared memory (each CTA owns an even-sized share of the 4096
+// bins); each CTA finds the first radix digit, lists its keys above and inside that bin,
+// gathers the row's in-bin keys into rank 0, resolves digits 2 and 3 locally and writes its
+// selected positions in order.  Neither the scores nor the histogram leave the chip.
 #pragma once
 
 #include <cooperative_groups.h>
