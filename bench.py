@@ -52,7 +52,7 @@ def step_kernels(w) -> tuple[int, bool]:
     if w.mode == "mla":
         return 3, False                                  # selection, tensor-core attention, merge
     fused = w.dk <= 128 and w.G <= 16
-    return (1 if fused else 2), fused
+    return (1 if fused else 2) + (w.layers - 1), fused   # + one dense kernel per local layer
 
 
 def parse():
@@ -65,13 +65,15 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--kp", default="bf16", choices=["bf16", "e4m3"], help="projected scoring cache type")
+    ap.add_argument("--k", type=int, default=0, help="token budget (default: the workload's)")
     return ap.parse_args()
 
 
 # --------------------------------------------------------------------------- helpers
 def byte_model(w, T, k, window, out_bytes=2, kp_bytes=2):
     """Algorithmic bytes of one step and of the dense step (HBM roofline numerator);
-    kp_bytes = bytes per projected-cache element (2 bf16, 1 E4M3)."""
+    kp_bytes = bytes per projected-cache element (2 bf16, 1 E4M3).  A hybrid model's step also
+    runs w.layers - 1 local layers: dense attention over their window-sized caches."""
     n = T - min(window, T)
     keff = min(k, n)
     rows = w.B * w.Hkv
@@ -84,7 +86,9 @@ def byte_model(w, T, k, window, out_bytes=2, kp_bytes=2):
     # out, indices and counts out (the scores and histograms stay on chip)
     select = (kp + w.B * w.Hq * w.dk * 2 + w.Hkv * w.dk * w.r * 4 + rows * (w.dk * 2 + w.r * kp_bytes)
               + rows * (k * 4 + 4))
-    return dict(kp=kp, selected=sel, qo=qo, step=kp + sel + qo, dense=dense, scores=rows * n * 4, select=select)
+    local = (w.layers - 1) * (rows * min(window, T) * kv_row + qo)
+    return dict(kp=kp, selected=sel, qo=qo, step=kp + sel + qo + local, dense=dense + local, scores=rows * n * 4,
+                select=select, local=local)
 
 
 def peaks():
@@ -192,7 +196,25 @@ class Setup:
         self.O = torch.empty(w.B, w.Hq, w.dv, dtype=torch.bfloat16, device=device)
         self.idx = torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=device)
         self.nsel = torch.empty(w.B, w.Hkv, dtype=torch.int32, device=device)
+        # a hybrid model's local layers: each keeps a cache of its window of W tokens only
+        self.local = []
+        if w.layers > 1:
+            g = torch.Generator(device=device)
+            g.manual_seed(w.seed * 7 + seed_offset)
+            W = w.window
+            for _ in range(w.layers - 1):
+                Kl = torch.randn(w.B, w.Hkv, W, w.dk, generator=g, device=device).to(torch.bfloat16)
+                Vl = torch.randn(w.B, w.Hkv, W, w.dv, generator=g, device=device).to(torch.bfloat16)
+                Kpl = torch.empty(w.B, w.Hkv, W, w.r, dtype=torch.bfloat16, device=device)   # unused by dense layers
+                Ll = jssa.make_layout(Kl, Vl, Kpl, w.Hq, w.r, jssa.MODE_GQA, jssa.OUT_BF16)
+                self.local.append((Kl, Vl, Ll))
+            self.local_lens = torch.full((w.B,), W, dtype=torch.int32, device=device)
+            self.local_ws = jssa.alloc_workspace(self.local[0][2], 1, 0)
         torch.cuda.synchronize()
+
+    def local_layers(self, Q):
+        for (Kl, Vl, Ll) in self.local:
+            self.jssa.dense_decode(Ll, Q, Kl, Vl, self.local_lens, 0, self.w.sm_scale, self.O, None, self.local_ws)
 
     def scoring_cache(self, kp):
         """A projected scoring cache of this workload (bf16 or E4M3) filled from K, and its layout."""
@@ -207,11 +229,13 @@ class Setup:
 
     def step(self, Q, Kp=None, L=None):
         w = self.w
-        self.jssa.decode_step(self.L if L is None else L, Q, self.K, self.V, self.Kp if Kp is None else Kp, self.P, self.seq_lens,
-                              1, w.k, w.window, w.sm_scale, self.O, None, self.idx, self.nsel, self.ws)
+        self.jssa.decode_step(self.L if L is None else L, Q, self.K, self.V, self.Kp if Kp is None else Kp, self.P,
+                              self.seq_lens, 1, w.k, w.window, w.sm_scale, self.O, None, self.idx, self.nsel, self.ws)
+        self.local_layers(Q)
 
     def dense(self, Q):
         self.jssa.dense_decode(self.L, Q, self.K, self.V, self.seq_lens, 0, self.w.sm_scale, self.O, None, self.ws)
+        self.local_layers(Q)
 
 
 def graph_of(fn, qs):
@@ -355,6 +379,8 @@ def cpu_oracle_rate(w, seconds: float, data=None, kp="bf16"):
         for (Qg, Kh, Vh, Kp, Ph) in host:
             proj(Kh[T - 1:T], Ph)                 # the newest key, projected on write
             head(Qg, Kh, Vh, Kp, Ph, T, w.k, w.window, w.sm_scale)
+            for _ in range(w.layers - 1):         # local layers: dense over a window-sized cache
+                oracle.attention(Qg, Kh[T - w.window:T], Vh[T - w.window:T], np.arange(w.window), w.sm_scale)
             n += 1
         el = time.perf_counter() - t0
         if el >= seconds:
@@ -407,10 +433,14 @@ def main():
     args = parse()
     from token_level_sparse_jssa_b200 import synth
     w = synth.WORKLOADS[args.workload]
+    if args.k > 0:
+        w = w.with_(k=args.k)
     rank, world, local = rank_env()
     bm = byte_model(w, w.T, w.k, w.window, kp_bytes=1 if args.kp == "e4m3" else 2)
     cfg = {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} d_k={w.dk} d_v={w.dv} r={w.r} T={w.T} k={w.k}"
-                       + (f" W={w.window}" if w.window else "") + f" ({w.mode.upper()})",
+                       + (f" W={w.window}" if w.window else "") + f" ({w.mode.upper()})"
+                       + (f"; {w.layers} layers: 1 global (sparse), {w.layers - 1} local (dense over the "
+                          f"{w.window}-token window caches)" if w.layers > 1 else ""),
            "global_batch": w.B * max(world, args.gpus), "seq_len": w.T, "k": w.k, "r": w.r,
            "parallelism": f"dp{max(world, args.gpus)} (independent sequences per rank, no collective)",
            "kp": "FP8 E4M3 (unit scale)" if args.kp == "e4m3" else "bf16",
@@ -447,6 +477,13 @@ def main():
     ms_step = ms / args.steps
     value = whole_job_rate(world, args.steps, ms)
     del g_warm, g_timed
+
+    # spread of the step time: 10 replays of a 50-step graph (fresh queries), per-replay means
+    g_spread = graph_of(st.step, [Qs[(args.warmup + i) % nq] for i in range(50)])
+    g_spread.replay()
+    torch.cuda.synchronize()
+    spread = sorted(max_over_ranks(timed_graph(g_spread, barrier), dist) * 1000.0 / 50 for _ in range(10))
+    del g_spread
 
     # dense full-KV comparator at the same shape (GQA; the MLA path has no dense kernel)
     dense_ms = None
@@ -486,6 +523,9 @@ def main():
         st.K[:, :, w.T - 1].copy_(newk, non_blocking=True)
         if newv is not None:
             st.V[:, :, w.T - 1].copy_(newv, non_blocking=True)
+        for (Kl, Vl, _) in st.local:
+            Kl[:, :, -1].copy_(newk, non_blocking=True)
+            Vl[:, :, -1].copy_(newv, non_blocking=True)
         st.step(Qd)
         Oh.copy_(st.O, non_blocking=True)
     e1.record()
@@ -502,6 +542,9 @@ def main():
         st.K[:, :, w.T - 1].copy_(newk, non_blocking=True)
         if newv is not None:
             st.V[:, :, w.T - 1].copy_(newv, non_blocking=True)
+        for (Kl, Vl, _) in st.local:   # the local layers' newest rows too
+            Kl[:, :, -1].copy_(newk, non_blocking=True)
+            Vl[:, :, -1].copy_(newv, non_blocking=True)
         st.step(Qd)
         Oh_all[i].copy_(st.O, non_blocking=True)
 
@@ -510,7 +553,8 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(timed_graph(g_e2e, barrier), dist)
     del g_e2e
-    h2d = Qd.numel() * 2 + newk.numel() * 2 + (newv.numel() * 2 if newv is not None else 0)
+    h2d = (Qd.numel() * 2 + (1 + len(st.local)) * newk.numel() * 2
+           + (1 + len(st.local)) * (newv.numel() * 2 if newv is not None else 0))
     d2h = Oh.numel() * Oh.element_size()
 
     code, flags = st.jssa.read_device_status(st.ws)
@@ -527,6 +571,8 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
             "us_per_step": ms_step * 1000.0, "tokens_per_s": value * w.B,
+            "us_per_step_spread": {"p10": spread[1], "p50": spread[5], "p90": spread[8],
+                                   "of": "10 replays of a 50-step graph, mean step time of each"},
             "bytes_per_step": bm["step"], "effective_GBps": bm["step"] / (ms_step * 1e-3) / 1e9,
             "step_hbm_frac": bm["step"] / (ms_step * 1e-3) / 1e9 / hbm,
             "dense_us_per_step": dense_ms * 1000.0 if dense_ms else None,
@@ -540,6 +586,7 @@ def main():
                                    "select_kernel (query and newest-key projection, score scan, top-k)",
                          "bound": "hbm", "achieved": achieved, "peak": hbm,
                          "unit": "GB/s", "frac": achieved / hbm, "peak_kind": peak_kind,
+                         "frac_of_nominal_8000_GBps": achieved / 8000.0,
                          "traffic": traffic_for("select_kernel", w.name + ("-e4m3" if args.kp == "e4m3" else ""),
                                                 shash),
                          "algorithmic_bytes_per_launch": sel_bytes},
