@@ -95,3 +95,17 @@ def test_full_size_hybrid_global_and_local_layers():
     assert_status_clean(ws)
     del p
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("k", [512, 4096])
+def test_full_size_h128k_budget_sweep(k):
+    # the 128K workload at the other budgets of its sweep (k = 4096 fills each CTA's token list)
+    w = W["h128k"].with_(k=k)
+    p = Problem(w)
+    p.fill_kp()
+    O, idx, nsel, ws = _run_step(p, k, 0, n_new=0)
+    assert int(nsel.min()) == int(nsel.max()) == k
+    check_step_rows(p, k, 0, O, idx, nsel, _sample_rows(w), f"h128k k={k}")
+    assert_status_clean(ws)
+    del p
+    torch.cuda.empty_cache()

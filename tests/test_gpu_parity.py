@@ -371,6 +371,7 @@ def test_single_token_selection_returns_the_value_row():
     ("h128k", dict(B=8, T=6000, k=512), [6000, 5000, 4097, 6000, 3000, 2000, 6000, 5999], 0),  # 64 rows: 4-CTA clusters
     ("h128k", dict(B=16, T=3000, k=256), None, 0),                            # 128 rows: 2-CTA clusters
     ("hybrid", dict(B=8, T=5000, k=300), None, 1024),                         # 64 rows, d = 256, window
+    ("h128k", dict(B=1, Hq=8, Hkv=2, T=131072, k=4096), None, 0),           # k = 4096 inside the fused kernel
 ])
 def test_decode_step_end_to_end(name, kw, seq, window):
     w = W[name].with_(**kw)
@@ -400,6 +401,7 @@ def test_decode_step_end_to_end(name, kw, seq, window):
     ("mla", dict(B=2, T=7000, k=700), [7000, 6001], 0),
     ("h128k", dict(B=1, Hq=8, Hkv=2, T=131073, k=512), [131073], 0),   # one token beyond the fused kernel
     ("llama8b", dict(B=8, T=9000, k=600), None, 0),                      # 64 rows: 4-CTA clusters
+    ("h128k", dict(B=1, Hq=8, Hkv=2, T=131072, k=4096), None, 0),        # the largest budget of the k sweep
 ])
 def test_select_matches_the_oracle_selection(name, kw, seq, window):
     w = W[name].with_(**kw)
