@@ -190,7 +190,8 @@ __global__ void __launch_bounds__(256) merge_kernel(AttnArgs a) {
 }
 
 // ------------------------------------------------------------------ host side
-void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int num_sms, int* S_out, int* split_out) {
+void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int num_sms, int d, int* S_out,
+                       int* split_out) {
   // Choose the split length (a multiple of the 16-token subtile, at least 64 tokens) that
   // keeps the last wave of CTAs fullest; fewer splits win ties.
   if (mode == 1) {
@@ -211,7 +212,10 @@ void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int n
     return;
   }
   const int min_split = 64;
-  const int slots = num_sms * 2;
+  // resident CTAs per SM: two for d <= 128 (at most 112 KB of shared memory each), one for
+  // d = 256 (its eight-warp ring takes 208 KB).  The d = 256 dense pass keeps the two-slot count:
+  // measured on 1024-token windows, its smaller two-wave splits beat one wave of longer ones.
+  const int slots = num_sms * (d >= 256 && indexed ? 1 : 2);
   if (list_max <= 0) { *S_out = 1; *split_out = min_split; return; }
   int best_S = 0;
   int64_t best_len = 0;

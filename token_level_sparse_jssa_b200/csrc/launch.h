@@ -194,7 +194,7 @@ cudaError_t launch_vote_stats(const VoteArgs& a, cudaStream_t s);      // stats,
 cudaError_t launch_vote_broadcast(const VoteArgs& a, cudaStream_t s);
 
 // Split policy shared by the workspace sizing and the launch.
-void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int num_sms, int* S, int* split_len);
+void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int num_sms, int d, int* S, int* split_len);
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);   // GQA path
 cudaError_t launch_mla_attention(const AttnArgs& a, cudaStream_t s);  // MLA path (indexed only)
 int mla_max_split();  // tokens per CTA of the MLA kernel
