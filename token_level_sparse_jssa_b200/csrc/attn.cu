@@ -212,11 +212,29 @@ void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int n
     return;
   }
   const int min_split = 64;
-  // resident CTAs per SM: two for d <= 128 (at most 112 KB of shared memory each), one for
-  // d = 256 (its eight-warp ring takes 208 KB).  The d = 256 dense pass keeps the two-slot count:
-  // measured on 1024-token windows, its smaller two-wave splits beat one wave of longer ones.
-  const int slots = num_sms * (d >= 256 && indexed ? 1 : 2);
   if (list_max <= 0) { *S_out = 1; *split_out = min_split; return; }
+  if (d >= 256) {
+    // One resident CTA per SM (the eight-warp ring takes 208 KB), and a fixed cost per CTA
+    // (prologue, ring fill, merge) worth about 256 tokens of streaming: minimise
+    // waves x (1 + len / 256), fewer splits on ties.
+    const int cap = indexed ? 8 : 256;
+    int best_S = 1;
+    int64_t best_len = ceil_div(list_max, 16) * 16;
+    double best_cost = 1e300;
+    for (int S = 1; S <= cap; ++S) {
+      int64_t len = ceil_div(ceil_div(list_max, S), 16) * 16;
+      if (len < min_split) len = min_split;
+      if (ceil_div(list_max, len) != S) continue;
+      if (indexed && len > kMaxTokList) continue;  // the token list lives in shared memory
+      const int64_t waves = ceil_div(static_cast<int64_t>(rows) * S, num_sms);
+      const double cost = static_cast<double>(waves) * (1.0 + static_cast<double>(len) / 256.0);
+      if (cost < best_cost - 1e-9) { best_cost = cost; best_S = S; best_len = len; }
+    }
+    *S_out = best_S;
+    *split_out = static_cast<int>(best_len);
+    return;
+  }
+  const int slots = num_sms * 2;  // two resident CTAs per SM (at most 112 KB of shared memory each)
   int best_S = 0;
   int64_t best_len = 0;
   double best_eff = -1.0;
