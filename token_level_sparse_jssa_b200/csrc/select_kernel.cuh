@@ -42,6 +42,7 @@ constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelStage = 16384;                   // bytes per ring stage
 constexpr int kSelMaxCluster = 16;                 // up to 8 (portable) or 16 CTAs per row
 constexpr int kSelMinCluster = 2;                  // fewer than 8 only to keep every row in one wave
+constexpr int kSelMinSlice = 512;                  // or when slices would be shorter than this (latency-bound rows)
 constexpr int kSelBins1 = 4096;                    // digit 1: key bits [31:20]
 constexpr int kSelBins2 = 1024;                    // digits 2 and 3: bits [19:10] and [9:0]
 constexpr int kSelCapW = 64;                       // per-warp capacity of the definite / candidate lists
@@ -801,7 +802,8 @@ cudaError_t launch_select_r(SelectArgs a, int num_sms, cudaStream_t s) {
   const int rows = a.B * a.Hkv;
   // Cluster size and ring depth.  Sizes are tried from the largest down: 9..16 CTAs per row
   // only when 8 per row would leave SMs idle, fewer than 8 (down to 2) only when 8 per row
-  // cannot all be resident at once.  The first size whose clusters are all resident wins, with
+  // cannot all be resident at once, and no size whose slices would be shorter than
+  // kSelMinSlice tokens (on short rows the fixed cost of a larger cluster dominates).  The first size whose clusters are all resident wins, with
   // the deepest ring that keeps them so: a second wave of clusters would pay the scan and the
   // selection's serial tail twice.  If no size fits in one wave, 8 CTAs per row run in two.
   // With the attention inside, the ring and keys areas also hold the attention's buffers, and
@@ -815,6 +817,7 @@ cudaError_t launch_select_r(SelectArgs a, int num_sms, cudaStream_t s) {
   for (int c_try = c_max; c_try >= kSelMinCluster; --c_try) {
     const int per = static_cast<int>(ceil_div(ceil_div(a.T_cap, c_try), 32) * 32);
     if (per > kSelMaxSlice) continue;
+    if (c_try > kSelMinCluster && per < kSelMinSlice) continue;               // short rows: fewer, fuller CTAs
     if (ceil_div(a.d / 8, c_try) * 8 > kSelMaxDn) continue;                    // share of the projections
     const int own_words = sel_own_words(c_try);
     if (D > 0 && ceil_div(list_max, c_try) > own_words) continue;             // token list lives in own[]
