@@ -8,16 +8,19 @@
 // index list is the dense full-KV decode used as the baseline (§4.5).
 //
 // Grid: (split, sequence * KV head).  Each CTA owns one contiguous slice of the
-// attended list (selected positions followed by the sliding window).  Its 4 warps
-// take 16-token subtiles in turn; each warp streams the subtile's K and V rows with
-// 16-byte cp.async copies (one 2*d-byte coalesced row per token, XOR-swizzled in
-// shared memory) through a private multi-stage ring, so no block barrier sits in the
-// main loop.  All G query heads of the group stay in registers as MMA operands:
-//   S^T[16 tok x 8 heads] = K_sub[16 x d] . Q^T         (mma.sync m16n8k16, bf16 -> fp32)
+// attended list (selected positions followed by the sliding window).  Its 4 warp groups
+// take 16-token subtiles in turn (a group is one warp, or for d = 256 a pair of warps
+// that each take half of the head dims and add their score partials through shared
+// memory); each warp streams its part of the subtile's K and V rows with 16-byte cp.async
+// copies (XOR-swizzled in shared memory) through a private multi-stage ring, so no block
+// barrier sits in the main loop.  All G query heads of the group stay in registers as MMA
+// operands:
+//   S^T[16 tok x 8 heads] = K_sub[16 x d] . Q^T         (mma.sync m16n8k16, bf16 -> fp32,
+//                                                        even and odd K-steps in two chains)
 //   online softmax per head in fp32 (exp2 domain)
 //   O^T[d x 8 heads]     += V_sub^T . P^T               (P split into bf16 hi + lo parts,
 //                                                        so the weights keep ~16 bits)
-// The 4 warps' states are merged in shared memory into one normalised partial (o, lse)
+// The 4 groups' states are merged in shared memory into one normalised partial (o, lse)
 // per query head.  Indexed attention runs the S <= 8 splits of a row as one thread-block
 // cluster and combines the partials by log-sum-exp through distributed shared memory;
 // the dense decode, with many more splits, writes partials to the workspace and the last
