@@ -235,47 +235,3 @@ def decode_head_e4m3(Qg, K, V, Kp8, P, T: int, k: int, W: int, scale: float):
     toks = np.concatenate([idx[:k_eff].astype(np.int64), np.arange(n, T, dtype=np.int64)])
     O, lse = attention(Qg, K, V, toks, scale)
     return dict(idx=idx, k_eff=k_eff, O=O, lse=lse, scores=s)
-
-
-# --------------------------------------------------------------------------- whole tensors
-def project_cache(K: np.ndarray, P: np.ndarray, T: int | None = None) -> np.ndarray:
-    """Kp for rows [0, T) of every (b, h) of a [B, Hkv, T_cap, d] cache; rows >= T stay 0."""
-    B, H, Tc, d = K.shape
-    r = P.shape[-1]
-    T = Tc if T is None else T
-    Kp = np.zeros((B, H, Tc, r), np.uint16)
-    for b in range(B):
-        for h in range(H):
-            Kp[b, h, :T] = project_rows(K[b, h, :T], P[h])[0]
-    return Kp
-
-
-def decode_step(Q, K, V, Kp, P, seq_lens, k: int, W: int, scale: float, rows=None):
-    """Whole decode step over a batch (GQA: Hq = G * Hkv; MLA: Hkv = 1).
-
-    Q uint16 [B, Hq, dk]; K uint16 [B, Hkv, T_cap, dk]; V uint16 [B, Hkv, T_cap, dv]
-    (may be a strided view of K for MLA); Kp uint16 [B, Hkv, T_cap, r]; P float32 [Hkv, dk, r].
-    ``rows`` optionally restricts the work to a list of (b, h) pairs.
-    Returns dict(idx [B, Hkv, k], n_sel [B, Hkv], O [B, Hq, dv], lse [B, Hq], scores {(b,h): s}).
-    Entries for rows not computed are left as NaN / -1.
-    """
-    B, Hq, dk = Q.shape
-    Hkv = K.shape[1]
-    dv = V.shape[-1]
-    G = Hq // Hkv
-    idx = np.full((B, Hkv, k), -1, np.int32)
-    n_sel = np.full((B, Hkv), -1, np.int64)
-    O = np.full((B, Hq, dv), np.nan)
-    lse = np.full((B, Hq), np.nan)
-    sc = {}
-    todo = rows if rows is not None else [(b, h) for b in range(B) for h in range(Hkv)]
-    for (b, h) in todo:
-        T = int(seq_lens[b])
-        res = decode_head(Q[b, h * G:(h + 1) * G], K[b, h, :max(T, 1)], V[b, h, :max(T, 1)],
-                          Kp[b, h, :max(T, 1)], P[h], T, k, W, scale)
-        idx[b, h] = res["idx"]
-        n_sel[b, h] = res["k_eff"]
-        O[b, h * G:(h + 1) * G] = res["O"]
-        lse[b, h * G:(h + 1) * G] = res["lse"]
-        sc[(b, h)] = res["scores"]
-    return dict(idx=idx, n_sel=n_sel, O=O, lse=lse, scores=sc)

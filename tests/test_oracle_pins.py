@@ -336,18 +336,6 @@ def test_step_mla_shape_reduces_to_gqa_formula():
     np.testing.assert_allclose(res["O"], O, atol=1e-13)
 
 
-def test_whole_batch_decode_step_on_tiny_workload():
-    w = synth.WORKLOADS["tiny"].with_(T=512, k=32)
-    x = synth.make_inputs(w, seq_lens=[500])
-    Q, K, V, P = u16(x["Q"]), u16(x["K"]), u16(x["V"]), f32(x["P"])
-    Kp = oracle.project_cache(K, P)
-    out = oracle.decode_step(Q, K, V, Kp, P, x["seq_lens"].numpy(), w.k, 0, w.sm_scale)
-    assert out["idx"].shape == (1, 2, 32) and np.all(out["n_sel"] == 32)
-    assert np.all(out["idx"] < 500) and np.all(np.diff(out["idx"], axis=-1) > 0)
-    # heavy (x4) rows dominate the selection of this generator
-    assert np.isfinite(out["O"]).all()
-
-
 # ----------------------------------------------------------------------------- FP8 E4M3 projected cache
 def test_e4m3_decodes_the_format_constants():
     # OCP E4M3: bias 7, 3 mantissa bits, subnormals m * 2^-9, S.1111.111 is NaN, max 448
