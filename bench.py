@@ -48,9 +48,9 @@ def step_kernels(w) -> tuple[int, bool]:
     """Kernels one decode step launches, and whether the attention runs inside the selection
     kernel (GQA with d <= 128 and G <= 16 on caches the selection kernel covers)."""
     if w.T > FUSED_MAX_T:
-        return (4 if w.mode != "mla" else 5), False   # prologue, score, top-k, attention (+ merge)
+        return 4, False                                  # prologue, score, top-k, attention
     if w.mode == "mla":
-        return 3, False                                  # selection, tensor-core attention, merge
+        return 2, False                                  # selection, tensor-core attention (merge inside)
     fused = w.dk <= 128 and w.G <= 16
     return (1 if fused else 2) + (w.layers - 1), fused   # + one dense kernel per local layer
 
@@ -89,6 +89,16 @@ def byte_model(w, T, k, window, out_bytes=2, kp_bytes=2):
     local = (w.layers - 1) * (rows * min(window, T) * kv_row + qo)
     return dict(kp=kp, selected=sel, qo=qo, step=kp + sel + qo + local, dense=dense + local, scores=rows * n * 4,
                 select=select, local=local)
+
+
+def tensor_peak():
+    """Measured sustained dense bf16 tensor throughput (TFLOP/s), for kernels timed in long loops."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d["bf16_tflops_sustained"], "measured"
+    except Exception:
+        return 1400.0, "fallback"
 
 
 def peaks():
@@ -189,6 +199,18 @@ class Setup:
         self.seq_lens = x["seq_lens"]
         self.A = x["A"]
         self.T_cap = x["T_cap"]
+        # an appending workload (w.steps > 1 decode steps): the cache starts with T - steps
+        # tokens; step i writes token T - steps + i (its K/V row, kept aside here as the stream
+        # of generated rows) with jssa_append_kv, projects it on write (n_new = 1) and attends
+        # over the lengthened sequence; the loop wraps after w.steps steps
+        self.appending = w.steps > 1
+        if self.appending:
+            S, t0 = w.steps, w.T - w.steps
+            self.Knew = self.K[:, :, t0:w.T].permute(2, 0, 1, 3).contiguous()
+            self.Vnew = self.V[:, :, t0:w.T].permute(2, 0, 1, 3).contiguous() if w.mode != "mla" else None
+            ar = torch.arange(S, device=device, dtype=torch.int32)
+            self.SL = (t0 + 1 + ar).view(S, 1).repeat(1, w.B).contiguous()   # [S, B] lengths at step i
+            self.POS = (self.SL - 1).contiguous()                              # [S, B] the row step i writes
         self.Kp, self.L = self.scoring_cache(kp)
         self.kp = kp
         self.ws = jssa.alloc_workspace(self.L, w.k, w.window)
@@ -224,17 +246,33 @@ class Setup:
         L = jssa.make_layout(self.K, self.V, Kp, w.Hq, w.r, jssa.MODE_MLA if w.mode == "mla" else jssa.MODE_GQA,
                              jssa.OUT_BF16)
         tb = torch.zeros(w.B, dtype=torch.int32, device=self.K.device)
-        jssa.project_keys(L, self.K, self.P, Kp, self.T_cap, t_begin=tb)   # prefill fill
+        filled = self.T_cap - (w.steps if self.appending else 0)
+        jssa.project_keys(L, self.K, self.P, Kp, filled, t_begin=tb)   # prefill fill
+        if filled < self.T_cap:
+            Kp[:, :, filled:].zero_()   # rows the appending steps write
         return Kp, L
 
-    def step(self, Q, Kp=None, L=None):
+    def step(self, Q, i=0, Kp=None, L=None, kv_new=None):
+        """Decode step i with query Q.  Appending workloads first write the step's token (from
+        kv_new, else from the stream of generated rows) with jssa_append_kv; every step projects
+        the newest key on write (n_new = 1)."""
         w = self.w
-        self.jssa.decode_step(self.L if L is None else L, Q, self.K, self.V, self.Kp if Kp is None else Kp, self.P,
-                              self.seq_lens, 1, w.k, w.window, w.sm_scale, self.O, None, self.idx, self.nsel, self.ws)
+        L = self.L if L is None else L
+        if self.appending:
+            j = i % w.steps
+            kn, vn = kv_new if kv_new is not None else (self.Knew[j], self.Vnew[j] if self.Vnew is not None else None)
+            self.jssa.append_kv(L, kn, vn, self.K, self.V if vn is not None else None, self.POS[j])
+            sl = self.SL[j]
+        else:
+            sl = self.seq_lens
+        self.jssa.decode_step(L, Q, self.K, self.V, self.Kp if Kp is None else Kp, self.P,
+                              sl, 1, w.k, w.window, w.sm_scale, self.O, None, self.idx, self.nsel, self.ws)
         self.local_layers(Q)
 
     def dense(self, Q):
-        self.jssa.dense_decode(self.L, Q, self.K, self.V, self.seq_lens, 0, self.w.sm_scale, self.O, None, self.ws)
+        # an appending workload's comparator runs at the loop's mean length
+        sl = self.SL[self.w.steps // 2] if self.appending else self.seq_lens
+        self.jssa.dense_decode(self.L, Q, self.K, self.V, sl, 0, self.w.sm_scale, self.O, None, self.ws)
         self.local_layers(Q)
 
 
@@ -280,15 +318,15 @@ def stage_times(st, Q, reps=50):
         "vote_select_us": lambda: jssa.vote_select(st.L, Q, st.K, st.Kp, st.P, st.seq_lens, 1, w.k, w.window,
                                                    w.sm_scale, st.idx, st.nsel, st.ws),
     }
-    if st.w.mode != "mla":  # the MLA path is indexed only
-        calls["dense_us"] = lambda: st.dense(Q)
+    calls["dense_us"] = lambda: st.dense(Q)
+    if st.w.mode != "mla":  # (the gather-based comparator is GQA only)
         # the gather-based baseline of the pages: copy the attended rows, then dense decode on them
         calls["gather_then_attend_us"] = lambda: jssa.gather_decode(st.L, Q, st.K, st.V, st.idx, w.k, st.nsel,
                                                                     st.seq_lens, w.window, w.sm_scale, st.O, None,
                                                                     st.gbuf, st.ws)
     other = "bf16" if st.kp == "e4m3" else "e4m3"
     Kp2, L2 = st.scoring_cache(other)
-    calls[f"step_kp_{other}_us"] = lambda: st.step(Q, Kp2, L2)
+    calls[f"step_kp_{other}_us"] = lambda: st.step(Q, 0, Kp2, L2)
     out = {}
     for name, fn in calls.items():
         fn()
@@ -392,6 +430,20 @@ def cpu_oracle_rate(w, seconds: float, data=None, kp="bf16"):
     return 1.0 / step_s, desc
 
 
+def host_cpu() -> dict:
+    """The host the CPU baseline runs on: its logical CPU count and model name."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cpus": os.cpu_count(), "cpu_model": model}
+
+
 # --------------------------------------------------------------------------- ranks
 def rank_env():
     """(rank, world, local_rank) from the launcher's environment (1 process when absent)."""
@@ -423,7 +475,8 @@ def run_reference(args, w, cfg):
     line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / rate, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
-            "cpu_baseline": {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
+                             **host_cpu()},
             "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -436,11 +489,16 @@ def main():
     if args.k > 0:
         w = w.with_(k=args.k)
     rank, world, local = rank_env()
-    bm = byte_model(w, w.T, w.k, w.window, kp_bytes=1 if args.kp == "e4m3" else 2)
+    # an appending workload's sequences grow from T - steps + 1 to T over its loop: bytes at the mean length
+    T_bytes = w.T - w.steps // 2 if w.steps > 1 else w.T
+    bm = byte_model(w, T_bytes, w.k, w.window, kp_bytes=1 if args.kp == "e4m3" else 2)
     cfg = {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} d_k={w.dk} d_v={w.dv} r={w.r} T={w.T} k={w.k}"
                        + (f" W={w.window}" if w.window else "") + f" ({w.mode.upper()})"
                        + (f"; {w.layers} layers: 1 global (sparse), {w.layers - 1} local (dense over the "
-                          f"{w.window}-token window caches)" if w.layers > 1 else ""),
+                          f"{w.window}-token window caches)" if w.layers > 1 else "")
+                       + (f"; appending: each step writes one token (jssa_append_kv) and projects it on write, "
+                          f"the sequences growing from T={w.T - w.steps + 1} to T={w.T} over a {w.steps}-step loop"
+                          if w.steps > 1 else ""),
            "global_batch": w.B * max(world, args.gpus), "seq_len": w.T, "k": w.k, "r": w.r,
            "parallelism": f"dp{max(world, args.gpus)} (independent sequences per rank, no collective)",
            "kp": "FP8 E4M3 (unit scale)" if args.kp == "e4m3" else "bf16",
@@ -467,10 +525,13 @@ def main():
     nq = args.warmup + args.steps
     Qs = synth.fresh_queries(w, nq, st.A, device="cuda", seed=7 + rank)
     # warm-up (untimed), then exactly `steps` timed steps, each in one CUDA graph
-    g_warm = graph_of(st.step, [Qs[i] for i in range(args.warmup)])
+    run = lambda it: st.step(it[1], it[0])   # (step index, query)
+    g_warm = graph_of(run, [(i, Qs[i]) for i in range(args.warmup)])
     g_warm.replay()
     torch.cuda.synchronize()
-    g_timed = graph_of(st.step, [Qs[args.warmup + i] for i in range(args.steps)])
+    g_timed = graph_of(run, [(args.warmup + i, Qs[args.warmup + i]) for i in range(args.steps)])
+    g_timed.replay()   # the graph's first launch uploads it to the device: keep that out of the timing
+    torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         ms = timed_graph(g_timed, barrier)
     ms = max_over_ranks(ms, dist)
@@ -479,16 +540,16 @@ def main():
     del g_warm, g_timed
 
     # spread of the step time: 10 replays of a 50-step graph (fresh queries), per-replay means
-    g_spread = graph_of(st.step, [Qs[(args.warmup + i) % nq] for i in range(50)])
+    g_spread = graph_of(run, [(args.warmup + i, Qs[(args.warmup + i) % nq]) for i in range(50)])
     g_spread.replay()
     torch.cuda.synchronize()
     spread = sorted(max_over_ranks(timed_graph(g_spread, barrier), dist) * 1000.0 / 50 for _ in range(10))
     del g_spread
 
-    # dense full-KV comparator at the same shape (GQA; the MLA path has no dense kernel)
+    # dense full-KV comparator at the same shape (the latent model's runs on the tensor cores)
     dense_ms = None
-    if w.mode != "mla":
-        nd = max(5, min(200, args.steps // 10))
+    if True:
+        nd = max(5, min(200 if w.mode != "mla" else 20, args.steps // 10))
         g_dw = graph_of(st.dense, [Qs[i] for i in range(3)])
         g_dw.replay()
         g_d = graph_of(st.dense, [Qs[i % nq] for i in range(nd)])
@@ -503,66 +564,65 @@ def main():
     sel_s = stages["select_us"] * 1e-6
     shash = source_hash("select_kernel.cuh", "attn_core.cuh", "common.cuh")
 
-    # end to end through the public API with host buffers: per step, H2D of the query and of
-    # the newest token's K/V rows from pinned memory, the step, and D2H of the output
+    # end to end through the public API with host buffers.  Per step: ONE host-to-device copy
+    # of a packed pinned buffer [query | newest K rows | newest V rows] into a device staging
+    # buffer, the append-on-write call that writes the newest rows into every layer's cache
+    # (jssa_append_kv), the decode step reading its query from the staging buffer, and ONE
+    # device-to-host copy of the output.
     ne = max(10, min(500, args.steps // 4))
-    Qh = Qs[:ne].cpu().pin_memory()
-    newk = st.K[:, :, w.T - 1].contiguous().cpu().pin_memory()
-    newv = st.V[:, :, w.T - 1].contiguous().cpu().pin_memory() if w.mode != "mla" else None
-    Oh = torch.empty(st.O.shape, dtype=st.O.dtype).pin_memory()
-    Qd = torch.empty_like(Qs[0])
+    jssa = st.jssa
+    nq, nk = w.B * w.Hq * w.dk, w.B * w.Hkv * w.dk
+    nv = w.B * w.Hkv * w.dv if w.mode != "mla" else 0
+    stage_h = torch.empty(ne, nq + nk + nv, dtype=torch.bfloat16).pin_memory()
+    stage_h[:, :nq] = Qs[:ne].reshape(ne, nq).cpu()
+    stage_h[:, nq:nq + nk] = st.K[:, :, w.T - 1].reshape(1, nk).cpu()
+    if nv:
+        stage_h[:, nq + nk:] = st.V[:, :, w.T - 1].reshape(1, nv).cpu()
+    stage_d = torch.empty(nq + nk + nv, dtype=torch.bfloat16, device="cuda")
+    Qd = stage_d[:nq].view(w.B, w.Hq, w.dk)
+    Kn = stage_d[nq:nq + nk].view(w.B, w.Hkv, w.dk)
+    Vn = stage_d[nq + nk:].view(w.B, w.Hkv, w.dv) if nv else None
+    pos = (st.seq_lens - 1).to(torch.int32)
+    local_pos = torch.full((w.B,), w.window - 1, dtype=torch.int32, device="cuda") if st.local else None
+    Oh_all = torch.empty((ne,) + tuple(st.O.shape), dtype=st.O.dtype).pin_memory()
+
+    def e2e_step(i):
+        stage_d.copy_(stage_h[i], non_blocking=True)
+        if not st.appending:   # (an appending workload's step appends from the staging buffer itself)
+            jssa.append_kv(st.L, Kn, Vn, st.K, st.V if nv else None, pos)
+        for (Kl, Vl, Ll) in st.local:   # the local layers' caches take the same newest rows
+            jssa.append_kv(Ll, Kn, Vn, Kl, Vl, local_pos)
+        st.step(Qd, i, kv_new=(Kn, Vn))
+        Oh_all[i].copy_(st.O, non_blocking=True)
+
     for i in range(3):
-        Qd.copy_(Qh[i], non_blocking=True)
-        st.step(Qd)
+        e2e_step(i)
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for i in range(ne):
-        Qd.copy_(Qh[i], non_blocking=True)
-        st.K[:, :, w.T - 1].copy_(newk, non_blocking=True)
-        if newv is not None:
-            st.V[:, :, w.T - 1].copy_(newv, non_blocking=True)
-        for (Kl, Vl, _) in st.local:
-            Kl[:, :, -1].copy_(newk, non_blocking=True)
-            Vl[:, :, -1].copy_(newv, non_blocking=True)
-        st.step(Qd)
-        Oh.copy_(st.O, non_blocking=True)
+        e2e_step(i)
     e1.record()
     torch.cuda.synchronize()
     barrier()
     e2e_eager_ms = max_over_ranks(e0.elapsed_time(e1), dist)
     # the same loop as a decode server would run it: the ne steps' copies and calls captured in
-    # one CUDA graph (the entry points are capturable), replayed once; every step still copies
-    # its own query and K/V rows from pinned host memory and its own output back to the host
-    Oh_all = torch.empty((ne,) + tuple(st.O.shape), dtype=st.O.dtype).pin_memory()
-
-    def e2e_step(i):
-        Qd.copy_(Qh[i], non_blocking=True)
-        st.K[:, :, w.T - 1].copy_(newk, non_blocking=True)
-        if newv is not None:
-            st.V[:, :, w.T - 1].copy_(newv, non_blocking=True)
-        for (Kl, Vl, _) in st.local:   # the local layers' newest rows too
-            Kl[:, :, -1].copy_(newk, non_blocking=True)
-            Vl[:, :, -1].copy_(newv, non_blocking=True)
-        st.step(Qd)
-        Oh_all[i].copy_(st.O, non_blocking=True)
-
+    # one CUDA graph (the entry points are capturable), replayed once untimed, then timed
     g_e2e = graph_of(e2e_step, list(range(ne)))
     g_e2e.replay()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(timed_graph(g_e2e, barrier), dist)
     del g_e2e
-    h2d = (Qd.numel() * 2 + (1 + len(st.local)) * newk.numel() * 2
-           + (1 + len(st.local)) * (newv.numel() * 2 if newv is not None else 0))
-    d2h = Oh.numel() * Oh.element_size()
+    h2d = (nq + nk + nv) * 2
+    d2h = st.O.numel() * st.O.element_size()
 
     code, flags = st.jssa.read_device_status(st.ws)
     if rank == 0:
         cpu = None
         if not args.no_cpu_baseline and world == 1:
             rate, desc = cpu_oracle_rate(w, args.cpu_seconds, data=(st.K, st.V, Qs[0], st.P), kp=args.kp)
-            cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+            cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc, **host_cpu()}
         # the dominant kernel: with the attention inside, the step is that one kernel and its
         # launch time is the step time measured above; otherwise the selection kernel alone
         achieved = sel_bytes / (ms_step * 1e-3 if fused else sel_s) / 1e9
@@ -579,6 +639,10 @@ def main():
             "speedup_vs_dense": dense_ms / ms_step if dense_ms else None,
             "byte_ratio": bm["dense"] / bm["step"],
             "dense_hbm_frac": bm["dense"] / (dense_ms * 1e-3) / 1e9 / hbm if dense_ms else None,
+            # the latent model's dense step is a contraction (2 B Hq T (d_k + d_v) flops): its fraction
+            # of the measured sustained bf16 tensor peak
+            "dense_tensor_frac": (2.0 * w.B * w.Hq * w.T * (w.dk + w.dv) / (dense_ms * 1e-3) / 1e12 /
+                                  tensor_peak()[0]) if (dense_ms and w.mode == "mla") else None,
             "stage_us": stages,
             "calibration": calib,
             "roofline": {"kernel": ("select_kernel (the whole step: query and newest-key projection, score scan, "
@@ -593,8 +657,9 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": whole_job_rate(world, ne, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": ne,
-                    "mode": "per step: H2D of the query and the newest K/V rows from pinned memory, the "
-                            "decode_step call, D2H of the output; the steps captured in one CUDA graph"},
+                    "mode": "per step: one H2D copy of a packed pinned buffer (query, newest K and V rows), "
+                            "jssa_append_kv into every layer's cache, the decode_step call, one D2H copy of the "
+                            "output; the steps captured in one CUDA graph"},
             "e2e_eager": {"value": whole_job_rate(world, ne, e2e_eager_ms), "unit": UNIT,
                           "mode": "the same loop issued call by call from Python"},
             "gpu_launches": n_kernels * args.steps,

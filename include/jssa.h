@@ -135,6 +135,20 @@ JSSA_API int32_t jssa_version(void);
 JSSA_API jssa_status jssa_workspace_size(const jssa_layout* L, int32_t k, int32_t window, size_t* bytes);
 
 /*
+ * Append on write (§3.1, §E.1: a generated key enters the cache, and is projected, when it
+ * is written): copies the newest key and value rows of every (sequence, KV head) into
+ * row t_pos[b] of the caches; jssa_decode_step with n_new = 1 then projects that row.
+ *   K_new  device bf16 [B, Hkv, d_k], contiguous, 16-byte aligned;
+ *   V_new  device bf16 [B, Hkv, d_v], contiguous, 16-byte aligned (GQA); NULL in MLA mode,
+ *          where V is the leading d_v dims of the latent row K (V is then ignored);
+ *   K, V   the layout's caches;
+ *   t_pos  device int32 [B]; sequences whose t_pos lies outside [0, T_cap) are not written.
+ * Asynchronous on `stream`; allocates nothing.
+ */
+JSSA_API jssa_status jssa_append_kv(const jssa_layout* L, const void* K_new, const void* V_new, void* K, void* V,
+                                    const int32_t* t_pos, void* stream);
+
+/*
  * Projected scoring cache on write (§3.1, §3.4, §E.1):
  *   Kp[b, h, t, :] = rnd(K[b, h, t, :] . P_h)   for t in [t_begin[b], t_begin[b] + n_tokens)
  * with rnd = bf16 or E4M3 (saturating) rounding to nearest even, by kp_dtype.
@@ -183,7 +197,8 @@ JSSA_API jssa_status jssa_topk(const jssa_layout* L, const float* scores, const 
  * address (once per device); make that first call before any stream capture.  All
  * calls share one scratch, so calls that may overlap on the GPU (other streams, other
  * host threads) race and must be serialised by the caller.  No device status word is
- * kept.
+ * kept: a row whose bounded wait gave up returns an empty selection (n_sel = 0, idx all
+ * -1), which is how a caller of this entry point detects it.
  */
 JSSA_API jssa_status jssa_topk_noalloc(const jssa_layout* L, const float* scores, const int32_t* seq_lens,
                                        int32_t k, int32_t window, int32_t* idx, int32_t* n_sel, void* stream);
@@ -296,6 +311,20 @@ JSSA_API jssa_status jssa_calibrate(const jssa_layout* L, const void* Qc, const 
  * its first use by any compute call, and again after a call that returned an error.
  */
 JSSA_API jssa_status jssa_workspace_init(void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Test of the bounded waits (the paper has no counterpart; this is for checking the
+ * library's failure path on a working GPU, without faulting it).  Arms a one-shot request
+ * in the workspace, asynchronously on `stream`: the next selection launch that scans with
+ * this workspace (jssa_select, jssa_decode_step, jssa_topk; rows of at least k + 1
+ * candidates) withholds one bulk copy in the first CTA of row (0, 0), whose wait on it
+ * then gives up after wait_limit_us microseconds (1 .. 1,000,000).  The launch returns
+ * normally: its device status has JSSA_DEV_TIMEOUT (jssa_read_device_status returns
+ * JSSA_ERR_TIMEOUT), row (0, 0) has an empty selection (n_sel = 0, idx all -1; with the
+ * attention inside the step, its output is the attention over the window alone, zero
+ * without one) and the other rows are unaffected.  The launch disarms the request.
+ */
+JSSA_API jssa_status jssa_test_withhold_copy(void* workspace, size_t ws_bytes, int32_t wait_limit_us, void* stream);
 
 /*
  * Read and clear the device status word kept in the workspace (JSSA_DEV_* bits).

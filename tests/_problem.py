@@ -28,6 +28,7 @@ class Problem:
         self.w = w
         x = synth.make_inputs(w, device=gen_device, T_cap=T_cap, seq_lens=seq_lens, seed=seed)
         self.T_cap = x["T_cap"]
+        self.A = x["A"]
         self.Q = x["Q"].to(device)
         self.K = x["K"].to(device)
         if w.mode == "mla":

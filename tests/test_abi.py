@@ -119,10 +119,16 @@ def test_bad_layouts_are_rejected_on_the_host(lib, kw, code):
         assert got == code
 
 
-def test_mla_dense_decode_is_unsupported(lib):
-    # the MLA path is indexed only: the dense entry point refuses the layout before launching
+def test_mla_dense_decode_validates_on_the_host(lib):
+    # the latent layout has a dense (full-cache comparator) path: its arguments are checked
+    # before anything is launched
     L = _layout(mode=1, B=1, Hq=128, Hkv=1, d=576, dv=512, r=64)
-    assert lib.jssa_dense_decode(C.byref(L), FAKE, FAKE, FAKE, FAKE, 0, 1.0, FAKE, None, C.c_void_p(FAKE), 1 << 30,
+    assert lib.jssa_dense_decode(C.byref(L), None, FAKE, FAKE, FAKE, 0, 1.0, FAKE, None, C.c_void_p(FAKE), 1 << 30,
+                                 None) == 1
+    assert lib.jssa_dense_decode(C.byref(L), FAKE, FAKE, FAKE, FAKE, -1, 1.0, FAKE, None, C.c_void_p(FAKE), 1 << 30,
+                                 None) == 1
+    bad = _layout(mode=1, B=1, Hq=64, Hkv=1, d=576, dv=512, r=64)   # the latent kernel takes 128 heads
+    assert lib.jssa_dense_decode(C.byref(bad), FAKE, FAKE, FAKE, FAKE, 0, 1.0, FAKE, None, C.c_void_p(FAKE), 1 << 30,
                                  None) == 2
 
 

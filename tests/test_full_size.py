@@ -50,25 +50,40 @@ def test_full_size_single_step(name):
     torch.cuda.empty_cache()
 
 
-def test_full_size_llama8b_appending_steps():
-    # the Llama-3.1-8B-shaped layer: each decode step appends one token (its K/V row is
-    # written to the cache) and the step projects it into the scoring cache on write
+def test_full_size_llama8b_appending_loop():
+    # the Llama-3.1-8B-shaped layer as its workload runs it: 1000 decode steps, each appending
+    # one token (jssa_append_kv writes its K/V row into the cache) that the step projects into
+    # the scoring cache on write, with a fresh query batch every step; the selection and the
+    # output are checked against the oracle after the first, a middle and the last step
     w = W["llama8b"]
-    steps = 3
-    p = Problem(w, seq_lens=[w.T - steps] * w.B)
+    steps = w.steps
+    t0 = w.T - steps
+    p = Problem(w, seq_lens=[t0] * w.B)
+    new_k = p.K[:, :, t0:w.T].permute(2, 0, 1, 3).contiguous()   # the generated rows, step by step
+    new_v = p.V[:, :, t0:w.T].permute(2, 0, 1, 3).contiguous()
+    p.K[:, :, t0:].zero_()
+    p.V[:, :, t0:].zero_()
     tb = torch.zeros(w.B, dtype=torch.int32, device="cuda")
-    jssa.project_keys(p.L, p.K, p.P, p.Kp, w.T - steps, t_begin=tb)
+    jssa.project_keys(p.L, p.K, p.P, p.Kp, t0, t_begin=tb)
+    Qs = synth.fresh_queries(w, steps, p.A, device="cuda", seed=11)
     ws = p.workspace(w.k)
     O = torch.empty((w.B, w.Hq, w.dv), device="cuda")
     idx = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device="cuda")
     nsel = torch.empty((w.B, w.Hkv), dtype=torch.int32, device="cuda")
-    for _ in range(steps):
+    checked = 0
+    for i in range(steps):
+        jssa.append_kv(p.L, new_k[i], new_v[i], p.K, p.V, p.seq_lens)   # row seq_len: the new token
         p.seq_lens += 1
-        jssa.decode_step(p.L, p.Q, p.K, p.V, p.Kp, p.P, p.seq_lens, 1, w.k, 0, w.sm_scale, O, None, idx, nsel, ws)
-    torch.cuda.synchronize()
-    assert int(p.seq_lens.min()) == w.T
-    check_step_rows(p, w.k, 0, O, idx, nsel, _sample_rows(w), "llama8b full size", kp_checked=True)
-    assert_status_clean(ws)
+        jssa.decode_step(p.L, Qs[i], p.K, p.V, p.Kp, p.P, p.seq_lens, 1, w.k, 0, w.sm_scale, O, None, idx, nsel,
+                         ws)
+        if i in (0, steps // 2, steps - 1):
+            torch.cuda.synchronize()
+            assert int(p.seq_lens.min()) == int(p.seq_lens.max()) == t0 + i + 1
+            p.Q = Qs[i].contiguous()
+            check_step_rows(p, w.k, 0, O, idx, nsel, _sample_rows(w), f"llama8b step {i}", kp_checked=True)
+            assert_status_clean(ws)
+            checked += 1
+    assert checked == 3 and int(p.seq_lens.min()) == w.T
     del p
     torch.cuda.empty_cache()
 

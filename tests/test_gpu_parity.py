@@ -204,6 +204,8 @@ def test_topk_with_few_distinct_values(T, k, levels):
     ("mla", dict(B=1, T=4100), [4100], 2048, 0, 0),                          # 16 full 128-token tiles
     ("mla", dict(B=3, T=2000), [2000, 333, 1999], 150, 64, 0),               # ragged tiles + window
     ("mla", dict(B=1, T=1000), [1000], 37, 5, 1),                            # bf16 output
+    ("mla", dict(B=1, T=20000), [20000], 4096, 0, 0),                        # four tiles per CTA
+    ("mla", dict(B=16, T=3000), None, 2048, 0, 0),                           # the workload's 16 sequences
 ])
 def test_indexed_attention_matches_oracle(name, kw, seq, k, window, out):
     w = W[name].with_(**kw)
@@ -332,13 +334,33 @@ def test_mla_single_token_returns_the_latent_value_row():
     _assert_status_clean(ws)
 
 
-def test_mla_has_no_dense_path():
-    w = W["mla"].with_(B=1, T=300)
+@pytest.mark.parametrize("B,T,window,growth,qscale", [
+    (1, 300, 0, 0.0, 1.0),        # one tile per CTA (eight CTAs, ragged)
+    (2, 2500, 0, 0.0, 1.0),       # several tiles per CTA
+    (3, 1800, 700, 0.0, 1.0),     # the window form (local layer of a latent model)
+    (1, 4000, 0, 6.0, 24.0),      # logits growing along the cache: the running maxima move and the
+                                  # resident output is rescaled on later tiles
+])
+def test_mla_dense_decode_matches_oracle(B, T, window, growth, qscale):
+    # the full-cache comparator of the latent model (§4.5 full-KV baseline) on the tensor cores
+    w = W["mla"].with_(B=B, T=T)
     p = Problem(w)
-    ws = p.workspace(4)
-    O = torch.empty((w.B, w.Hq, w.dv), device="cuda")
-    with pytest.raises(jssa.JssaError):
-        jssa.dense_decode(p.L, p.Q, p.K, p.V, p.seq_lens, 0, w.sm_scale, O, ws=ws)
+    if growth:
+        ramp = 1.0 + growth * torch.arange(T, device="cuda", dtype=torch.float32) / T
+        p.K.copy_((p.K.float() * ramp.view(1, 1, T, 1)).to(torch.bfloat16))
+        p.Q.copy_((p.Q.float() * qscale).to(torch.bfloat16))
+    ws = p.workspace(4, window)
+    O = torch.full((w.B, w.Hq, w.dv), float("nan"), device="cuda")
+    lse = torch.full((w.B, w.Hq), float("nan"), device="cuda")
+    jssa.dense_decode(p.L, p.Q, p.K, p.V, p.seq_lens, window, w.sm_scale, O, lse, ws=ws)
+    torch.cuda.synchronize()
+    for b in range(w.B):
+        hst = p.host(b, 0)
+        toks = np.arange(T - window, T) if window else np.arange(T)
+        O_ref, lse_ref = oracle.attention(hst["Q"], hst["K"], hst["V"], toks, w.sm_scale)
+        check_attention(O[b].cpu().numpy().astype(np.float64), O_ref, f"b={b}")
+        np.testing.assert_allclose(lse[b].cpu().numpy(), lse_ref, atol=1e-4, rtol=1e-5)
+    _assert_status_clean(ws)
 
 
 def test_single_token_selection_returns_the_value_row():

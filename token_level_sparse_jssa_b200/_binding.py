@@ -28,7 +28,7 @@ EXPORTS = ("jssa_status_string", "jssa_version", "jssa_workspace_size", "jssa_pr
            "jssa_topk", "jssa_topk_noalloc", "jssa_select", "jssa_indexed_attn", "jssa_decode_step",
            "jssa_dense_decode", "jssa_gather_size", "jssa_gather_decode", "jssa_calibrate_workspace_size",
            "jssa_calibrate", "jssa_vote_select",
-           "jssa_workspace_init", "jssa_read_device_status")
+           "jssa_workspace_init", "jssa_read_device_status", "jssa_test_withhold_copy", "jssa_append_kv")
 
 
 class JssaError(RuntimeError):
@@ -77,6 +77,8 @@ def load(path: str = LIB_PATH):
         "jssa_vote_select": (C.c_int, [LP, vp, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, sz, vp]),
         "jssa_workspace_init": (C.c_int, [vp, sz, vp]),
         "jssa_read_device_status": (C.c_int, [vp, sz, C.POINTER(i32), vp]),
+        "jssa_test_withhold_copy": (C.c_int, [vp, sz, i32, vp]),
+        "jssa_append_kv": (C.c_int, [LP, vp, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -164,6 +166,12 @@ def alloc_workspace(L: Layout, k: int, window: int = 0, device=None) -> torch.Te
     ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
     workspace_init(ws)
     return ws
+
+
+def append_kv(L, K_new, V_new, K, V, t_pos, stream=None):
+    """Write the newest K (and V) row of every (sequence, KV head) into row t_pos[b]."""
+    _check("jssa_append_kv", load().jssa_append_kv(C.byref(L), _c(K_new), _c(V_new), _p(K), _p(V), _c(t_pos),
+                                                   _stream(stream)))
 
 
 def project_keys(L, K, P, Kp, n_tokens: int, t_begin=None, seq_lens=None, stream=None):
@@ -260,6 +268,13 @@ def dense_decode(L, Q, K, V, seq_lens, window: int, sm_scale: float, O, lse=None
 def workspace_init(ws, stream=None):
     w, n = _ws(ws)
     _check("jssa_workspace_init", load().jssa_workspace_init(w, n, _stream(stream)))
+
+
+def arm_withheld_copy(ws, wait_limit_us: int, stream=None):
+    """Arm the one-shot test of the bounded waits in this workspace: the next selection
+    launch withholds one bulk copy in row (0, 0) and gives up waiting after wait_limit_us."""
+    w, n = _ws(ws)
+    _check("jssa_test_withhold_copy", load().jssa_test_withhold_copy(w, n, wait_limit_us, _stream(stream)))
 
 
 def read_device_status(ws, stream=None):

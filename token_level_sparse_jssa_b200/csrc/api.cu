@@ -88,9 +88,9 @@ jssa_status carve(const jssa_layout* L, int64_t k, int64_t window, void* base, W
   const int rows = L->B * L->Hkv;
   // partials for every split count a call with this (k, window) can use
   int S_cap = 1, S = 1, len = 0;
-  attn_split_policy(L->mode, true, rows, min64(k + window, L->T_cap), num_sms, L->d_k, &S, &len);
-  S_cap = S > S_cap ? S : S_cap;
-  if (L->mode != JSSA_MODE_MLA) {  // MLA has no dense path
+  if (L->mode != JSSA_MODE_MLA) {  // (the MLA kernel merges its splits inside a cluster: no partials)
+    attn_split_policy(L->mode, true, rows, min64(k + window, L->T_cap), num_sms, L->d_k, &S, &len);
+    S_cap = S > S_cap ? S : S_cap;
     attn_split_policy(L->mode, false, rows, L->T_cap, num_sms, L->d_k, &S, &len);
     S_cap = S > S_cap ? S : S_cap;
   }
@@ -136,6 +136,12 @@ jssa_status get_ws(const jssa_layout* L, int64_t k, int64_t window, void* ws, si
   if (st != JSSA_OK) return st;
   if (ws_bytes < w->bytes) return JSSA_ERR_WORKSPACE;
   return JSSA_OK;
+}
+
+// Arms the one-shot test of the bounded waits (words 1 and 2 after the status word).
+__global__ void arm_wait_test_kernel(int* status, int limit_us) {
+  status[2] = limit_us;
+  status[1] = 1;
 }
 
 jssa_status cu(cudaError_t e) {
@@ -236,7 +242,7 @@ jssa_status run_topk(const jssa_layout* L, const float* scores, int64_t sc_ld, c
 jssa_status run_attention(const jssa_layout* L, const void* Q, const void* K, const void* V, const int32_t* idx,
                           int idx_ld, const int32_t* n_sel, const int32_t* seq_lens, int window, float sm_scale,
                           void* O, float* lse, const Workspace& w, bool counters_zeroed, cudaStream_t s) {
-  if (!counters_zeroed) {
+  if (!counters_zeroed && L->mode != JSSA_MODE_MLA) {  // (the MLA kernel keeps no arrival counters)
     jssa_status st = cu(cudaMemsetAsync(w.counters, 0, sizeof(int) * L->B * L->Hkv, s));
     if (st != JSSA_OK) return st;
   }
@@ -261,6 +267,15 @@ jssa_status run_attention(const jssa_layout* L, const void* Q, const void* K, co
   const bool indexed = idx != nullptr;
   a.list_max = indexed ? static_cast<int64_t>(idx_ld) + window : (window > 0 ? window : L->T_cap);
   if (a.list_max > L->T_cap) a.list_max = L->T_cap;
+  if (L->mode == JSSA_MODE_MLA) {  // token groups merged inside a cluster per (sequence, head half)
+    a.S = mla_split_groups(L->B, num_sms_current());
+    a.split_len = static_cast<int>(ceil_div(a.list_max > 0 ? a.list_max : 1, a.S));
+    a.O = O;
+    a.lse = lse;
+    a.out_bf16 = (L->out_dtype == JSSA_OUT_BF16);
+    a.status = w.status;
+    return cu(launch_mla_split(a, !indexed, s));
+  }
   attn_split_policy(L->mode, indexed, L->B * L->Hkv, a.list_max, num_sms_current(), L->d_k, &a.S, &a.split_len);
   if (a.S > w.S_cap) return JSSA_ERR_WORKSPACE;
   a.part_o = w.part_o;
@@ -270,11 +285,6 @@ jssa_status run_attention(const jssa_layout* L, const void* Q, const void* K, co
   a.lse = lse;
   a.out_bf16 = (L->out_dtype == JSSA_OUT_BF16);
   a.status = w.status;
-  if (L->mode == JSSA_MODE_MLA) {
-    jssa_status st = cu(launch_mla_attention(a, s));
-    if (st != JSSA_OK) return st;
-    return cu(launch_merge(a, s));
-  }
   return cu(launch_attention(a, s));  // merges in its last CTA per row
 }
 
@@ -393,6 +403,31 @@ jssa_status jssa_project_keys(const jssa_layout* L, const void* K, const float* 
   if (!aligned(K, 16) || !aligned(Kp, 16) || !aligned(P, 16)) return JSSA_ERR_INVALID_ARG;
   ProjectArgs a = project_args(L, K, P, Kp, t_begin, seq_lens, n_tokens, nullptr);
   return cu(launch_project_keys(a, static_cast<cudaStream_t>(stream)));
+}
+
+jssa_status jssa_append_kv(const jssa_layout* L, const void* K_new, const void* V_new, void* K, void* V,
+                           const int32_t* t_pos, void* stream) {
+  jssa_status st = check_layout(L);
+  if (st != JSSA_OK) return st;
+  const bool mla = L->mode == JSSA_MODE_MLA;
+  if (!K_new || !K || !t_pos || (!mla && (!V_new || !V)) || (mla && V_new)) return JSSA_ERR_INVALID_ARG;
+  if (!aligned(K_new, 16) || !aligned(K, 16) || (V_new && (!aligned(V_new, 16) || !aligned(V, 16))) ||
+      !aligned(t_pos, 4))
+    return JSSA_ERR_INVALID_ARG;
+  AppendArgs a{};
+  a.K_new = K_new;
+  a.V_new = mla ? nullptr : V_new;
+  a.K = K;
+  memcpy(a.ks, L->k_stride, sizeof a.ks);
+  a.V = V;
+  memcpy(a.vs, L->v_stride, sizeof a.vs);
+  a.t_pos = t_pos;
+  a.B = L->B;
+  a.Hkv = L->Hkv;
+  a.dk = L->d_k;
+  a.dv = L->d_v;
+  a.T_cap = L->T_cap;
+  return cu(launch_append_rows(a, static_cast<cudaStream_t>(stream)));
 }
 
 jssa_status jssa_score(const jssa_layout* L, const void* Q, const float* P, const void* Kp, const int32_t* seq_lens,
@@ -653,7 +688,6 @@ jssa_status jssa_dense_decode(const jssa_layout* L, const void* Q, const void* K
                               void* workspace, size_t ws_bytes, void* stream) {
   jssa_status st = check_layout(L);
   if (st != JSSA_OK) return st;
-  if (L->mode == JSSA_MODE_MLA) return JSSA_ERR_UNSUPPORTED;
   if (!Q || !K || !V || !seq_lens || !O || window < 0) return JSSA_ERR_INVALID_ARG;
   if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 4)) return JSSA_ERR_INVALID_ARG;
   Workspace w{};
@@ -711,6 +745,13 @@ jssa_status jssa_calibrate(const jssa_layout* L, const void* Qc, const void* K, 
 jssa_status jssa_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
   if (!workspace || !aligned(workspace, kAlign) || ws_bytes < sizeof(int)) return JSSA_ERR_WORKSPACE;
   return cu(cudaMemsetAsync(workspace, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
+}
+
+jssa_status jssa_test_withhold_copy(void* workspace, size_t ws_bytes, int32_t wait_limit_us, void* stream) {
+  if (!workspace || !aligned(workspace, kAlign) || ws_bytes < 3 * sizeof(int)) return JSSA_ERR_WORKSPACE;
+  if (wait_limit_us < 1 || wait_limit_us > 1000000) return JSSA_ERR_INVALID_ARG;
+  arm_wait_test_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<int*>(workspace), wait_limit_us);
+  return cu(cudaGetLastError());
 }
 
 jssa_status jssa_read_device_status(void* workspace, size_t ws_bytes, int32_t* flags, void* stream) {

@@ -27,6 +27,31 @@ __device__ __forceinline__ void flag_error(int* status, int bit) {
   if (status) atomicOr(status, bit);
 }
 
+// Default limit of a bounded wait, and the one-shot test of the bounded waits that
+// jssa_test_withhold_copy() arms in the words after the status word: word 1 = 1 asks the
+// first CTA of row 0 of the next selection launch to withhold one bulk copy, word 2 is that
+// CTA's wait limit in microseconds.  The CTA disarms word 1 once it has read it.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+struct WaitTest {
+  bool withhold;
+  uint64_t limit_ns;
+};
+__device__ __forceinline__ WaitTest wait_test_read(const int* status, bool first_cta) {
+  WaitTest t{false, kWaitLimitNs};
+  if (status && first_cta) {
+    const volatile int* w = status;
+    if (w[1] == 1) {
+      t.withhold = true;
+      const int us = w[2];
+      t.limit_ns = static_cast<uint64_t>(us > 0 ? us : 1) * 1000ull;
+    }
+  }
+  return t;
+}
+__device__ __forceinline__ void wait_test_disarm(int* status) {
+  if (status) *reinterpret_cast<volatile int*>(status + 1) = 0;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -205,6 +230,19 @@ __device__ __forceinline__ int kp_vector_rotation(int tid) {
   if constexpr (VPT == 1) return 0;
   else if constexpr (VPT == 2) return (tid >> 2) & 1;
   else return (tid >> 1) & 3;
+}
+
+// Sum of a thread's per-vector partial dot products, read in the rotated order above
+// (a[j] belongs to vector (j + rot) % VPT).  The pairing (a0 + a2) + (a1 + a3) is the same
+// fp32 value for every rotation, because each of its additions is commutative; so two
+// tokens with identical projected rows get bit-identical scores whichever threads score
+// them, and an exact tie stays exact (the lower position then wins the selection).
+template <int VPT>
+__device__ __forceinline__ float kp_rotated_sum(const float (&a)[VPT]) {
+  static_assert(VPT == 1 || VPT == 2 || VPT == 4, "1, 2 or 4 vectors per thread");
+  if constexpr (VPT == 1) return a[0];
+  else if constexpr (VPT == 2) return a[0] + a[1];
+  else return (a[0] + a[2]) + (a[1] + a[3]);
 }
 
 // Dot product of one 16-byte vector of a projected-key row with the matching slice of the

@@ -23,6 +23,20 @@ struct ProjectArgs {
 };
 cudaError_t launch_project_keys(const ProjectArgs& a, cudaStream_t s);
 
+// Append on write: the newest K (and V) row of every (sequence, KV head) into row t_pos[b].
+struct AppendArgs {
+  const void* K_new;   // [B, Hkv, dk] contiguous
+  const void* V_new;   // [B, Hkv, dv] contiguous, nullable
+  void* K;
+  int64_t ks[3];
+  void* V;
+  int64_t vs[3];
+  const int32_t* t_pos;
+  int B, Hkv, dk, dv;
+  int64_t T_cap;
+};
+cudaError_t launch_append_rows(const AppendArgs& a, cudaStream_t s);
+
 // Per-step prologue: projected group queries qs, plus the projection of the newest
 // n_new (<= 16) rows of each sequence into Kp.
 struct PrologueArgs {
@@ -197,6 +211,10 @@ cudaError_t launch_vote_broadcast(const VoteArgs& a, cudaStream_t s);
 void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int num_sms, int d, int* S, int* split_len);
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);   // GQA path
 cudaError_t launch_mla_attention(const AttnArgs& a, cudaStream_t s);  // MLA path (indexed only)
+// MLA attention, indexed or dense, many tiles per CTA with the split merge in a cluster of S
+// CTAs per (sequence, head half); S from mla_split_groups, split_len = tokens per CTA.
+int mla_split_groups(int B, int num_sms);
+cudaError_t launch_mla_split(const AttnArgs& a, bool dense, cudaStream_t s);
 int mla_max_split();  // tokens per CTA of the MLA kernel
 cudaError_t launch_merge(const AttnArgs& a, cudaStream_t s);
 

@@ -108,6 +108,33 @@ cudaError_t launch_project_keys(const ProjectArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ append on write
+// One CTA per (sequence, KV head): the newest key (and value) row, 16 bytes per thread,
+// from the contiguous [B, Hkv, d] input into row t_pos[b] of the strided caches.
+constexpr int kAppendThreads = 64;
+
+__global__ void __launch_bounds__(kAppendThreads) append_rows_kernel(AppendArgs a) {
+  const int row = blockIdx.x;
+  const int b = row / a.Hkv, h = row % a.Hkv;
+  const int64_t t = a.t_pos[b];
+  if (t < 0 || t >= a.T_cap) return;
+  const uint4* ks = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.K_new) +
+                                                   static_cast<int64_t>(row) * a.dk);
+  uint4* kd = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.K) + b * a.ks[0] + h * a.ks[1] + t * a.ks[2]);
+  for (int i = threadIdx.x; i < a.dk / 8; i += kAppendThreads) kd[i] = __ldg(ks + i);
+  if (a.V_new) {
+    const uint4* vs = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.V_new) +
+                                                     static_cast<int64_t>(row) * a.dv);
+    uint4* vd = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.V) + b * a.vs[0] + h * a.vs[1] + t * a.vs[2]);
+    for (int i = threadIdx.x; i < a.dv / 8; i += kAppendThreads) vd[i] = __ldg(vs + i);
+  }
+}
+
+cudaError_t launch_append_rows(const AppendArgs& a, cudaStream_t s) {
+  append_rows_kernel<<<a.B * a.Hkv, kAppendThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ step prologue
 constexpr int kPrologueThreads = 256;
 constexpr int kMaxNewRowsInPrologue = 16;

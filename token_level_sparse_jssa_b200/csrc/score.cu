@@ -206,9 +206,7 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a) {
             const uint4 raw = *reinterpret_cast<const uint4*>(trow + (sub * VPT + (j + rot) % VPT) * 16);
             acc[j] = kp_vector_dot<F8>(q[j], raw);
           }
-          float sc = acc[0];
-#pragma unroll
-          for (int j = 1; j < VPT; ++j) sc += acc[j];
+          float sc = kp_rotated_sum<VPT>(acc);
           if (TPT == 2) sc += __shfl_xor_sync(0xFFFFFFFFu, sc, 1);
           if (sub == 0 && tok < cnt) {
             out[tok] = sc;

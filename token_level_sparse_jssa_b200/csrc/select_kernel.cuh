@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
   __shared__ __align__(8) uint64_t full[8], empty[8];
   __shared__ float qs[kSelMaxR];
   __shared__ uint32_t dig, krem_s, gcnt, gbase;
-  __shared__ uint32_t cta_gt[kSelMaxCluster], cta_eq[kSelMaxCluster];
+  __shared__ uint32_t cta_gt[kSelMaxCluster], cta_eq[kSelMaxCluster], cta_ab[kSelMaxCluster];
   __shared__ uint32_t warp_gt[kSelWarps], warp_eq[kSelWarps], warp_nc[kSelWarps];
   __shared__ uint32_t scan_tmp[32];
   __shared__ int aborted_s;
@@ -203,6 +203,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
   const int n_new = static_cast<int>(min64(max64(a.n_new, 0), T));
   const int64_t t_new0 = T - n_new;  // newest rows [t_new0, T) are projected here
   int32_t* out = a.idx + static_cast<int64_t>(row) * a.k;
+  const WaitTest wt = wait_test_read(a.status, row == 0 && crank == 0);
 
   if (tid == 0) {
     gcnt = 0;
@@ -221,6 +222,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
   }
   for (int j = k_eff + crank * kSelThreads + tid; j < a.k; j += C * kSelThreads) out[j] = -1;
   __syncthreads();
+  if (wt.withhold && tid == 0) wait_test_disarm(a.status);  // every thread has read it
 
   // ---- the producer warp streams the slice's Kp rows.  The consumers form this CTA's share
   // of the projections (dims [dlo, dlo + dn): the d / 8 chunks of 8 dims split over the
@@ -238,6 +240,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
           atomicExch(&aborted_s, 1);
           break;
         }
+        if (wt.withhold && c == 0) continue;  // the armed test: this stage's copy never comes
         const int t0 = lo + c * CH;
         const uint32_t cnt = static_cast<uint32_t>(min(CH, lo + len - t0));
         mbar_arrive_expect_tx(&full[s], cnt * R * EB);
@@ -348,7 +351,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
       bool dead = false;
       for (int c = 0; c < nch; ++c) {
         const int s = c % S;
-        if (!dead && !mbar_wait_bounded(&full[s], static_cast<uint32_t>((c / S) & 1), a.status)) {
+        if (!dead && !mbar_wait_bounded(&full[s], static_cast<uint32_t>((c / S) & 1), a.status, wt.limit_ns)) {
           dead = true;
           atomicExch(&aborted_s, 1);
         }
@@ -368,9 +371,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
               const uint4 raw = *reinterpret_cast<const uint4*>(trow + (sub * VPT + (jj + rot) % VPT) * 16);
               accv[jj] = kp_vector_dot<F8>(q[jj], raw);
             }
-            float sc = accv[0];
-#pragma unroll
-            for (int jj = 1; jj < VPT; ++jj) sc += accv[jj];
+            float sc = kp_rotated_sum<VPT>(accv);
             if (TPT == 2) sc += __shfl_xor_sync(0xFFFFFFFFu, sc, 1);
             if (sub == 0 && tok < cnt) {
               const uint32_t key = float_to_ordered(sc);
@@ -399,7 +400,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
     const bool aborted = aborted_s != 0;
     if (aborted && tid == kSelConsumers) {  // let every copy still in flight land before the CTA moves on
       for (int s = 0; s < S; ++s)
-        for (int par = 0; par < 2; ++par) mbar_wait_bounded(&full[s], par, nullptr, 50000000ull);
+        for (int par = 0; par < 2; ++par)
+          mbar_wait_bounded(&full[s], par, nullptr, wt.limit_ns < 50000000ull ? wt.limit_ns : 50000000ull);
     }
     __syncthreads();
 
@@ -604,10 +606,14 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelectArgs a) {
       for (int w = 0; w < kSelWarps; ++w) { g += warp_gt[w]; e += warp_eq[w]; }
       *cluster.map_shared_rank(&cta_gt[crank], tid) = g;
       *cluster.map_shared_rank(&cta_eq[crank], tid) = e;
+      *cluster.map_shared_rank(&cta_ab[crank], tid) = aborted ? 1u : 0u;
     }
     cluster.sync();  // the counts are everywhere; other CTAs' memory is no longer read
-    if (aborted) {   // a wait gave up (flagged): report an empty selection
+    bool any_aborted = false;
+    for (int c = 0; c < C; ++c) any_aborted |= (cta_ab[c] != 0u);
+    if (any_aborted) {  // a wait gave up in some CTA of the row (flagged): the row's selection is empty
       for (int j = crank * kSelThreads + tid; j < k_eff; j += C * kSelThreads) out[j] = -1;
+      if (crank == 0 && tid == 0) a.n_sel[row] = 0;
       if constexpr (D > 0) for (int j = tid; j < L; j += kSelThreads) tok_list[j] = -1;
     } else {
 

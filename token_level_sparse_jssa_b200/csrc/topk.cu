@@ -128,13 +128,14 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   uint32_t* masks = hloc;                                               // output bitmaps alias hloc
   __shared__ uint64_t bar;
   __shared__ uint32_t dig, krem_s, gcnt, gbase;
-  __shared__ uint32_t cta_gt[kMaxCluster], cta_eq[kMaxCluster];
+  __shared__ uint32_t cta_gt[kMaxCluster], cta_eq[kMaxCluster], cta_ab[kMaxCluster];
   __shared__ uint32_t warp_gt[kTopkWarps], warp_eq[kTopkWarps], warp_nc[kTopkWarps];
   __shared__ uint32_t scan_tmp[32];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.y;
   const int b = row / a.Hkv;
+  const WaitTest wt = wait_test_read(a.status, row == 0 && crank == 0);
   if (tid == 0) {
     gcnt = 0;
     mbar_init(&bar, 1);
@@ -169,7 +170,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
   __syncthreads();
   const bool bulk = STAGED && (reinterpret_cast<uintptr_t>(srow) & 15u) == 0;
   const int nbulk = bulk ? (len & ~3) : 0;
-  if (tid == 0) {  // the slice (when staged) and the row's digit-1 histogram, in one transaction
+  if (wt.withhold && tid == 0) wait_test_disarm(a.status);  // every thread has read it
+  if (tid == 0 && !wt.withhold) {  // the slice (when staged) and the row's digit-1 histogram, in one transaction
     const uint64_t pol = l2_policy_evict_first();
     mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nbulk) * 4u + kBins1 * 4u);
     if (nbulk > 0) bulk_g2s(fs, srow, static_cast<uint32_t>(nbulk) * 4u, &bar, pol);
@@ -179,7 +181,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     for (int i = nbulk + tid; i < len; i += kTopkThreads) fs[i] = __ldg(srow + i);
   auto key_at = [&](int i) -> uint32_t { return float_to_ordered(STAGED ? fs[i] : __ldg(srow + i)); };
   cluster.sync();  // S0: every CTA runs and rank 0's gather count is zero (overlaps the copies)
-  const bool staged_ok = mbar_wait_bounded(&bar, 0, a.status);
+  const bool staged_ok = mbar_wait_bounded(&bar, 0, a.status, wt.limit_ns);
   const bool aborted = __syncthreads_or(!staged_ok);
 
   // digit 1 from the row's histogram (every CTA computes the same digit)
@@ -333,10 +335,15 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a, int per_
     for (int w = 0; w < kTopkWarps; ++w) { g += warp_gt[w]; e += warp_eq[w]; }
     *cluster.map_shared_rank(&cta_gt[crank], tid) = g;
     *cluster.map_shared_rank(&cta_eq[crank], tid) = e;
+    *cluster.map_shared_rank(&cta_ab[crank], tid) = aborted ? 1u : 0u;
   }
   cluster.sync();  // S2: last access to another CTA's shared memory
-  if (aborted) {  // the staging copy never completed (flagged): report an empty selection
+  bool any_aborted = false;
+  for (int c = 0; c < C; ++c) any_aborted |= (cta_ab[c] != 0u);
+  if (any_aborted) {  // a staging copy of the row never completed (flagged): the selection is empty
     for (int j = crank * kTopkThreads + tid; j < k_eff; j += C * kTopkThreads) out[j] = -1;
+    if (crank == 0 && tid == 0) a.n_sel[row] = 0;
+    if (aborted && tid == 0) mbar_wait_bounded(&bar, 0, nullptr, wt.limit_ns);  // a late copy lands before exit
     return;
   }
   // output base and quota of keys == kstar: of this CTA, then of this warp
