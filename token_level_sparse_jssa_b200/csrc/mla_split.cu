@@ -66,6 +66,9 @@ __device__ __forceinline__ void sp_wait_groups(int kb) {
   }
 }
 
+__device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
 // Bring `bytes` (a multiple of 16, from a 16-byte aligned address) into L2.
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
@@ -74,13 +77,15 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) 
 template <bool DENSE>
 __global__ void __launch_bounds__(kSpThreads, 1) mla_split_kernel(AttnArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  __shared__ int32_t tok_s[kSpTile];
+  __shared__ int32_t tok_s[2][kSpTile];               // cache rows of this tile and the next
   __shared__ __align__(8) uint64_t bars[kSpKB + 1];  // [kb]: score MMAs through block kb; [9]: value MMAs
   __shared__ uint32_t tmem_base_s;
   __shared__ float m_s[kSpHeads];                     // running maximum per head (log2 units)
   __shared__ float alpha_s[kSpHeads];
   __shared__ float red_s[4][kSpHeads];                // per TMEM lane quadrant: tile maxima, then sums
-  __shared__ float lse_s[kSpHeads], invl_s[kSpHeads];
+  __shared__ __align__(16) float invl_s[kSpHeads];
+  __shared__ float lse_all[kSpMaxCluster][kSpHeads];  // every CTA's lse, pushed before the merge
+  __shared__ float w_s[kSpMaxCluster][kSpHeads];      // merge weight of each partial per head
 
   cg::cluster_group cluster = cg::this_cluster();
   const int G = static_cast<int>(cluster.num_blocks());
@@ -131,6 +136,7 @@ __global__ void __launch_bounds__(kSpThreads, 1) mla_split_kernel(AttnArgs a) {
   }
   if (tid < kSpHeads) m_s[tid] = -INFINITY;
   if (warp == 0) tmem_alloc(&tmem_base_s, kSpTmemCols);
+  cluster_arrive_relaxed();  // matched by the wait before the first access to a peer's shared memory
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -159,20 +165,18 @@ __global__ void __launch_bounds__(kSpThreads, 1) mla_split_kernel(AttnArgs a) {
   int last_commit = -1;
   uint32_t par = 0;  // phase parity of the per-tile barriers
 
+  // cache row of list position pos of this CTA's range (-1 past it)
+  auto row_at = [&](int64_t pos) -> int32_t {
+    return (pos < my_lo + my_len) ? static_cast<int32_t>(token_at(pos)) : -1;
+  };
+  if (ntiles > 0 && tid < kSpTile) tok_s[0][tid] = row_at(my_lo + tid);
+
   for (int tile = 0; tile < ntiles && !dead; ++tile, par ^= 1u) {
     const int64_t pos0 = my_lo + static_cast<int64_t>(tile) * kSpTile;
     const int tlen = static_cast<int>(min64(kSpTile, my_lo + my_len - pos0));
-    if (tid < kSpTile) {
-      tok_s[tid] = (tid < tlen) ? static_cast<int32_t>(token_at(pos0 + tid)) : -1;
-      // the next tile's rows, into L2 while this one runs
-      if (tile + 1 < ntiles) {
-        const int64_t p2 = pos0 + kSpTile + tid;
-        if (p2 < my_lo + my_len) {
-          const int64_t t2 = token_at(p2);
-          if (t2 >= 0) prefetch_l2_bulk(Cb + t2 * a.ks[2], kSpDk * 2);
-        }
-      }
-    }
+    const int32_t* tok = tok_s[tile & 1];
+    // this thread's row of the next tile: loaded now, stored once this tile's copies are issued
+    const int32_t next_row = (tid < kSpTile && tile + 1 < ntiles) ? row_at(pos0 + kSpTile + tid) : -1;
     __syncthreads();
     const int N = (tlen + 15) & ~15;  // K extent of the value MMA
 
@@ -181,7 +185,7 @@ __global__ void __launch_bounds__(kSpThreads, 1) mla_split_kernel(AttnArgs a) {
     uint32_t bytes_c[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int32_t t = tok_s[r0 + 32 * u];
+      const int32_t t = tok[r0 + 32 * u];
       src_c[u] = (t >= 0) ? Cb + static_cast<int64_t>(t) * a.ks[2] + ch * 8 : Cb;
       bytes_c[u] = (t >= 0) ? 16u : 0u;  // masked rows are zero-filled
     }
@@ -200,6 +204,11 @@ __global__ void __launch_bounds__(kSpThreads, 1) mla_split_kernel(AttnArgs a) {
         }
       }
       cp_async_commit();
+    }
+    // the next tile's rows: into tok_s (the other buffer, free since the previous tile) and L2
+    if (tid < kSpTile && tile + 1 < ntiles) {
+      tok_s[(tile + 1) & 1][tid] = next_row;
+      if (next_row >= 0) prefetch_l2_bulk(Cb + static_cast<int64_t>(next_row) * a.ks[2], kSpDk * 2);
     }
 
     // ---- S^T over the 9 K-blocks, the query ring refilled behind it
@@ -241,7 +250,7 @@ __global__ void __launch_bounds__(kSpThreads, 1) mla_split_kernel(AttnArgs a) {
     // ---- softmax of this thread's token over its 32 heads
     float x[32];
     tmem_ld32(trow + hw * 32, x);
-    const bool valid = t_lane < tlen && tok_s[t_lane] >= 0;
+    const bool valid = t_lane < tlen && tok[t_lane] >= 0;
     bool big = false;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
@@ -339,23 +348,31 @@ __global__ void __launch_bounds__(kSpThreads, 1) mla_split_kernel(AttnArgs a) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  cluster_wait();  // every CTA of the cluster has started
   if (tid < kSpHeads) {
     const float L = red_s[0][tid] + red_s[1][tid] + red_s[2][tid] + red_s[3][tid];
     const float m = m_s[tid];
     const bool ok = !dead && ntiles > 0 && L > 0.f && m != -INFINITY;
-    lse_s[tid] = ok ? (m + log2f(L)) * 0.6931471805599453f : -INFINITY;
+    const float lse = ok ? (m + log2f(L)) * 0.6931471805599453f : -INFINITY;
     invl_s[tid] = ok ? 1.f / L : 0.f;
+    for (int q = 0; q < G; ++q) cluster.map_shared_rank(&lse_all[0][0], q)[g * kSpHeads + tid] = lse;
   }
   __syncthreads();
   // normalised partial o[head][dim] into shared memory (the latent tile is free)
   if (!dead && ntiles > 0) {
+    float il[32];
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+      const float4 v4 = *reinterpret_cast<const float4*>(&invl_s[hw * 32 + i]);
+      il[i] = v4.x, il[i + 1] = v4.y, il[i + 2] = v4.z, il[i + 3] = v4.w;
+    }
 #pragma unroll 1
     for (int j = 0; j < 4; ++j) {
       float v[32];
       tmem_ld32(trow + kSpOCol + 64 * j + hw * 32, v);
       const int d = 128 * j + quad * 32 + lane;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) ob[(hw * 32 + i) * kSpDv + d] = v[i] * invl_s[hw * 32 + i];
+      for (int i = 0; i < 32; ++i) ob[(hw * 32 + i) * kSpDv + d] = v[i] * il[i];
     }
   } else {
     for (int i = tid; i < kSpHeads * kSpDv; i += kSpThreads) ob[i] = 0.f;
@@ -367,33 +384,80 @@ __global__ void __launch_bounds__(kSpThreads, 1) mla_split_kernel(AttnArgs a) {
     tmem_dealloc(tmem, kSpTmemCols);
   }
 
-  // ---- merge the G partials of the cluster: CTA g writes its share of the 64 x 512 outputs
+  // ---- merge the G partials of the cluster: CTA g writes its share of the 64 x 512 outputs.
+  // The weight of partial q for head h is exp(lse_q - M) / sum_q' exp(lse_q' - M), computed
+  // once per head from the lse values every CTA pushed; the partial rows are then read over
+  // distributed shared memory 16 bytes at a time, a batch of loads in flight before the first
+  // is used.
   cluster.sync();
-  const int per = (kSpHeads * kSpDv + G - 1) / G;
-  const int e_lo = g * per, e_hi = min(kSpHeads * kSpDv, e_lo + per);
-  for (int e = e_lo + tid; e < e_hi; e += kSpThreads) {
-    const int h = e / kSpDv, d = e % kSpDv;
-    float l[kSpMaxCluster], v[kSpMaxCluster];
+  if (tid < kSpHeads) {
+    float l[kSpMaxCluster];
 #pragma unroll
-    for (int q = 0; q < kSpMaxCluster; ++q) {  // all remote loads in flight before the first use
-      l[q] = (q < G) ? cluster.map_shared_rank(lse_s, q)[h] : -INFINITY;
-      v[q] = (q < G) ? cluster.map_shared_rank(ob, q)[e] : 0.f;
-    }
+    for (int q = 0; q < kSpMaxCluster; ++q) l[q] = (q < G) ? lse_all[q][tid] : -INFINITY;
     float M = -INFINITY;
 #pragma unroll
     for (int q = 0; q < kSpMaxCluster; ++q) M = fmaxf(M, l[q]);
-    float L = 0.f, o = 0.f;
+    float L = 0.f;
 #pragma unroll
     for (int q = 0; q < kSpMaxCluster; ++q) {
-      const float w = (M == -INFINITY || q >= G) ? 0.f : expf(l[q] - M);
-      L += w;
-      o = fmaf(w, v[q], o);
+      l[q] = (M == -INFINITY) ? 0.f : expf(l[q] - M);
+      L += l[q];
     }
-    o = (L > 0.f) ? o / L : 0.f;
-    const int64_t qi = qrow0 + h;
-    if (a.lse && d == 0) a.lse[qi] = (M == -INFINITY) ? -INFINITY : M + logf(L);
-    if (a.out_bf16) static_cast<__nv_bfloat16*>(a.O)[qi * kSpDv + d] = __float2bfloat16_rn(o);
-    else static_cast<float*>(a.O)[qi * kSpDv + d] = o;
+#pragma unroll
+    for (int q = 0; q < kSpMaxCluster; ++q) w_s[q][tid] = (L > 0.f) ? l[q] / L : 0.f;
+    if (a.lse && g == 0) a.lse[qrow0 + tid] = (M == -INFINITY) ? -INFINITY : M + logf(L);
+  }
+  __syncthreads();
+  constexpr int kVec = kSpHeads * kSpDv / 4;  // float4 elements of the output block
+  const int per4 = (kVec + G - 1) / G;
+  const int v_lo = g * per4, v_hi = min(kVec, v_lo + per4);
+  const float4* obq[kSpMaxCluster];
+#pragma unroll
+  for (int q = 0; q < kSpMaxCluster; ++q)
+    obq[q] = reinterpret_cast<const float4*>(cluster.map_shared_rank(ob, q < G ? q : 0));
+  constexpr int kBatch = 2;
+  const bool o_vec = (reinterpret_cast<uintptr_t>(a.O) & 15u) == 0;  // 16-byte stores (8 for bf16)
+  for (int v0 = v_lo + tid; v0 < v_hi; v0 += kBatch * kSpThreads) {
+    float4 x[kBatch][kSpMaxCluster];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int v = v0 + u * kSpThreads;
+#pragma unroll
+      for (int q = 0; q < kSpMaxCluster; ++q)
+        x[u][q] = (q < G && v < v_hi) ? obq[q][v] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int v = v0 + u * kSpThreads;
+      if (v >= v_hi) break;
+      const int h = (v * 4) / kSpDv, d = (v * 4) % kSpDv;
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < kSpMaxCluster; ++q) {
+        const float wq = (q < G) ? w_s[q][h] : 0.f;
+        o.x = fmaf(wq, x[u][q].x, o.x);
+        o.y = fmaf(wq, x[u][q].y, o.y);
+        o.z = fmaf(wq, x[u][q].z, o.z);
+        o.w = fmaf(wq, x[u][q].w, o.w);
+      }
+      const int64_t off = (qrow0 + h) * kSpDv + d;
+      if (a.out_bf16) {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.O) + off;
+        if (o_vec) {
+          uint2 pk;
+          pk.x = pack_bf16x2(o.x, o.y);
+          pk.y = pack_bf16x2(o.z, o.w);
+          *reinterpret_cast<uint2*>(dst) = pk;
+        } else {
+          dst[0] = __float2bfloat16_rn(o.x), dst[1] = __float2bfloat16_rn(o.y);
+          dst[2] = __float2bfloat16_rn(o.z), dst[3] = __float2bfloat16_rn(o.w);
+        }
+      } else {
+        float* dst = static_cast<float*>(a.O) + off;
+        if (o_vec) *reinterpret_cast<float4*>(dst) = o;
+        else dst[0] = o.x, dst[1] = o.y, dst[2] = o.z, dst[3] = o.w;
+      }
+    }
   }
   cluster.sync();  // the partials stay until every CTA has read them
 }
