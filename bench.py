@@ -307,7 +307,8 @@ def stage_times(st, Q, reps=50):
     cluster); attention = indexed attention with its merge; dense = the full-KV comparator;
     gather_then_attend = the same attention done the gather-based way (copy, then dense);
     step_other_kp = the whole step over the other scoring-cache type (E4M3 when the run is bf16);
-    vote_select = the head-shared soft-voting selection."""
+    vote_select = the head-shared soft-voting selection; local_layers = a hybrid model's local
+    layers of one step."""
     jssa, w = st.jssa, st.w
     calls = {
         "select_us": lambda: jssa.select(st.L, Q, st.K, st.Kp, st.P, st.seq_lens, 1, w.k, w.window, st.idx,
@@ -319,6 +320,8 @@ def stage_times(st, Q, reps=50):
                                                    w.sm_scale, st.idx, st.nsel, st.ws),
     }
     calls["dense_us"] = lambda: st.dense(Q)
+    if st.local:  # a hybrid model's local layers (dense over their own window caches, together > L2)
+        calls["local_layers_us"] = lambda: st.local_layers(Q)
     if st.w.mode != "mla":  # (the gather-based comparator is GQA only)
         # the gather-based baseline of the pages: copy the attended rows, then dense decode on them
         calls["gather_then_attend_us"] = lambda: jssa.gather_decode(st.L, Q, st.K, st.V, st.idx, w.k, st.nsel,

@@ -89,13 +89,13 @@ jssa_status carve(const jssa_layout* L, int64_t k, int64_t window, void* base, W
   // partials for every split count a call with this (k, window) can use
   int S_cap = 1, S = 1, len = 0;
   if (L->mode != JSSA_MODE_MLA) {  // (the MLA kernel merges its splits inside a cluster: no partials)
-    attn_split_policy(L->mode, true, rows, min64(k + window, L->T_cap), num_sms, L->d_k, &S, &len);
+    attn_split_policy(true, rows, min64(k + window, L->T_cap), num_sms, L->d_k, &S, &len);
     S_cap = S > S_cap ? S : S_cap;
-    attn_split_policy(L->mode, false, rows, L->T_cap, num_sms, L->d_k, &S, &len);
+    attn_split_policy(false, rows, L->T_cap, num_sms, L->d_k, &S, &len);
     S_cap = S > S_cap ? S : S_cap;
   }
   if (window > 0 && L->mode != JSSA_MODE_MLA) {
-    attn_split_policy(L->mode, false, rows, min64(window, L->T_cap), num_sms, L->d_k, &S, &len);
+    attn_split_policy(false, rows, min64(window, L->T_cap), num_sms, L->d_k, &S, &len);
     S_cap = S > S_cap ? S : S_cap;
   }
   size_t off = 0;
@@ -276,7 +276,7 @@ jssa_status run_attention(const jssa_layout* L, const void* Q, const void* K, co
     a.status = w.status;
     return cu(launch_mla_split(a, !indexed, s));
   }
-  attn_split_policy(L->mode, indexed, L->B * L->Hkv, a.list_max, num_sms_current(), L->d_k, &a.S, &a.split_len);
+  attn_split_policy(indexed, L->B * L->Hkv, a.list_max, num_sms_current(), L->d_k, &a.S, &a.split_len);
   if (a.S > w.S_cap) return JSSA_ERR_WORKSPACE;
   a.part_o = w.part_o;
   a.part_lse = w.part_lse;
@@ -678,7 +678,7 @@ jssa_status jssa_gather_decode(const jssa_layout* L, const void* Q, const void* 
   const int64_t pst[3] = {Lmax * L->r, Lmax * L->r, L->r};
   memcpy(Lg.kp_stride, pst, sizeof pst);
   int S = 0, len = 0;
-  attn_split_policy(Lg.mode, false, Lg.B * Lg.Hkv, Lmax, num_sms_current(), Lg.d_k, &S, &len);
+  attn_split_policy(false, Lg.B * Lg.Hkv, Lmax, num_sms_current(), Lg.d_k, &S, &len);
   if (S > w.S_cap) return JSSA_ERR_WORKSPACE;
   return run_attention(&Lg, Q, gb, gb + off_v, nullptr, 0, nullptr, g.glen, 0, sm_scale, O, lse, w, false, s);
 }

@@ -19,7 +19,9 @@
 //                                                        even and odd K-steps in two chains)
 //   online softmax per head in fp32 (exp2 domain)
 //   O^T[d x 8 heads]     += V_sub^T . P^T               (P split into bf16 hi + lo parts,
-//                                                        so the weights keep ~16 bits)
+//                                                        so the weights keep ~16 bits; with at
+//                                                        most 4 heads both parts share one MMA,
+//                                                        the lo parts in columns 4-7)
 // The 4 groups' states are merged in shared memory into one normalised partial (o, lse)
 // per query head.  Indexed attention runs the S <= 8 splits of a row as one thread-block
 // cluster and combines the partials by log-sum-exp through distributed shared memory;
@@ -129,91 +131,11 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS) attn_kernel(AttnArgs a) {
                              smem_raw);
 }
 
-// ------------------------------------------------------------------ LSE merge
-// O = sum_s w_s o_s with w_s = exp(lse_s - M) / sum_s' exp(lse_s' - M), M = max lse; lse =
-// M + log(sum exp(lse_s - M)).  One CTA per (sequence, query head), one thread per 4 output
-// dims (16-byte loads); warp 0 forms the split weights, then every thread issues the loads
-// of 8 splits at a time before using them.
-constexpr int kMergeBatch = 8;
-__global__ void __launch_bounds__(256) merge_kernel(AttnArgs a) {
-  extern __shared__ float wsh[];  // [S]
-  __shared__ float sh_L;
-  const int64_t q = blockIdx.x;   // b * Hq + hq
-  const int S = a.S, D = a.dv;
-  const float* lse_s = a.part_lse + q * S;
-  if (threadIdx.x < 32) {
-    float M = -INFINITY;
-    for (int s = threadIdx.x; s < S; s += 32) M = fmaxf(M, lse_s[s]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, off));
-    float L = 0.f;
-    for (int s = threadIdx.x; s < S; s += 32) {
-      const float w = (M == -INFINITY) ? 0.f : expf(lse_s[s] - M);
-      wsh[s] = w;
-      L += w;
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, off);
-    if (threadIdx.x == 0) {
-      sh_L = L;
-      if (a.lse) a.lse[q] = (M == -INFINITY) ? -INFINITY : M + logf(L);
-    }
-  }
-  __syncthreads();
-  const float inv = (sh_L > 0.f) ? 1.f / sh_L : 0.f;
-  const int d4 = threadIdx.x;
-  if (4 * d4 >= D) return;
-  const float4* po = reinterpret_cast<const float4*>(a.part_o + q * S * D) + d4;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < S; s0 += kMergeBatch) {
-    float4 v[kMergeBatch];
-#pragma unroll
-    for (int u = 0; u < kMergeBatch; ++u)
-      v[u] = (s0 + u < S) ? __ldcs(po + static_cast<int64_t>(s0 + u) * (D / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int u = 0; u < kMergeBatch; ++u) {
-      const float w = (s0 + u < S) ? wsh[s0 + u] : 0.f;
-      acc.x = fmaf(w, v[u].x, acc.x);
-      acc.y = fmaf(w, v[u].y, acc.y);
-      acc.z = fmaf(w, v[u].z, acc.z);
-      acc.w = fmaf(w, v[u].w, acc.w);
-    }
-  }
-  acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
-  if (a.out_bf16) {
-    __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.O) + q * D) + 2 * d4;
-    o[0] = __floats2bfloat162_rn(acc.x, acc.y);
-    o[1] = __floats2bfloat162_rn(acc.z, acc.w);
-  } else if ((reinterpret_cast<uintptr_t>(a.O) & 15u) == 0) {
-    reinterpret_cast<float4*>(static_cast<float*>(a.O) + q * D)[d4] = acc;
-  } else {  // the API only guarantees 4-byte alignment of O
-    float* o = static_cast<float*>(a.O) + q * D + 4 * d4;
-    o[0] = acc.x; o[1] = acc.y; o[2] = acc.z; o[3] = acc.w;
-  }
-}
-
 // ------------------------------------------------------------------ host side
-void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int num_sms, int d, int* S_out,
+void attn_split_policy(bool indexed, int rows, int64_t list_max, int num_sms, int d, int* S_out,
                        int* split_out) {
   // Choose the split length (a multiple of the 16-token subtile, at least 64 tokens) that
   // keeps the last wave of CTAs fullest; fewer splits win ties.
-  if (mode == 1) {
-    // MLA (tensor-core kernel): one tile of at most 128 tokens per CTA and one CTA per SM.
-    // Every CTA also streams the 147 KB query block and writes a 256 KB partial, about as
-    // much as a full tile's token work, so the cost is waves x (1 + len / 128).
-    if (list_max <= 0) { *S_out = 1; *split_out = mla_max_split(); return; }
-    int best_len = mla_max_split();
-    double best_cost = 1e300;
-    for (int len = mla_max_split(); len >= 16; len -= 16) {
-      const int64_t S = ceil_div(list_max, len);
-      const int64_t waves = ceil_div(static_cast<int64_t>(rows) * S, num_sms);
-      const double cost = static_cast<double>(waves) * (1.0 + len / 128.0);
-      if (cost < best_cost - 1e-9) { best_cost = cost; best_len = len; }
-    }
-    *split_out = best_len;
-    *S_out = static_cast<int>(ceil_div(list_max, best_len));
-    return;
-  }
   const int min_split = 64;
   if (list_max <= 0) { *S_out = 1; *split_out = min_split; return; }
   if (d >= 256) {
@@ -290,10 +212,5 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s) {
   }
 }
 
-cudaError_t launch_merge(const AttnArgs& a, cudaStream_t s) {
-  if (a.dv % 4 != 0 || a.dv / 4 > 256) return cudaErrorInvalidValue;
-  merge_kernel<<<a.B * a.Hq, ((a.dv / 4 + 31) / 32) * 32, a.S * sizeof(float), s>>>(a);
-  return cudaGetLastError();
-}
 
 }  // namespace jssa

@@ -219,6 +219,7 @@ __device__ __forceinline__ void attn_core(const AttnArgs& a, int row, int split,
   float* pbuf = reinterpret_cast<float*>(smem_raw + Cfg::COMBINE_BYTES);   // [16][D] (cluster merge)
   float* plse = pbuf + 16 * D;                                              // [16]
   const float scale_log2 = a.sm_scale * kLog2e;
+  const bool pack = NTILE == 1 && G <= 4;  // hi and lo parts of P in one value MMA
   float m_run[NTILE][2], l_run[NTILE][2];
   float acc[KSTEPS][NTILE][4];
 #pragma unroll
@@ -315,6 +316,10 @@ __device__ __forceinline__ void attn_core(const AttnArgs& a, int row, int split,
         for (int e = 0; e < 4; ++e) sacc[nt][e] += theirs[nt * 4 + e];
     }
     // ---- online softmax over the 16 tokens of this subtile
+    // (with at most 4 heads, the hi and lo parts of P share one MMA: B columns 0-3 carry the
+    // hi parts of heads 0-3 and columns 4-7 the lo parts, which the lanes holding columns 4-7
+    // take from the lanes two to their left; those lanes' accumulators then follow the
+    // rescaling of the head whose lo part they hold)
     const bool v0 = token_at(sub * kSub + g) >= 0;
     const bool v1 = token_at(sub * kSub + g + 8) >= 0;
     uint32_t bhi[NTILE][2], blo[NTILE][2];
@@ -339,10 +344,12 @@ __device__ __forceinline__ void attn_core(const AttnArgs& a, int row, int split,
         p[2 + e] = exp2f(x[2 + e] - m_use);
         l_run[nt][e] = l_run[nt][e] * alpha + p[e] + p[2 + e];
         m_run[nt][e] = m_new;
+        const float alpha_lo = __shfl_xor_sync(0xFFFFFFFFu, alpha, 2);
+        const float alpha_acc = (pack && c >= 2) ? alpha_lo : alpha;
 #pragma unroll
         for (int mt = 0; mt < KSTEPS; ++mt) {
-          acc[mt][nt][e] *= alpha;
-          acc[mt][nt][2 + e] *= alpha;
+          acc[mt][nt][e] *= alpha_acc;
+          acc[mt][nt][2 + e] *= alpha_acc;
         }
       }
       // P^T as B fragments (tokens x heads) via an in-register 8x8 transpose
@@ -350,10 +357,16 @@ __device__ __forceinline__ void attn_core(const AttnArgs& a, int row, int split,
       const uint32_t h1 = pack_bf16x2(p[2], p[3]);
       const uint32_t l0 = pack_bf16x2(p[0] - bf16_bits_to_float(h0 & 0xFFFFu), p[1] - bf16_bits_to_float(h0 >> 16));
       const uint32_t l1 = pack_bf16x2(p[2] - bf16_bits_to_float(h1 & 0xFFFFu), p[3] - bf16_bits_to_float(h1 >> 16));
-      bhi[nt][0] = movmatrix_trans(h0);
-      bhi[nt][1] = movmatrix_trans(h1);
-      blo[nt][0] = movmatrix_trans(l0);
-      blo[nt][1] = movmatrix_trans(l1);
+      if (pack) {
+        const uint32_t x0 = __shfl_xor_sync(0xFFFFFFFFu, l0, 2), x1 = __shfl_xor_sync(0xFFFFFFFFu, l1, 2);
+        bhi[nt][0] = movmatrix_trans(c < 2 ? h0 : x0);
+        bhi[nt][1] = movmatrix_trans(c < 2 ? h1 : x1);
+      } else {
+        bhi[nt][0] = movmatrix_trans(h0);
+        bhi[nt][1] = movmatrix_trans(h1);
+        blo[nt][0] = movmatrix_trans(l0);
+        blo[nt][1] = movmatrix_trans(l1);
+      }
     }
     // ---- O^T += V_sub^T . P^T
     {
@@ -366,13 +379,19 @@ __device__ __forceinline__ void attn_core(const AttnArgs& a, int row, int split,
 #pragma unroll
         for (int nt = 0; nt < NTILE; ++nt) {
           mma_bf16_16816(acc[mt][nt], vf, bhi[nt][0], bhi[nt][1]);
-          mma_bf16_16816(acc[mt][nt], vf, blo[nt][0], blo[nt][1]);
+          if (!pack) mma_bf16_16816(acc[mt][nt], vf, blo[nt][0], blo[nt][1]);
         }
       }
     }
     __syncwarp();
   }
   cp_async_wait<0>();
+  if (pack) {  // the lo parts' accumulators (columns 4-7) onto the hi parts' (columns 0-3)
+#pragma unroll
+    for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][0][e] += __shfl_xor_sync(0xFFFFFFFFu, acc[mt][0][e], 2);
+  }
 
   // ---- merge the 4 warps' states in shared memory
 #pragma unroll

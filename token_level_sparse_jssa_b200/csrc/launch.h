@@ -207,15 +207,12 @@ struct VoteArgs {
 cudaError_t launch_vote_stats(const VoteArgs& a, cudaStream_t s);      // stats, then the votes
 cudaError_t launch_vote_broadcast(const VoteArgs& a, cudaStream_t s);
 
-// Split policy shared by the workspace sizing and the launch.
-void attn_split_policy(int mode, bool indexed, int rows, int64_t list_max, int num_sms, int d, int* S, int* split_len);
+// Split policy of the GQA attention, shared by the workspace sizing and the launch.
+void attn_split_policy(bool indexed, int rows, int64_t list_max, int num_sms, int d, int* S, int* split_len);
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);   // GQA path
-cudaError_t launch_mla_attention(const AttnArgs& a, cudaStream_t s);  // MLA path (indexed only)
 // MLA attention, indexed or dense, many tiles per CTA with the split merge in a cluster of S
 // CTAs per (sequence, head half); S from mla_split_groups, split_len = tokens per CTA.
 int mla_split_groups(int B, int num_sms);
 cudaError_t launch_mla_split(const AttnArgs& a, bool dense, cudaStream_t s);
-int mla_max_split();  // tokens per CTA of the MLA kernel
-cudaError_t launch_merge(const AttnArgs& a, cudaStream_t s);
 
 }  // namespace jssa
