@@ -149,6 +149,18 @@ JSSA_API jssa_status jssa_append_kv(const jssa_layout* L, const void* K_new, con
                                     const int32_t* t_pos, void* stream);
 
 /*
+ * Staging copy by a kernel instead of a copy engine, for the small per-step transfers of a
+ * decode loop (the query and the newest K/V rows in, the attention output out): copies
+ * `bytes` from src to dst, where each of dst and src is device memory or page-locked host
+ * memory that the device can address (cudaHostAlloc / pinned tensors under unified
+ * addressing).  Both pointers 16-byte aligned, bytes a multiple of 16; pageable host memory,
+ * misalignment or a null pointer return JSSA_ERR_INVALID_ARG without launching anything.
+ * Asynchronous on `stream` and ordered with the calls around it like any kernel; allocates
+ * nothing.  The kernel reads or writes host memory over the host link, 16 bytes per thread.
+ */
+JSSA_API jssa_status jssa_copy_mapped(void* dst, const void* src, size_t bytes, void* stream);
+
+/*
  * Projected scoring cache on write (§3.1, §3.4, §E.1):
  *   Kp[b, h, t, :] = rnd(K[b, h, t, :] . P_h)   for t in [t_begin[b], t_begin[b] + n_tokens)
  * with rnd = bf16 or E4M3 (saturating) rounding to nearest even, by kp_dtype.

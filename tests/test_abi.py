@@ -203,3 +203,14 @@ def test_voting_and_gather_entry_points_validate_on_the_host(lib):
     assert lib.jssa_vote_select(C.byref(L), None, *args[1:], C.c_float(0.1), FAKE, FAKE, ws, 1 << 30, None) == 1
     n = C.c_size_t(0)
     assert lib.jssa_gather_size(C.byref(L), 0, 0, C.byref(n)) == 1
+
+
+def test_staging_copy_validates_on_the_host(lib):
+    # null pointers, sizes that are not whole 16-byte words and misaligned pointers are
+    # rejected before any CUDA call; an empty copy is a no-op
+    assert lib.jssa_copy_mapped(None, FAKE, 16, None) == 1
+    assert lib.jssa_copy_mapped(FAKE, None, 16, None) == 1
+    assert lib.jssa_copy_mapped(FAKE, FAKE, 24, None) == 1
+    assert lib.jssa_copy_mapped(FAKE + 8, FAKE, 16, None) == 1
+    assert lib.jssa_copy_mapped(FAKE, FAKE + 4, 16, None) == 1
+    assert lib.jssa_copy_mapped(None, None, 0, None) == 0

@@ -277,6 +277,7 @@ def test_gather_then_attend_comparator_matches_oracle(name, kw, seq, k, window):
     ("tiny", {}, None, 0),
     ("h128k", dict(B=2, T=7000), [7000, 333], 0),
     ("hybrid", dict(B=2, T=5000), [5000, 800], 1024),    # local layer: dense over the window
+    ("h128k", dict(B=2, T=7000), [7000, 5000], 300),     # few splits per row: merged in a cluster
 ])
 def test_dense_decode_matches_oracle(name, kw, seq, window):
     w = W[name].with_(**kw)

@@ -11,6 +11,7 @@ fails loudly if it has not been built.
 from ._binding import (  # noqa: F401
     EXPORTS, KP_BF16, KP_FP8_E4M3, LIB_PATH, MODE_GQA, MODE_MLA, OUT_BF16, OUT_F32, JssaError, Layout,
     alloc_calibration_workspace, alloc_gather_buffer, alloc_workspace, append_kv, arm_withheld_copy, calibrate,
+    copy_mapped,
     decode_step, gather_decode,
     dense_decode, indexed_attn, load, make_layout, project_keys, read_device_status, score, select, status_string, topk,
     topk_noalloc, version, vote_select, workspace_init, workspace_size)

@@ -28,7 +28,8 @@ EXPORTS = ("jssa_status_string", "jssa_version", "jssa_workspace_size", "jssa_pr
            "jssa_topk", "jssa_topk_noalloc", "jssa_select", "jssa_indexed_attn", "jssa_decode_step",
            "jssa_dense_decode", "jssa_gather_size", "jssa_gather_decode", "jssa_calibrate_workspace_size",
            "jssa_calibrate", "jssa_vote_select",
-           "jssa_workspace_init", "jssa_read_device_status", "jssa_test_withhold_copy", "jssa_append_kv")
+           "jssa_workspace_init", "jssa_read_device_status", "jssa_test_withhold_copy", "jssa_append_kv",
+           "jssa_copy_mapped")
 
 
 class JssaError(RuntimeError):
@@ -79,6 +80,7 @@ def load(path: str = LIB_PATH):
         "jssa_read_device_status": (C.c_int, [vp, sz, C.POINTER(i32), vp]),
         "jssa_test_withhold_copy": (C.c_int, [vp, sz, i32, vp]),
         "jssa_append_kv": (C.c_int, [LP, vp, vp, vp, vp, vp, vp]),
+        "jssa_copy_mapped": (C.c_int, [vp, vp, C.c_size_t, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -172,6 +174,19 @@ def append_kv(L, K_new, V_new, K, V, t_pos, stream=None):
     """Write the newest K (and V) row of every (sequence, KV head) into row t_pos[b]."""
     _check("jssa_append_kv", load().jssa_append_kv(C.byref(L), _c(K_new), _c(V_new), _p(K), _p(V), _c(t_pos),
                                                    _stream(stream)))
+
+
+def copy_mapped(dst, src, nbytes=None, stream=None):
+    """Copy nbytes (default: all of src) between device memory and pinned host memory with a
+    kernel (jssa_copy_mapped); dst and src are contiguous tensors, either on the device or
+    pinned on the host."""
+    for t in (dst, src):
+        if not t.is_contiguous():
+            raise ValueError("contiguous tensors expected")
+    n = src.numel() * src.element_size() if nbytes is None else int(nbytes)
+    if n > min(src.numel() * src.element_size(), dst.numel() * dst.element_size()):
+        raise ValueError("nbytes exceeds a tensor")
+    _check("jssa_copy_mapped", load().jssa_copy_mapped(dst.data_ptr(), src.data_ptr(), n, _stream(stream)))
 
 
 def project_keys(L, K, P, Kp, n_tokens: int, t_begin=None, seq_lens=None, stream=None):

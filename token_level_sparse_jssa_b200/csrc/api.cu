@@ -430,6 +430,31 @@ jssa_status jssa_append_kv(const jssa_layout* L, const void* K_new, const void* 
   return cu(launch_append_rows(a, static_cast<cudaStream_t>(stream)));
 }
 
+// Address the current device dereferences for p: device (or managed) memory as is, page-locked
+// host memory through its mapping; nullptr for pageable host memory or an unknown pointer.
+static const void* device_view(const void* p) {
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  switch (at.type) {
+    case cudaMemoryTypeDevice:
+    case cudaMemoryTypeManaged:
+    case cudaMemoryTypeHost: return at.devicePointer;
+    default: return nullptr;
+  }
+}
+
+jssa_status jssa_copy_mapped(void* dst, const void* src, size_t bytes, void* stream) {
+  if (bytes == 0) return JSSA_OK;
+  if (!dst || !src || bytes % 16 != 0 || !aligned(dst, 16) || !aligned(src, 16)) return JSSA_ERR_INVALID_ARG;
+  void* d = const_cast<void*>(device_view(dst));
+  const void* sv = device_view(src);
+  if (!d || !sv || !aligned(d, 16) || !aligned(sv, 16)) return JSSA_ERR_INVALID_ARG;
+  return cu(launch_copy16(d, sv, bytes / 16, num_sms_current(), static_cast<cudaStream_t>(stream)));
+}
+
 jssa_status jssa_score(const jssa_layout* L, const void* Q, const float* P, const void* Kp, const int32_t* seq_lens,
                        int32_t window, float* scores, void* workspace, size_t ws_bytes, void* stream) {
   jssa_status st = check_layout(L);

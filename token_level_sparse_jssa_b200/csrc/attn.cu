@@ -23,10 +23,11 @@
 //                                                        most 4 heads both parts share one MMA,
 //                                                        the lo parts in columns 4-7)
 // The 4 groups' states are merged in shared memory into one normalised partial (o, lse)
-// per query head.  Indexed attention runs the S <= 8 splits of a row as one thread-block
-// cluster and combines the partials by log-sum-exp through distributed shared memory;
-// the dense decode, with many more splits, writes partials to the workspace and the last
-// CTA of each row to finish (a per-row arrival counter) combines them.
+// per query head.  Indexed attention, and the dense decode when it uses at most 8 splits (a
+// short window), runs the splits of a row as one thread-block cluster and combines the
+// partials by log-sum-exp through distributed shared memory; the dense decode with more
+// splits writes partials to the workspace and the last CTA of each row to finish (a per-row
+// arrival counter) combines them.
 #include "attn_core.cuh"
 
 namespace jssa {
@@ -89,7 +90,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS) attn_kernel(AttnArgs a) {
   float* pbuf = reinterpret_cast<float*>(smem_raw + Cfg::COMBINE_BYTES);   // [16][D] (cluster merge)
   float* plse = pbuf + 16 * D;                                              // [16]
   if (my_len == 0) {  // empty split: weight zero in the merge
-    if constexpr (!DENSE) {
+    if (!DENSE || a.cluster_merge) {
       for (int i = threadIdx.x; i < G * D; i += NT) pbuf[i] = 0.f;
       if (threadIdx.x < G) plse[threadIdx.x] = -INFINITY;
       cluster_merge<D>(a, hq0, G, pbuf, plse);
@@ -190,9 +191,13 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
   static int done[64] = {0};
   cudaError_t e = set_smem_limit_once(attn_kernel<D, NTILE, DENSE>, smem, done);
   if (e != cudaSuccess) return e;
-  // indexed: the S (<= 8) splits of a row form one cluster and merge through shared memory
+  // indexed, and dense with at most 8 splits: the S splits of a row form one cluster and
+  // merge through distributed shared memory; dense with more splits merges through the
+  // workspace (the row's last CTA to finish)
+  AttnArgs c = a;
+  c.cluster_merge = (!DENSE || a.S <= 8) ? 1 : 0;
   return launch_ex(attn_kernel<D, NTILE, DENSE>, dim3(a.S, a.B * a.Hkv), dim3(AttnCfg<D>::THREADS), smem, s,
-                   DENSE ? 0 : a.S, a);
+                   c.cluster_merge ? a.S : 0, c);
 }
 
 template <int D, bool DENSE>

@@ -202,8 +202,9 @@ __device__ __forceinline__ void load_q_frags(const void* Q, int64_t hq0, int G, 
 // range win_start + my_lo + [0, my_len) (dense).  The first AttnCfg<D>::WARPS warps stream and
 // multiply (qf holds the Q fragments of the warp's dims); every thread of the block must call
 // this (it holds block and cluster barriers).
-// Writes the split's partial through the cluster merge (indexed) or the workspace and the
-// row's last CTA (dense).  smem_raw: AttnCfg<D>::MAIN_BYTES of shared memory.
+// Writes the split's partial through the cluster merge (indexed, and dense launches of at
+// most 8 splits) or the workspace and the row's last CTA (dense with more splits).
+// smem_raw: AttnCfg<D>::MAIN_BYTES of shared memory.
 template <int D, int NTILE, bool DENSE>
 __device__ __forceinline__ void attn_core(const AttnArgs& a, int row, int split, int b, int h, int G, int64_t hq0,
                                           const uint32_t (&qf)[NTILE][AttnCfg<D>::DW / 16][2], const int32_t* tok_s,
@@ -218,6 +219,7 @@ __device__ __forceinline__ void attn_core(const AttnArgs& a, int row, int split,
   unsigned char* ring = smem_raw + (streams ? warp : 0) * STAGES * Cfg::STAGE_BYTES;
   float* pbuf = reinterpret_cast<float*>(smem_raw + Cfg::COMBINE_BYTES);   // [16][D] (cluster merge)
   float* plse = pbuf + 16 * D;                                              // [16]
+  const bool in_cluster = !DENSE || a.cluster_merge != 0;  // the row's splits merge over DSMEM
   const float scale_log2 = a.sm_scale * kLog2e;
   const bool pack = NTILE == 1 && G <= 4;  // hi and lo parts of P in one value MMA
   float m_run[NTILE][2], l_run[NTILE][2];
@@ -442,7 +444,7 @@ __device__ __forceinline__ void attn_core(const AttnArgs& a, int row, int split,
       o /= L;
       lse = (M + log2f(L)) * kLn2;
     }
-    if (!DENSE) {
+    if (in_cluster) {
       pbuf[i] = o;
       if (dim == 0) plse[head] = lse;
     } else {
@@ -450,7 +452,7 @@ __device__ __forceinline__ void attn_core(const AttnArgs& a, int row, int split,
       if (dim == 0) a.part_lse[(hq0 + head) * a.S + split] = lse;
     }
   }
-  if (!DENSE) {
+  if (in_cluster) {
     __syncthreads();
     cluster_merge<D>(a, hq0, G, pbuf, plse);
     return;

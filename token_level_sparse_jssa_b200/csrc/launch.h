@@ -36,6 +36,8 @@ struct AppendArgs {
   int64_t T_cap;
 };
 cudaError_t launch_append_rows(const AppendArgs& a, cudaStream_t s);
+// Copy of n16 16-byte words between device-addressable buffers (device or mapped pinned host).
+cudaError_t launch_copy16(void* dst, const void* src, size_t n16, int num_sms, cudaStream_t s);
 
 // Per-step prologue: projected group queries qs, plus the projection of the newest
 // n_new (<= 16) rows of each sequence into Kp.
@@ -116,6 +118,7 @@ struct AttnArgs {
   float* lse;        // nullable
   int out_bf16;
   int* status;
+  int cluster_merge;  // set by the launcher: the splits of a row form a cluster and merge over DSMEM
 };
 // Fused selection (query projection, newest-key projection, score scan, top-k) with one
 // 2-16 CTA cluster per (sequence, KV head); rows of up to select_max_candidates() tokens.

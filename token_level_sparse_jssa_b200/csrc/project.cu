@@ -135,6 +135,33 @@ cudaError_t launch_append_rows(const AppendArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// Staging copy of n16 16-byte words (device or device-addressable pinned host memory on
+// either side): grid-stride, all of a thread's loads issued before its stores.
+__global__ void __launch_bounds__(256) copy16_kernel(uint4* __restrict__ dst, const uint4* __restrict__ src,
+                                                     size_t n16) {
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n16; i += 4 * stride) {
+    const uint4 v0 = src[i], v1 = src[i + stride], v2 = src[i + 2 * stride], v3 = src[i + 3 * stride];
+    dst[i] = v0;
+    dst[i + stride] = v1;
+    dst[i + 2 * stride] = v2;
+    dst[i + 3 * stride] = v3;
+  }
+  for (; i < n16; i += stride) dst[i] = src[i];
+}
+
+cudaError_t launch_copy16(void* dst, const void* src, size_t n16, int num_sms, cudaStream_t s) {
+  if (n16 == 0) return cudaSuccess;
+  // one 256-thread block per 4 KB, at most 2 per SM: enough 16-byte requests in flight to
+  // cover the host link's latency for the few tens of KB a decode step moves
+  const size_t want = (n16 + 255) / 256;
+  const size_t cap = static_cast<size_t>(num_sms > 0 ? 2 * num_sms : 256);
+  const unsigned blocks = static_cast<unsigned>(want < cap ? want : cap);
+  copy16_kernel<<<blocks, 256, 0, s>>>(static_cast<uint4*>(dst), static_cast<const uint4*>(src), n16);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ step prologue
 constexpr int kPrologueThreads = 256;
 constexpr int kMaxNewRowsInPrologue = 16;
