@@ -317,12 +317,14 @@ __global__ void __launch_bounds__(kSpThreads, 1) mla_split_kernel(AttnArgs a) {
     // ---- O^T += V^T . P^T (hi and lo parts), accumulated over the CTA's tiles
     if (tid == 0) {
       tc_fence_after();
-      for (int j = 0; j < 4; ++j) {
-        for (int kt = 0; kt < N / 16; ++kt) {
-          const uint64_t adesc = smem_desc(c_s + (2 * j) * kSpBlkC + kt * 2048, kSpBlkC, 1024);
+      // the four dims blocks' accumulators take turns, so consecutive MMAs are independent
+      for (int kt = 0; kt < N / 16; ++kt) {
 #pragma unroll
-          for (int pl = 0; pl < 2; ++pl) {
-            const uint64_t bdesc = smem_desc(p_s + pl * kSpBlkP + kt * 2048, kSpBlkP, 1024);
+        for (int pl = 0; pl < 2; ++pl) {
+          const uint64_t bdesc = smem_desc(p_s + pl * kSpBlkP + kt * 2048, kSpBlkP, 1024);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t adesc = smem_desc(c_s + (2 * j) * kSpBlkC + kt * 2048, kSpBlkC, 1024);
             umma_bf16(tmem + kSpOCol + 64 * j, adesc, bdesc, idesc_v, (tile > 0 || kt > 0 || pl > 0) ? 1u : 0u);
           }
         }
