@@ -380,7 +380,7 @@ const char* jssa_status_string(jssa_status s) {
   return "unknown status";
 }
 
-int32_t jssa_version(void) { return 10100; }
+int32_t jssa_version(void) { return 10200; }
 
 jssa_status jssa_workspace_size(const jssa_layout* L, int32_t k, int32_t window, size_t* bytes) {
   jssa_status st = check_layout(L);

@@ -17,12 +17,14 @@
 // resident over the CTA's tiles.  The latent tile (128-byte swizzled, 147 KB) is the K-major A
 // operand of the score MMA and the MN-major A operand of the value MMA; the query streams
 // through a four-stage ring; P^T (bf16 hi + lo parts, rows = tokens) is the MN-major B
-// operand of the value MMA.  Every tile's rows of the next tile are prefetched into L2.
+// operand of the value MMA, whose MMAs take the four dims blocks' accumulators in turn.  The
+// next tile's cache rows are resolved, and prefetched into L2, while a tile runs.
 // Softmax over S^T: one thread per (token, 32 heads); the running maximum of a head moves only
 // when a tile brings a logit more than 2^8 above it (then the resident O^T columns and the
 // sums are rescaled), so most tiles need no reduction across threads.
-// After the last tile each CTA writes its normalised partial (o, lse) into shared memory and
-// the cluster merges the G partials of every output element over distributed shared memory.
+// After the last tile each CTA pushes its lse of every head to all CTAs of the cluster, writes
+// its normalised partial o into shared memory, and the cluster merges the G partials of every
+// output element over distributed shared memory with per-head weights formed once.
 // Every wait is bounded; on a timeout the kernel raises DEVFLAG_TIMEOUT, stops issuing, writes
 // an empty partial, drains its copies and MMAs, and frees its tensor memory.
 #include <cooperative_groups.h>
