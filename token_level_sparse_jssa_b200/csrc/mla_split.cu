@@ -18,7 +18,7 @@
 // operand of the score MMA and the MN-major A operand of the value MMA; the query streams
 // through a four-stage ring; P^T (bf16 hi + lo parts, rows = tokens) is the MN-major B
 // operand of the value MMA, whose MMAs take the four dims blocks' accumulators in turn.  The
-// next tile's cache rows are resolved, and prefetched into L2, while a tile runs.
+// next tile's cache rows are resolved, and prefetched into L2 line by line, while a tile runs.
 // Softmax over S^T: one thread per (token, 32 heads); the running maximum of a head moves only
 // when a tile brings a logit more than 2^8 above it (then the resident O^T columns and the
 // sums are rescaled), so most tiles need no reduction across threads.
@@ -71,9 +71,9 @@ __device__ __forceinline__ void sp_wait_groups(int kb) {
 __device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
-// Bring `bytes` (a multiple of 16, from a 16-byte aligned address) into L2.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+// Bring the 128-byte line at `p` into L2.
+__device__ __forceinline__ void prefetch_l2_line(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 template <bool DENSE>
@@ -210,7 +210,13 @@ __global__ void __launch_bounds__(kSpThreads, 1) mla_split_kernel(AttnArgs a) {
     // the next tile's rows: into tok_s (the other buffer, free since the previous tile) and L2
     if (tid < kSpTile && tile + 1 < ntiles) {
       tok_s[(tile + 1) & 1][tid] = next_row;
-      if (next_row >= 0) prefetch_l2_bulk(Cb + static_cast<int64_t>(next_row) * a.ks[2], kSpDk * 2);
+      // one head half prefetches each row, a line at a time (the plain prefetch is issued by the
+      // load unit; bulk prefetches of whole rows queue on the copy engine behind one another)
+      if (next_row >= 0 && (tid >> 6) == hh) {
+        const char* rp = reinterpret_cast<const char*>(Cb + static_cast<int64_t>(next_row) * a.ks[2]);
+#pragma unroll
+        for (int l = 0; l < kSpDk * 2 / 128; ++l) prefetch_l2_line(rp + l * 128);
+      }
     }
 
     // ---- S^T over the 9 K-blocks, the query ring refilled behind it
