@@ -196,6 +196,7 @@ def test_topk_with_few_distinct_values(T, k, levels):
     ("tiny", dict(T=1000, dk=64, dv=64, r=8), None, 100, 0, 0),
     ("h128k", dict(B=2, T=9000), [9000, 4000], 2048, 0, 0),
     ("h128k", dict(B=2, T=3000, Hq=16, Hkv=16), [3000, 2500], 300, 0, 0),     # G = 1
+    ("h128k", dict(B=2, T=3000, Hq=16, Hkv=8), [3000, 1700], 400, 0, 0),      # G = 2 (hi/lo parts in one MMA)
     ("h128k", dict(B=1, T=3000, Hq=32, Hkv=4), [3000], 500, 0, 0),           # G = 8
     ("h128k", dict(B=1, T=3000, Hq=32, Hkv=2), [3000], 257, 0, 0),           # G = 16
     ("hybrid", dict(B=2, T=6000), [6000, 1500], 1024, 1024, 0),              # d = 256 + window
@@ -388,6 +389,7 @@ def test_single_token_selection_returns_the_value_row():
     ("mla", dict(B=2, T=5000, k=512), [5000, 3210], 0),
     ("h128k", dict(B=1, Hq=8, Hkv=2, T=140000, k=1024), [140000], 0),   # rows beyond one cluster: unfused path
     ("h128k", dict(B=2, T=3000, Hq=16, Hkv=16, k=300), [3000, 2500], 0),   # G = 1
+    ("h128k", dict(B=2, T=3000, Hq=16, Hkv=8, k=400), [3000, 1700], 0),     # G = 2
     ("h128k", dict(B=1, T=3000, Hq=32, Hkv=2, k=257), [3000], 0),           # G = 16
     ("tiny", dict(T=1000, dk=64, dv=64, r=8, k=100), None, 0),               # d = 64
     ("h128k", dict(B=2, T=5000, k=512), [5000, 300], 700),                   # window; a row below k
